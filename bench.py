@@ -1,0 +1,456 @@
+#!/usr/bin/env python
+"""Benchmark of the MiniKV hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl minikv|reference]
+
+Default workload (the one the decode-bandwidth target is stated on): a
+Mistral-7B-shaped GQA decode -- 32 layers, 32 query heads over 8 KV heads,
+head size 128, batch 16, a 32768-token context of which 20% (6553 tokens) is
+kept and packed 2-bit (key group G=32, value group 128, fp16 residual R=128).
+A step is one generated token for the whole batch through all 32 layers: per
+layer one minikv_decode_attn call (append the new token, attend over the
+packed + residual cache, flush a key group to 2 bits every G steps).  The
+per-layer caches (2.5 GB per step) are walked in order, so the working set is
+far larger than the 126 MB L2.  The same run also times the prompt rows of
+the path on a LLaMA2-7B-shaped prefill (32 layers x 32 heads, 4096 tokens,
+W=32, keep 15%): minikv_select_prefill, minikv_topk_evict, minikv_quant_pack.
+
+Inputs are seeded synthetic N(0,1) fp16 with 4 outlier key channels x10 per
+KV head (no dataset, no weights).  Under torchrun every rank runs its own
+replica (weak scaling, no collective on the data path); the timed region is
+bracketed by barriers and the max over ranks is reported.
+"""
+from __future__ import annotations
+
+import argparse
+import concurrent.futures as cf
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "decode attn tokens/s and HBM GB/s (% of peak) over 2-bit KV; prefill select ms"
+
+DECODE = dict(workload="mistral7b_gqa_decode", layers=32, batch=16, q_heads=32, kv_heads=8, head_dim=128,
+              context=32768, keep_pct=20, G=32, Gv=128, R=128)
+PREFILL = dict(workload="llama2_7b_prefill_select", layers=32, batch=1, q_heads=32, kv_heads=32, head_dim=128,
+               prompt=4096, W=32, keep_pct=15, G=32, Gv=128, R=128)
+
+BYTES_PER_PACKED = 84     # per token and KV head at D=128, G=32, Gv=128: 64 code + 16 key + 4 value scale/zero
+BYTES_PER_RESIDUAL = 512  # fp16 K + V row
+
+
+def keep_of(T, pct):
+    return T * pct // 100
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return dict(hbm=float(p["hbm_gbs"]), bf16=float(p["bf16_tflops"]),
+                    bf16_sus=float(p["bf16_tflops_sustained"]), src="measured")
+    except Exception:
+        return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
+
+
+def recorded_traffic(kernel: str, source: str):
+    """dram bytes per launch from the committed ncu summary, if it was taken on
+    the current source of the kernel (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    try:
+        sha = hashlib.sha256(open(source, "rb").read()).hexdigest()[:16]
+        for line in open(path):
+            f = line.split()
+            if len(f) >= 4 and f[0] == kernel and f[1] == sha:
+                return float(f[2]), f[3]
+    except OSError:
+        pass
+    return None, None
+
+
+# ----------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """SM clock and clock-event reasons sampled by NVML while the timed region runs."""
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks",
+               0x10: "sync_boost", 0x1: "gpu_idle"}
+
+    def __init__(self, index: int, period_s: float = 0.01):
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+        self.period = period_s
+        self.samples, self.reasons = [], 0
+        self._stop = threading.Event()
+
+    def _reasons(self):
+        f = getattr(self.nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            self.nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        return f(self.h)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                self.reasons |= int(self._reasons())
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"], "samples": 0}
+        names = [n for bit, n in self.REASONS.items() if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz, "reasons": names,
+                "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------ CPU oracle
+
+def _oracle_unit(n_keep, g, seed):
+    import torch
+    from bit_quantized_evicted_b200 import synth
+    from oracle import minikv_oracle as O
+    k = synth.keys_fp16((n_keep, 128), synth.seed_of(77, seed, synth.T_K)).numpy()
+    v = synth.normal_fp16((n_keep, 128), synth.seed_of(77, seed, synth.T_V)).numpy()
+    cache = O.SliceCache.from_kept(k, v, DECODE["R"], DECODE["G"], DECODE["Gv"])
+    q = synth.normal_fp16((g, 128), synth.seed_of(77, seed, synth.T_QDEC)).numpy()
+    kn = synth.keys_fp16((128,), synth.seed_of(77, seed, synth.T_KNEW)).numpy()
+    vn = synth.normal_fp16((128,), synth.seed_of(77, seed, synth.T_VNEW)).numpy()
+    del torch
+    return cache, q, kn, vn
+
+
+def oracle_decode_rate(budget_s: float, threads: int):
+    """Unit-steps per second of the CPU oracle's decode step (one (sequence,
+    KV head) of one layer: append, attend over 6553 kept tokens with g = 4
+    query heads in fp64, flush when due), run on `threads` host threads."""
+    n_keep = keep_of(DECODE["context"], DECODE["keep_pct"])
+    g = DECODE["q_heads"] // DECODE["kv_heads"]
+    units = [_oracle_unit(n_keep, g, i) for i in range(threads)]
+    tau = 1.0 / math.sqrt(128.0)
+    counts = [0] * threads
+    deadline = time.perf_counter() + budget_s
+
+    def work(i):
+        c, q, kn, vn = units[i]
+        while time.perf_counter() < deadline:
+            c.step(q, kn, vn, tau)
+            counts[i] += 1
+
+    t0 = time.perf_counter()
+    with cf.ThreadPoolExecutor(threads) as ex:
+        list(ex.map(work, range(threads)))
+    dt = time.perf_counter() - t0
+    return sum(counts) / dt, sum(counts), dt
+
+
+def cpu_tokens_per_s(rate):
+    units_per_step = DECODE["layers"] * DECODE["batch"] * DECODE["kv_heads"]
+    return rate * DECODE["batch"] / units_per_step
+
+
+def decode_config(extra=None):
+    c = {k: v for k, v in DECODE.items()}
+    c["keep"] = keep_of(DECODE["context"], DECODE["keep_pct"])
+    c["l2"] = "inputs larger than L2: 32 distinct layer caches, 2.52 GB read per step"
+    if extra:
+        c.update(extra)
+    return c
+
+
+def run_reference(args):
+    """The oracle as the reference arm: rank 0 only, host cores."""
+    if int(os.environ.get("RANK", "0")) != 0:
+        return
+    threads = os.cpu_count() or 1
+    per_step = max(0.05, min(0.5, 120.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_decode_rate(per_step, threads)
+    rates, units = [], 0
+    for _ in range(args.steps):
+        r, n, _ = oracle_decode_rate(per_step, threads)
+        rates.append(r)
+        units += n
+    rate = statistics.median(rates)
+    v = cpu_tokens_per_s(rate)
+    sample = (f"{units} decode unit-steps (one sequence x KV head of one layer: 6553 kept tokens, 4 query heads, fp64) "
+              f"over {args.steps} steps of {per_step:.2f} s on {threads} threads; tokens/s = unit-steps/s x batch / "
+              f"(32 layers x 16 x 8 units)")
+    line = {"metric": METRIC, "value": v, "unit": "tokens/s", "impl": "reference", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * DECODE["batch"] / v,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": decode_config(),
+            "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": sample},
+            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------- GPU arm
+
+def make_decode_state(torch, mk, synth, device, warmup, steps):
+    L, B, Hq, Hkv = DECODE["layers"], DECODE["batch"], DECODE["q_heads"], DECODE["kv_heads"]
+    G, Gv, R = DECODE["G"], DECODE["Gv"], DECODE["R"]
+    N = keep_of(DECODE["context"], DECODE["keep_pct"])
+    total_steps = warmup + 2 * steps + 2
+    cap = ((N + total_steps) // G + 2) * G
+    ws = torch.zeros(mk.workspace_size(mk.OP_DECODE_ATTN, B, Hq, Hkv, cap + R + G), dtype=torch.uint8,
+                     device=device)
+    caches = []
+    for l in range(L):
+        k = torch.empty((B, Hkv, N, 128), dtype=torch.float16, device=device)
+        v = torch.empty_like(k)
+        for b in range(B):
+            k[b] = synth.keys_fp16((Hkv, N, 128), synth.seed_of(4, l, synth.T_K, 0, b), device)
+            v[b] = synth.normal_fp16((Hkv, N, 128), synth.seed_of(4, l, synth.T_V, 0, b), device)
+        c = mk.MiniKVCache(B, Hkv, cap, G=G, Gv=Gv, R=R, Hq=Hq, device=device, ws=ws)
+        mk.quant_pack(c, k, v)
+        caches.append(c)
+        del k, v
+    torch.cuda.synchronize()
+    # one pool of step inputs, laid out contiguously so that e2e copies are single transfers
+    P = 8
+    qin = torch.empty((P, L, B, Hq, 128), dtype=torch.float16, device=device)
+    knin = torch.empty((P, L, B, Hkv, 128), dtype=torch.float16, device=device)
+    vnin = torch.empty_like(knin)
+    for p in range(P):
+        for l in range(L):
+            qin[p, l] = synth.normal_fp16((B, Hq, 128), synth.seed_of(4, l, synth.T_QDEC, p), device)
+            knin[p, l] = synth.keys_fp16((B, Hkv, 128), synth.seed_of(4, l, synth.T_KNEW, p), device)
+            vnin[p, l] = synth.normal_fp16((B, Hkv, 128), synth.seed_of(4, l, synth.T_VNEW, p), device)
+    out = torch.empty((L, B, Hq, 128), dtype=torch.float16, device=device)
+    return caches, ws, qin, knin, vnin, out
+
+
+def unit_bytes(c):
+    return BYTES_PER_PACKED * c.n_packed + BYTES_PER_RESIDUAL * (c.n_res + 1)
+
+
+def run_prefill(torch, mk, synth, device):
+    """Prompt rows on the LLaMA2-7B shape: per layer select_prefill, topk_evict
+    and quant_pack, each timed with CUDA events (3 warm-up layers first)."""
+    L, B, H, T, W = PREFILL["layers"], PREFILL["batch"], PREFILL["q_heads"], PREFILL["prompt"], PREFILL["W"]
+    keep = keep_of(T, PREFILL["keep_pct"])
+    qs, ks, vs = [], [], []
+    for l in range(L):
+        qs.append(synth.normal_fp16((B, H, T, 128), synth.seed_of(2, l, synth.T_Q), device))
+        ks.append(synth.keys_fp16((B, H, T, 128), synth.seed_of(2, l, synth.T_K), device))
+        vs.append(synth.normal_fp16((B, H, T, 128), synth.seed_of(2, l, synth.T_V), device))
+    ws = torch.empty(mk.workspace_size(mk.OP_SELECT_PREFILL, B, H, H, T, 128, W), dtype=torch.uint8, device=device)
+    o = torch.empty_like(qs[0])
+    sc = torch.empty((B, H, T), dtype=torch.float32, device=device)
+    idx = torch.empty((B, H, keep), dtype=torch.int32, device=device)
+    kk = torch.empty((B, H, keep, 128), dtype=torch.float16, device=device)
+    vk = torch.empty_like(kk)
+    cache = mk.MiniKVCache(B, H, 640, G=PREFILL["G"], Gv=PREFILL["Gv"], R=PREFILL["R"], device=device)
+    for l in range(3):
+        mk.select_prefill(qs[l], ks[l], vs[l], W, o=o, scores=sc, ws=ws)
+        mk.topk_evict(sc, ks[l], vs[l], W, keep, idx=idx, k_kept=kk, v_kept=vk)
+        mk.quant_pack(cache, kk, vk)
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(L)]
+    for l in range(L):
+        e = ev[l]
+        e[0].record()
+        mk.select_prefill(qs[l], ks[l], vs[l], W, o=o, scores=sc, ws=ws)
+        e[1].record()
+        mk.topk_evict(sc, ks[l], vs[l], W, keep, idx=idx, k_kept=kk, v_kept=vk)
+        e[2].record()
+        mk.quant_pack(cache, kk, vk)
+        e[3].record()
+    torch.cuda.synchronize()
+    sel = sum(e[0].elapsed_time(e[1]) for e in ev)
+    top = sum(e[1].elapsed_time(e[2]) for e in ev)
+    pk = sum(e[2].elapsed_time(e[3]) for e in ev)
+    flops = L * (2.0 * T * T * 128 * H + 2.0 * W * T * 128 * H)    # causal QK^T + PV, plus the window pass
+    del qs, ks, vs
+    return {"workload": PREFILL["workload"], "config": {**PREFILL, "keep": keep},
+            "select_prefill_ms": sel, "select_prefill_ms_per_layer": sel / L,
+            "select_prefill_tflops": flops / (sel * 1e-3) / 1e12,
+            "topk_evict_ms": top, "quant_pack_ms": pk, "layers": L}
+
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    from bit_quantized_evicted_b200 import minikv as mk
+    from bit_quantized_evicted_b200 import synth
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=device)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    mk.lib()
+    pk = peaks()
+    L, B = DECODE["layers"], DECODE["batch"]
+    caches, ws, qin, knin, vnin, out = make_decode_state(torch, mk, synth, device, args.warmup, args.steps)
+    P = qin.shape[0]
+    stream = torch.cuda.current_stream(device)
+
+    def step(s, q_src, kn_src, vn_src, ev=None, nbytes=None):
+        p = s % P
+        for l in range(L):
+            if nbytes is not None:
+                nbytes.append(unit_bytes(caches[l]) * B * DECODE["kv_heads"])
+            if ev is not None:
+                ev[l][0].record(stream)
+            mk.decode_attn(caches[l], q_src[p, l], kn_src[p, l], vn_src[p, l], out=out[l], ws=ws)
+            if ev is not None:
+                ev[l][1].record(stream)
+
+    for s in range(args.warmup):
+        step(s, qin, knin, vnin)
+    torch.cuda.synchronize()
+
+    # ---- device-timed region
+    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(L)] for _ in range(args.steps)]
+    nbytes = []
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        t0.record(stream)
+        for s in range(args.steps):
+            step(args.warmup + s, qin, knin, vnin, ev=evs[s], nbytes=nbytes)
+        t1.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    ms = t0.elapsed_time(t1)
+    kern_ms = [evs[s][l][0].elapsed_time(evs[s][l][1]) for s in range(args.steps) for l in range(L)]
+    if world > 1:
+        t = torch.tensor([ms], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    tok_s = B * args.steps * world / (ms * 1e-3)
+    alg_bytes = sum(nbytes)
+    mean_launch_bytes = alg_bytes / len(nbytes)
+    mean_launch_s = statistics.mean(kern_ms) * 1e-3
+    achieved = mean_launch_bytes / mean_launch_s / 1e9
+    step_gbs = alg_bytes / (ms * 1e-3) / 1e9
+
+    # ---- end to end: inputs from pinned host memory, outputs back, each step
+    hq = qin.cpu().pin_memory()
+    hk = knin.cpu().pin_memory()
+    hv = vnin.cpu().pin_memory()
+    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    dq, dk, dv = torch.empty_like(qin[:1]), torch.empty_like(knin[:1]), torch.empty_like(vnin[:1])
+    h2d = (dq.numel() + dk.numel() + dv.numel()) * 2
+    d2h = out.numel() * 2
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for s in range(args.steps):
+        p = s % P
+        dq.copy_(hq[p:p + 1], non_blocking=True)
+        dk.copy_(hk[p:p + 1], non_blocking=True)
+        dv.copy_(hv[p:p + 1], non_blocking=True)
+        for l in range(L):
+            mk.decode_attn(caches[l], dq[0, l], dk[0, l], dv[0, l], out=out[l], ws=ws)
+        hout.copy_(out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_tok_s = B * args.steps * world / (e2e_ms * 1e-3)
+
+    prefill = run_prefill(torch, mk, synth, device) if not args.no_prefill else None
+    if prefill:
+        prefill["tensor_frac_of_bf16_peak"] = prefill["select_prefill_tflops"] / pk["bf16"]
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        threads = os.cpu_count() or 1
+        rate, n, dt = oracle_decode_rate(args.cpu_seconds, threads)
+        cpu = {"value": cpu_tokens_per_s(rate), "unit": "tokens/s", "cores": threads, "kind": "oracle",
+               "sample": f"{n} decode unit-steps (one sequence x KV head of one layer: 6553 kept tokens, 4 query "
+                         f"heads, fp64) in {dt:.1f} s on {threads} threads, scaled to 32 layers x 16 x 8 units "
+                         f"per step"}
+
+    traffic, traffic_note = recorded_traffic(
+        "decode_kernel", os.path.join(ROOT, "bit_quantized_evicted_b200", "csrc", "decode.cu"))
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": tok_s, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "u2+f16 (2-bit codes, fp16 scales/residual, fp32 accumulate)",
+            "data": "synthetic", "config": decode_config({"parallelism": f"replicas x{world}"}),
+            "hbm_gbs": step_gbs, "hbm_frac_of_peak": step_gbs / pk["hbm"],
+            "roofline": {"bound": "hbm", "kernel": "decode_kernel", "achieved": achieved, "peak": pk["hbm"],
+                         "unit": "GB/s", "frac": achieved / pk["hbm"], "traffic": traffic,
+                         "algorithmic_bytes_per_launch": mean_launch_bytes,
+                         "mean_launch_us": mean_launch_s * 1e6, "peak_source": pk["src"],
+                         "traffic_source": traffic_note},
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_tok_s, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": L * args.steps,
+            "clocks": clk.summary(),
+            "prefill": prefill,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=256)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="minikv", choices=["minikv", "reference"])
+    ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,191 @@
+// Shared device helpers of libminikv (sm_100a).
+#pragma once
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/minikv.h"
+
+namespace minikv {
+
+// Host-side error reporting (minikv_api.cu).  Returns `code`.
+int fail(int code, const char *fmt, ...);
+int check_launch(const char *what);
+
+constexpr int kD = 128;                  // the one supported head size
+constexpr float kLog2e = 1.4426950408889634f;
+
+__device__ __forceinline__ float h2f(uint16_t b) { return __half2float(__ushort_as_half(b)); }
+__device__ __forceinline__ uint16_t f2h(float f) { return __half_as_ushort(__float2half_rn(f)); }
+
+// Two floats -> half2 bits (lo in bits 0..15), round to nearest even.
+__device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;\n" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+__device__ __forceinline__ float2 unpack_half2(uint32_t x) {
+    __half2 h = *reinterpret_cast<__half2 *>(&x);
+    return __half22float2(h);
+}
+
+// D (16x8 fp32) += A (16x16 fp16, row) * B (16x8 fp16, col).
+// Fragment ownership, g = lane/4, t = lane%4:
+//   A: a[0]={(g,2t),(g,2t+1)} a[1]={(g+8,2t),(g+8,2t+1)} a[2]={(g,2t+8),(g,2t+9)} a[3]={(g+8,2t+8),(g+8,2t+9)}
+//   B: b[0]={(2t,g),(2t+1,g)} b[1]={(2t+8,g),(2t+9,g)}       (k, n)
+//   D: d[0]=(g,2t) d[1]=(g,2t+1) d[2]=(g+8,2t) d[3]=(g+8,2t+1)
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Transpose an 8x8 b16 matrix held one row-pair per thread: in, thread (g,t)
+// holds (row g, cols 2t..2t+1); out, it holds (row g, cols 2t..2t+1) of the transpose.
+__device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
+    uint32_t y;
+    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(y) : "r"(x));
+    return y;
+}
+
+__device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], uint32_t saddr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(saddr));
+}
+__device__ __forceinline__ void ldmatrix_x4_t(uint32_t (&r)[4], uint32_t saddr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(saddr));
+}
+
+__device__ __forceinline__ uint32_t smem_addr(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// 16-byte global->shared copy (Ampere-style cp.async), zero-filled when !pred.
+__device__ __forceinline__ void cp_async16(uint32_t saddr, const void *g, bool pred) {
+    int n = pred ? 16 : 0;
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(saddr), "l"(g), "r"(n));
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N)); }
+
+// ---- mbarrier + bulk (TMA, non-tensor) copies -------------------------------
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(smem_addr(bar)), "r"(count));
+}
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_addr(bar)), "r"(bytes)
+                 : "memory");
+}
+// Wait for phase `parity` of the barrier to complete.  Bounded: gives up after
+// ~`limit` polls and returns false, so a lost transfer can never hang the GPU.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint32_t limit = (1u << 26)) {
+    uint32_t addr = smem_addr(bar);
+    for (uint32_t i = 0; i < limit; ++i) {
+        uint32_t done;
+        asm volatile(
+            "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+            : "=r"(done) : "r"(addr), "r"(parity) : "memory");
+        if (done) return true;
+    }
+    return false;
+}
+// Bulk copy of `bytes` (multiple of 16, both addresses 16-byte aligned) from
+// global to this CTA's shared memory, completing on `bar`.
+__device__ __forceinline__ void bulk_g2s(void *sdst, const void *gsrc, uint32_t bytes, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(smem_addr(sdst)),
+        "l"(gsrc), "r"(bytes), "r"(smem_addr(bar))
+        : "memory");
+}
+
+// ---- the 2-bit quantizer (bit-exact: one IEEE fp32 op per step) -------------
+
+// scale = fp16_rn(fp32(mx - mn) / 3); mn/mx already canonical (+0 for zero).
+__device__ __forceinline__ uint16_t quant_scale(float mn, float mx) {
+    return f2h(__fdiv_rn(__fsub_rn(mx, mn), 3.0f));
+}
+// code = clamp(rint((x - zero) / scale), 0, 3), 0 when scale == 0.
+__device__ __forceinline__ uint32_t quant_code(float x, float zero, float scale) {
+    if (scale == 0.0f) return 0u;
+    float q = rintf(__fdiv_rn(__fsub_rn(x, zero), scale));
+    q = fminf(fmaxf(q, 0.0f), 3.0f);
+    return static_cast<uint32_t>(q);
+}
+// -0 and +0 are the same extreme; store +0.
+__device__ __forceinline__ float canon_zero(float x) { return __fadd_rn(x, 0.0f); }
+
+// Pack one key group: G tokens x 128 channels -> codes (token-major words),
+// one (scale, zero) per channel.  Called by all 128 threads of a CTA
+// (thread c = channel c).  row(t) returns a pointer to token t's 128 fp16.
+template <class RowFn>
+__device__ __forceinline__ void pack_key_group(RowFn row, int G, uint32_t *codes /* [G][8] */,
+                                               uint16_t *scale_out /* [128] */, uint16_t *zero_out) {
+    const int c = threadIdx.x;
+    float mn = INFINITY, mx = -INFINITY;
+    for (int t = 0; t < G; ++t) {
+        float x = h2f(row(t)[c]);
+        mn = fminf(mn, x);
+        mx = fmaxf(mx, x);
+    }
+    mn = canon_zero(mn);
+    mx = canon_zero(mx);
+    uint16_t sb = quant_scale(mn, mx);
+    float s = h2f(sb);
+    scale_out[c] = sb;
+    zero_out[c] = f2h(mn);
+    const int lane = c & 31;
+    for (int t = 0; t < G; ++t) {
+        uint32_t w = quant_code(h2f(row(t)[c]), mn, s) << (2 * (lane & 15));
+        w |= __shfl_xor_sync(0xffffffffu, w, 1);
+        w |= __shfl_xor_sync(0xffffffffu, w, 2);
+        w |= __shfl_xor_sync(0xffffffffu, w, 4);
+        w |= __shfl_xor_sync(0xffffffffu, w, 8);
+        if ((lane & 15) == 0) codes[t * 8 + (c >> 4)] = w;
+    }
+}
+
+// Pack value tokens: each of n tokens is quantized per block of Gv channels.
+// Called by all 128 threads (4 warps, one token per warp at a time; lane l
+// owns channels 4l..4l+3).  Gv in {16, 32, 64, 128}.
+template <class RowFn>
+__device__ __forceinline__ void pack_value_tokens(RowFn row, int n, int Gv, uint32_t *codes /* [n][8] */,
+                                                  uint16_t *scale_out /* [n][128/Gv] */, uint16_t *zero_out) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int lanes_per_block = Gv >> 2;
+    for (int t = warp; t < n; t += 4) {
+        const uint16_t *p = row(t) + 4 * lane;
+        uint2 raw = *reinterpret_cast<const uint2 *>(p);
+        float x[4] = {h2f(raw.x & 0xffff), h2f(raw.x >> 16), h2f(raw.y & 0xffff), h2f(raw.y >> 16)};
+        float mn = fminf(fminf(x[0], x[1]), fminf(x[2], x[3]));
+        float mx = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
+        for (int o = 1; o < lanes_per_block; o <<= 1) {
+            mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        }
+        mn = canon_zero(mn);
+        mx = canon_zero(mx);
+        uint16_t sb = quant_scale(mn, mx);
+        float s = h2f(sb);
+        if ((lane & (lanes_per_block - 1)) == 0) {
+            int blk = lane / lanes_per_block;
+            scale_out[t * (kD / Gv) + blk] = sb;
+            zero_out[t * (kD / Gv) + blk] = f2h(mn);
+        }
+        // lane l holds channels 4l..4l+3 -> bits 8*(l%4) .. of word l/4
+        uint32_t w = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) w |= quant_code(x[i], mn, s) << (2 * (4 * (lane & 3) + i));
+        w |= __shfl_xor_sync(0xffffffffu, w, 1);
+        w |= __shfl_xor_sync(0xffffffffu, w, 2);
+        if ((lane & 3) == 0) codes[t * 8 + (lane >> 2)] = w;
+    }
+}
+
+}  // namespace minikv

@@ -1,0 +1,89 @@
+// minikv_quant_pack: quantize a compacted kept sequence into the 2-bit cache.
+//
+// Source: gptget.net summary of arXiv 2411.18077, section 方法论 / 方法详解:
+// sub-channel (per-channel) key quantization and per-token value quantization
+// into a compact layout.  The newest r tokens stay fp16 in the residual ring.
+//
+// Grid (n_groups + n_res_blocks, B*Hkv), 128 threads.  Block x < n_groups packs
+// key group x (G tokens, thread = channel) and the same G value tokens (warp =
+// token); the remaining blocks copy residual tokens into ring slots 0..r-1.
+// Memory-bound: 512 B read and 84 B written per packed token and KV head.
+#include "common.cuh"
+
+namespace minikv {
+
+namespace {
+
+struct PackArgs {
+    const uint16_t *k, *v;
+    uint32_t *k_codes, *v_codes;
+    uint16_t *k_scale, *k_zero, *v_scale, *v_zero;
+    uint16_t *k_res, *v_res;
+    int N, n_q, r, G, Gv, cap, ring, n_groups;
+};
+
+constexpr int kResPerBlock = 32;   // residual tokens copied per block
+
+__global__ void __launch_bounds__(128) pack_kernel(const PackArgs a) {
+    const int unit = blockIdx.y;
+    const uint16_t *ku = a.k + (size_t)unit * a.N * kD;
+    const uint16_t *vu = a.v + (size_t)unit * a.N * kD;
+    if ((int)blockIdx.x < a.n_groups) {
+        const int grp = blockIdx.x;
+        const int t0 = grp * a.G;
+        auto krow = [&](int t) { return ku + (size_t)(t0 + t) * kD; };
+        auto vrow = [&](int t) { return vu + (size_t)(t0 + t) * kD; };
+        const size_t tok = (size_t)unit * a.cap + t0;
+        const size_t grow = (size_t)unit * (a.cap / a.G) + grp;
+        pack_key_group(krow, a.G, a.k_codes + tok * 8, a.k_scale + grow * kD, a.k_zero + grow * kD);
+        pack_value_tokens(vrow, a.G, a.Gv, a.v_codes + tok * 8, a.v_scale + tok * (kD / a.Gv),
+                          a.v_zero + tok * (kD / a.Gv));
+    } else {
+        const int i0 = ((int)blockIdx.x - a.n_groups) * kResPerBlock;
+        // 16 x 16-byte chunks per token row; 128 threads copy 8 rows per pass
+        for (int e = threadIdx.x; e < kResPerBlock * 16; e += 128) {
+            const int i = i0 + e / 16, ch = e % 16;
+            if (i >= a.r) break;
+            const size_t src = (size_t)(a.n_q + i) * kD;
+            const size_t dst = ((size_t)unit * a.ring + i) * kD;
+            reinterpret_cast<uint4 *>(a.k_res + dst)[ch] = reinterpret_cast<const uint4 *>(ku + src)[ch];
+            reinterpret_cast<uint4 *>(a.v_res + dst)[ch] = reinterpret_cast<const uint4 *>(vu + src)[ch];
+        }
+    }
+}
+
+}  // namespace
+
+int pack_launch(minikv_cache *c, const uint16_t *k, const uint16_t *v, int N, cudaStream_t stream) {
+    int n_q, r;
+    if (N >= c->R) {
+        r = c->R + (N - c->R) % c->G;
+        n_q = N - r;
+    } else {
+        r = N;
+        n_q = 0;
+    }
+    if (n_q > c->cap)
+        return fail(MINIKV_ERR_CAPACITY, "quant_pack: %d packed tokens exceed cap=%d", n_q, c->cap);
+    PackArgs a;
+    a.k = k; a.v = v;
+    a.k_codes = c->k_codes; a.v_codes = c->v_codes;
+    a.k_scale = c->k_scale; a.k_zero = c->k_zero; a.v_scale = c->v_scale; a.v_zero = c->v_zero;
+    a.k_res = c->k_res; a.v_res = c->v_res;
+    a.N = N; a.n_q = n_q; a.r = r; a.G = c->G; a.Gv = c->Gv; a.cap = c->cap; a.ring = c->R + c->G;
+    a.n_groups = n_q / c->G;
+    const int n_res_blocks = (r + kResPerBlock - 1) / kResPerBlock;
+    const int gx = a.n_groups + n_res_blocks;
+    const int units = c->B * c->Hkv;
+    if (gx > 0 && units > 0) {
+        pack_kernel<<<dim3(gx, units), 128, 0, stream>>>(a);
+        int rc = check_launch("quant_pack");
+        if (rc) return rc;
+    }
+    c->n_packed = n_q;
+    c->n_res = r;
+    c->res_start = 0;
+    return MINIKV_OK;
+}
+
+}  // namespace minikv

@@ -1,0 +1,192 @@
+/*
+ * minikv.h -- C ABI of libminikv.so: the MiniKV hot path on NVIDIA B200 (sm_100a).
+ *
+ * MiniKV ("MiniKV: Pushing the Limits of LLM Inference via 2-Bit
+ * Layer-Discriminative KV Cache") keeps, per layer, only the keys that earned
+ * the most attention from the last W prompt queries, stores them in 2 bits, and
+ * attends over that cache during decoding.  The pages that describe it give the
+ * ideas, not the formulas:
+ *   - abstract: a 2-bit, layer-discriminative KV cache, with CUDA kernels made
+ *     compatible with FlashAttention;
+ *   - gptget.net summary of arXiv 2411.18077, section 方法论 / 方法详解:
+ *     sub-channel (per-channel) key quantization, per-token value quantization,
+ *     a compact cache layout, and "selective flash attention" done by a second
+ *     kernel;
+ *   - same page, glossary 术语表 "adaptive KV": keep the KV states that matter;
+ *   - pre.notesum.ai LongBench table, "MiniKV Pyramid" rows: a keep budget that
+ *     differs by layer.
+ * The four calls below are this library's reading of those steps.
+ *
+ * Conventions for every call
+ *   - All tensor pointers are DEVICE pointers, owned by the caller.  The library
+ *     never allocates, frees or keeps them.  fp16 values are passed as uint16_t
+ *     bit patterns (IEEE binary16).  Tensors are contiguous, row-major.
+ *   - Work is queued on `stream` (a cudaStream_t; NULL = legacy default stream)
+ *     and runs asynchronously.  No call synchronizes the device.
+ *   - Return value: MINIKV_OK (0) or a negative MINIKV_ERR_* code.  On error
+ *     nothing was queued, the cache descriptor is unchanged, and
+ *     minikv_last_error_string() (per host thread) says why.  A device fault, if
+ *     any, surfaces at the caller's next synchronization; kernels never trap.
+ *   - Head size D must be 128.  Query head h reads KV head h / (Hq / Hkv)
+ *     (grouped-query attention with contiguous groups).
+ */
+#ifndef MINIKV_H
+#define MINIKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MINIKV_API __attribute__((visibility("default")))
+#else
+#define MINIKV_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MINIKV_OK                0
+#define MINIKV_ERR_INVALID_ARG  -1  /* null pointer, bad shape, W > keep, ... */
+#define MINIKV_ERR_UNSUPPORTED  -2  /* D != 128, G not a multiple of 32, ...  */
+#define MINIKV_ERR_CAPACITY     -3  /* the packed cache would exceed `cap`     */
+#define MINIKV_ERR_CUDA         -4  /* a CUDA launch or attribute call failed  */
+
+/*
+ * Packed 2-bit cache of ONE layer, for B sequences x Hkv KV heads.
+ * Device arrays (caller-allocated; minikv_cache_bytes/minikv_cache_bind carve
+ * them from one buffer):
+ *   k_codes, v_codes [B, Hkv, cap, D/16] uint32: packed token t holds 16 codes
+ *       per word; code of channel 16w+i sits in bits 2i..2i+1 of word w.
+ *   k_scale, k_zero  [B, Hkv, cap/G, D] fp16: one (scale, zero) per key channel
+ *       per group of G consecutive packed tokens (groups start at token 0).
+ *   v_scale, v_zero  [B, Hkv, cap, D/Gv] fp16: one (scale, zero) per token per
+ *       block of Gv consecutive value channels.
+ *   k_res, v_res     [B, Hkv, R+G, D] fp16: ring of the newest tokens, kept in
+ *       fp16; logical residual token i (0 = oldest) is in slot
+ *       (res_start + i) mod (R+G).
+ * Host-side state (same for every sequence and head of the layer): n_packed
+ * packed tokens (a multiple of G), n_res residual tokens, ring origin
+ * res_start.  Calls update it synchronously when they queue their work.
+ * Dequantized value of a code c: c * scale + zero.
+ */
+typedef struct minikv_cache {
+    int B, Hkv, D, G, Gv, R, cap;
+    uint32_t *k_codes, *v_codes;
+    uint16_t *k_scale, *k_zero;
+    uint16_t *v_scale, *v_zero;
+    uint16_t *k_res, *v_res;
+    int n_packed, n_res, res_start;
+} minikv_cache;
+
+/* Bytes of device memory one layer's cache needs (each array 256-byte aligned),
+ * or 0 if the shape is invalid. */
+MINIKV_API size_t minikv_cache_bytes(int B, int Hkv, int D, int G, int Gv, int R, int cap);
+
+/* Fill *c with the shape, point its arrays into `base` (a device buffer of at
+ * least minikv_cache_bytes(...) bytes, 256-byte aligned) and reset the state to
+ * empty.  Touches no device memory. */
+MINIKV_API int minikv_cache_bind(minikv_cache *c, void *base, size_t bytes,
+                      int B, int Hkv, int D, int G, int Gv, int R, int cap);
+
+/*
+ * minikv_quant_pack -- load a fresh compacted sequence into the cache.
+ * Source: summary page, 方法论 (sub-channel key quantization, per-token value
+ * quantization, compact layout); the fp16 residual of the newest tokens.
+ *   k, v      [B, Hkv, n_tokens, D] fp16, the kept tokens in position order.
+ * Split: with N = n_tokens, the newest r tokens stay fp16, r = R + (N-R) mod G
+ * if N >= R, else r = N; the oldest N - r (a multiple of G) are quantized:
+ *   keys  : per channel over each group of G tokens; values: per token over
+ *           each block of Gv channels;
+ *   mn = min x, mx = max x (a zero extreme counts as +0);
+ *   scale = fp16_rn(fp32(mx - mn) / 3), zero = mn;
+ *   code = 0 if scale == 0, else clamp(rint((x - zero) / scale), 0, 3) in fp32
+ *   (IEEE round-to-nearest-even at every step).
+ * The cache state becomes n_packed = N - r, n_res = r, res_start = 0.
+ * Errors: INVALID_ARG (null, n_tokens < 0), CAPACITY (N - r > cap),
+ * UNSUPPORTED (shape).
+ */
+MINIKV_API int minikv_quant_pack(minikv_cache *c, const uint16_t *k, const uint16_t *v,
+                      int n_tokens, void *stream);
+
+/*
+ * minikv_select_prefill -- "selective flash attention" over the prompt.
+ * Source: summary page, 方法详解, third bullet (selective flash attention by a
+ * second kernel); abstract (FlashAttention compatibility).
+ *   q [B, Hq, T, D], k, v [B, Hkv, T, D] fp16.
+ *   o [B, Hq, T, D] fp16: o_i = sum_{j<=i} softmax_j(sm_scale * q_i.k_j) v_j.
+ *   scores [B, Hkv, T] fp32: scores[j] = sum over the Hq/Hkv query heads of the
+ *       KV head and over the last W rows i in [T-W, T) of the softmax
+ *       probability P[i, j] (0 where j > i).
+ * Pass 1 is a causal flash-attention forward that also records the row
+ * log-sum-exp of the window rows in `ws`; pass 2 (the second kernel) recomputes
+ * the window rows' probabilities from it and sums them per key.
+ *   ws: device scratch of minikv_workspace_size(MINIKV_OP_SELECT_PREFILL, ...)
+ *       bytes, no initial contents required.
+ * Errors: INVALID_ARG (null, W < 1, W > T, Hq % Hkv, ws too small),
+ * UNSUPPORTED (D != 128).
+ */
+MINIKV_API int minikv_select_prefill(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                          int B, int Hq, int Hkv, int T, int D, int W, float sm_scale,
+                          uint16_t *o, float *scores, void *ws, size_t ws_bytes,
+                          void *stream);
+
+/*
+ * minikv_topk_evict -- adaptive KV: keep the tokens that matter.
+ * Source: summary page, glossary 术语表 "adaptive KV" (keep KV states by
+ * importance); notesum LongBench table, "MiniKV Pyramid" (the caller picks
+ * `keep` per layer).
+ *   scores [B, Hkv, T] fp32 (from minikv_select_prefill); k, v [B, Hkv, T, D].
+ *   If keep >= T every position is kept (n = T).  Otherwise (W <= keep) the
+ *   window [T-W, T) is kept, plus the keep-W positions j < T-W with the highest
+ *   scores; equal scores go to the lower index.  n = min(keep, T).
+ *   idx [B, Hkv, n] int32: kept positions, ascending.
+ *   k_kept, v_kept [B, Hkv, n, D] fp16: rows k[idx], v[idx] (exact copies).
+ *   ws: minikv_workspace_size(MINIKV_OP_TOPK_EVICT, ...) bytes (may be 0).
+ * Errors: INVALID_ARG (null, keep < 1, W > keep < T).
+ */
+MINIKV_API int minikv_topk_evict(const float *scores, const uint16_t *k, const uint16_t *v,
+                      int B, int Hkv, int T, int D, int W, int keep,
+                      int32_t *idx, uint16_t *k_kept, uint16_t *v_kept,
+                      void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * minikv_decode_attn -- one decoding step of one layer over the 2-bit cache.
+ * Source: abstract ("specialized CUDA kernels ... compatible with
+ * FlashAttention"); summary page, 方法论 (the compact 2-bit layout it reads).
+ *   q [B, Hq, D] fp16; k_new, v_new [B, Hkv, D] fp16 (this step's token).
+ *   out [B, Hq, D] fp16.
+ * 1. Append (k_new, v_new) as the newest residual token.
+ * 2. out_h = sum_t softmax_t(sm_scale * q_h . kappa_t) nu_t over all packed
+ *    tokens (dequantized in registers) and all residual tokens, new one
+ *    included.  Flash-decoding: the tokens are split across CTAs and the
+ *    partial softmax states are merged by the last CTA of each KV head.
+ * 3. If the residual now holds R+G tokens, its oldest G are quantized (same
+ *    rules as minikv_quant_pack) into key group n_packed/G: n_packed += G,
+ *    n_res -= G.
+ *   ws: minikv_workspace_size(MINIKV_OP_DECODE_ATTN, B, Hq, Hkv, cap, D, 0)
+ *       bytes, ZERO-FILLED before its first use; every call leaves it ready for
+ *       the next (its arrival counters return to zero).  Calls that share one
+ *       ws must not overlap on the GPU.
+ * Errors: INVALID_ARG (null, Hq % Hkv, ws too small), CAPACITY (a flush would
+ * exceed cap), UNSUPPORTED (D != 128, Gv != D, G not a multiple of 32).
+ */
+MINIKV_API int minikv_decode_attn(minikv_cache *c, const uint16_t *q, const uint16_t *k_new,
+                       const uint16_t *v_new, int Hq, float sm_scale, uint16_t *out,
+                       void *ws, size_t ws_bytes, void *stream);
+
+#define MINIKV_OP_SELECT_PREFILL 1
+#define MINIKV_OP_TOPK_EVICT     2
+#define MINIKV_OP_DECODE_ATTN    3
+
+/* Scratch bytes an op needs.  For MINIKV_OP_DECODE_ATTN pass the cache
+ * capacity plus R+G as T (the most tokens a step can attend to). */
+MINIKV_API size_t minikv_workspace_size(int op, int B, int Hq, int Hkv, int T, int D, int W);
+
+/* Why the last failing call on this host thread failed ("" if none). */
+MINIKV_API const char *minikv_last_error_string(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MINIKV_H */
