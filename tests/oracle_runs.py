@@ -38,8 +38,8 @@ def compare_cache(cache, ref, check_residual=True):
             np.testing.assert_array_equal(a["v_scale"][b, h, :nq].view(np.uint16), s.v_scale)
             np.testing.assert_array_equal(a["v_zero"][b, h, :nq].view(np.uint16), s.v_zero)
             if check_residual:
-                np.testing.assert_array_equal(kr[b, h].view(np.uint16), np.array(s.res_k, np.uint16).reshape(s.r, -1))
-                np.testing.assert_array_equal(vr[b, h].view(np.uint16), np.array(s.res_v, np.uint16).reshape(s.r, -1))
+                np.testing.assert_array_equal(kr[b, h].view(np.uint16), np.array(s.res_k, np.uint16).reshape(s.r, s.D))
+                np.testing.assert_array_equal(vr[b, h].view(np.uint16), np.array(s.res_v, np.uint16).reshape(s.r, s.D))
 
 
 def decode_reference_step(ref, q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor, tau: float) -> np.ndarray:

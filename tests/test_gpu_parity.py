@@ -201,6 +201,6 @@ def test_pipeline_tiny_layer_end_to_end():
         assert all(abs(sref[0, h, j] - cut) < 1e-4 for j in diff), (h, diff)
     # downstream stages take the GPU's kept set as their input
     ref = pack_reference(kk, vk, R, G, Gv)
-    compare_cache(cache, ref)
     oref = decode_reference_step(ref, qd, kn, vn, TAU)
+    compare_cache(cache, ref)
     assert float(np.max(np.abs(out.float().cpu().numpy() - oref))) <= ATOL_OUT
