@@ -14,7 +14,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libminikv.so")
-SOURCES = ["minikv_api.cu", "pack.cu", "prefill.cu", "topk.cu", "decode.cu"]
+SOURCES = ["minikv_api.cu", "pack.cu", "prefill.cu", "topk.cu", "decode.cu", "decode_static.cu"]
 HEADERS = ["common.cuh"]
 NVCC = os.environ.get("NVCC", "nvcc")
 FLAGS = [

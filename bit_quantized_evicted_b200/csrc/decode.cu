@@ -519,6 +519,17 @@ size_t decode_workspace_bytes(int B, int Hkv, int max_tokens) {
     return ((units * 4 + 255) / 256) * 256 + units * S * 4 * kPartStride * 4;
 }
 
+// Bytes of the workspace prefix that holds the per-unit arrival counters.
+size_t decode_counter_bytes(int B, int Hkv) { return (((size_t)B * Hkv * 4 + 255) / 256) * 256; }
+
+// Workspace bytes the next decode call on this cache state will use.
+size_t decode_call_workspace_bytes(const minikv_cache *c) {
+    const int units = c->B * c->Hkv;
+    int n_chunks, chunk;
+    plan_chunks(units, c->n_packed, n_chunks, chunk);
+    return decode_counter_bytes(c->B, c->Hkv) + (size_t)units * (1 + n_chunks) * 4 * kPartStride * 4;
+}
+
 int decode_launch(minikv_cache *c, const uint16_t *q, const uint16_t *k_new, const uint16_t *v_new, int Hq,
                   float sm_scale, uint16_t *out, void *ws, size_t ws_bytes, cudaStream_t stream) {
     const int units = c->B * c->Hkv;

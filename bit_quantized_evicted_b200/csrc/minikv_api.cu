@@ -64,6 +64,25 @@ static int check_cache(const minikv_cache *c) {
     return MINIKV_OK;
 }
 
+// The argument checks of minikv_decode_attn other than the workspace, for
+// entry points that bring their own scratch.
+int decode_validate(minikv_cache *c, const uint16_t *q, const uint16_t *k_new, const uint16_t *v_new, int Hq,
+                    const uint16_t *out) {
+    g_err[0] = 0;
+    int rc = check_cache(c);
+    if (rc) return rc;
+    if (!q || !k_new || !v_new || !out) return fail(MINIKV_ERR_INVALID_ARG, "decode_attn: null pointer");
+    if (!aligned16(q) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(out))
+        return fail(MINIKV_ERR_INVALID_ARG, "decode_attn: pointers must be 16-byte aligned");
+    if (Hq < 1 || Hq % c->Hkv) return fail(MINIKV_ERR_INVALID_ARG, "decode_attn: Hq=%d, Hkv=%d", Hq, c->Hkv);
+    if (Hq / c->Hkv > 4) return fail(MINIKV_ERR_UNSUPPORTED, "decode_attn: more than 4 query heads per KV head");
+    if (c->Gv != c->D) return fail(MINIKV_ERR_UNSUPPORTED, "decode_attn: value group Gv=%d (needs Gv = D)", c->Gv);
+    if ((size_t)c->B * c->Hkv > 65535) return fail(MINIKV_ERR_UNSUPPORTED, "decode_attn: B*Hkv above 65535");
+    if (c->n_res + 1 == c->R + c->G && c->n_packed + c->G > c->cap)
+        return fail(MINIKV_ERR_CAPACITY, "decode_attn: flushing a key group would exceed cap=%d", c->cap);
+    return MINIKV_OK;
+}
+
 }  // namespace minikv
 
 using namespace minikv;

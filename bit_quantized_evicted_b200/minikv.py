@@ -42,6 +42,7 @@ _SIGS = {
     "minikv_select_prefill": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P, _Z, _P]),
     "minikv_topk_evict": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _Z, _P]),
     "minikv_decode_attn": (_I, [ctypes.POINTER(CacheStruct), _P, _P, _P, _I, _F, _P, _P, _Z, _P]),
+    "minikv_decode_attn_static": (_I, [ctypes.POINTER(CacheStruct), _P, _P, _P, _I, _F, _P, _P]),
     "minikv_workspace_size": (_Z, [_I, _I, _I, _I, _I, _I, _I]),
     "minikv_last_error_string": (ctypes.c_char_p, []),
 }
@@ -228,4 +229,22 @@ def decode_attn(cache: MiniKVCache, q: torch.Tensor, k_new: torch.Tensor, v_new:
         ctypes.byref(cache.c), _dev(q, torch.float16, "q"), _dev(k_new, torch.float16, "k_new"),
         _dev(v_new, torch.float16, "v_new"), Hq, float(sm_scale), _dev(out, torch.float16, "out"),
         _dev(ws, torch.uint8, "ws"), ws.numel(), _stream(stream, q.device)))
+    return out
+
+
+def decode_attn_static(cache: MiniKVCache, q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor,
+                       sm_scale: float | None = None, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """decode_attn for callers that may not allocate device memory: the split
+    partials live in the library's own fixed 8 MiB device array instead of a
+    workspace (no cudaMalloc anywhere in the call).  Calls whose GPU work
+    overlaps share that array and race on it."""
+    B, Hq, D = q.shape
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty_like(q)
+    _check(lib().minikv_decode_attn_static(
+        ctypes.byref(cache.c), _dev(q, torch.float16, "q"), _dev(k_new, torch.float16, "k_new"),
+        _dev(v_new, torch.float16, "v_new"), Hq, float(sm_scale), _dev(out, torch.float16, "out"),
+        _stream(stream, q.device)))
     return out

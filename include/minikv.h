@@ -175,6 +175,28 @@ MINIKV_API int minikv_decode_attn(minikv_cache *c, const uint16_t *q, const uint
                        const uint16_t *v_new, int Hq, float sm_scale, uint16_t *out,
                        void *ws, size_t ws_bytes, void *stream);
 
+/*
+ * minikv_decode_attn_static -- minikv_decode_attn without a caller workspace.
+ * The paper has no counterpart to this call; it exists for callers that may
+ * not allocate device memory: hosts whose device memory is entirely planned by
+ * their own allocator or pool (a cudaMalloc behind its back would break its
+ * accounting and budget) and latency-critical loops where cudaMalloc is not
+ * allowed because it can synchronize the device.
+ * Same arguments, semantics, results and errors as minikv_decode_attn, minus
+ * `ws`: the scratch is a fixed 8 MiB array inside the library's device module,
+ * held by every GPU that loads the library until the process exits.  A step
+ * whose scratch need is larger fails with MINIKV_ERR_UNSUPPORTED and queues
+ * nothing; minikv_decode_attn with a caller workspace has no such limit.
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress, that device current); make it before any stream
+ * capture.  All calls share the array: calls whose GPU work overlaps race on
+ * it.  Each call clears the array's arrival counters on `stream` first.  No
+ * call allocates or frees device memory.
+ */
+MINIKV_API int minikv_decode_attn_static(minikv_cache *c, const uint16_t *q, const uint16_t *k_new,
+                                         const uint16_t *v_new, int Hq, float sm_scale, uint16_t *out,
+                                         void *stream);
+
 #define MINIKV_OP_SELECT_PREFILL 1
 #define MINIKV_OP_TOPK_EVICT     2
 #define MINIKV_OP_DECODE_ATTN    3

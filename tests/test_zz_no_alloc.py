@@ -1,0 +1,62 @@
+"""minikv_decode_attn_static: the decode step for callers that may not
+allocate device memory (hosts whose device memory is all planned by their own
+allocator, latency-critical loops where cudaMalloc may synchronize the
+device).  It takes its scratch from a fixed array inside the library instead
+of a caller workspace; its results must match minikv_decode_attn.
+
+This file is named so that pytest collects it last.
+"""
+import ctypes
+import math
+
+import pytest
+import torch
+
+from bit_quantized_evicted_b200 import minikv as mk
+from bit_quantized_evicted_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+ATOL_OUT = 2e-3     # the attention-output tolerance of the parity tests
+
+
+@pytest.mark.gpu
+def test_static_scratch_decode_matches_workspace_decode_twice():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    dev = "cuda"
+    B, Hq, Hkv, N, R, G = 2, 8, 2, 1000, 128, 32
+    k = synth.keys_fp16((B, Hkv, N, 128), synth.seed_of(31, 0, synth.T_K), dev)
+    v = synth.normal_fp16((B, Hkv, N, 128), synth.seed_of(31, 0, synth.T_V), dev)
+    cap = ((N + 8) // G + 2) * G
+    with_ws = mk.MiniKVCache(B, Hkv, cap, R=R, G=G, Hq=Hq, device=dev)
+    no_alloc = mk.MiniKVCache(B, Hkv, cap, R=R, G=G, Hq=Hq, device=dev)
+    mk.quant_pack(with_ws, k, v)
+    mk.quant_pack(no_alloc, k, v)
+    for step in range(2):            # two calls in a row share the static scratch
+        q = synth.normal_fp16((B, Hq, 128), synth.seed_of(31, 0, synth.T_QDEC, step), dev)
+        kn = synth.keys_fp16((B, Hkv, 128), synth.seed_of(31, 0, synth.T_KNEW, step), dev)
+        vn = synth.normal_fp16((B, Hkv, 128), synth.seed_of(31, 0, synth.T_VNEW, step), dev)
+        ref = mk.decode_attn(with_ws, q, kn, vn)
+        got = mk.decode_attn_static(no_alloc, q, kn, vn)
+        torch.cuda.synchronize()
+        err = float((got.float() - ref.float()).abs().max())
+        assert err <= ATOL_OUT, (step, err)
+        assert (no_alloc.n_packed, no_alloc.n_res) == (with_ws.n_packed, with_ws.n_res)
+
+
+@pytest.mark.gpu
+def test_static_scratch_rejects_a_step_above_its_size():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    L = mk.lib()
+    c = mk.CacheStruct()
+    B, Hkv, cap = 512, 8, 64
+    n = L.minikv_cache_bytes(B, Hkv, 128, 32, 128, 32, cap)
+    assert L.minikv_cache_bind(ctypes.byref(c), 1 << 24, n, B, Hkv, 128, 32, 128, 32, cap) == 0
+    c.n_packed, c.n_res = 64, 32     # 4096 (sequence, KV head) units x 2 splits: above 8 MiB
+    p = 1 << 30
+    rc = L.minikv_decode_attn_static(ctypes.byref(c), p, p, p, 2 * Hkv, 1.0 / math.sqrt(128), p, None)
+    assert rc == mk.ERR_UNSUPPORTED
+    assert b"static buffer" in L.minikv_last_error_string()
+    assert (c.n_packed, c.n_res) == (64, 32)
