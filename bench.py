@@ -443,7 +443,10 @@ def main():
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--layers", type=int, default=DECODE["layers"],
+                    help="decode layers (fewer only for small profiling runs; the workload has 32)")
     args = ap.parse_args()
+    DECODE["layers"] = args.layers
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     if args.impl == "reference":

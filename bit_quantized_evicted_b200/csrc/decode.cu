@@ -4,27 +4,34 @@
 // FlashAttention) and the gptget.net summary of arXiv 2411.18077, section
 // 方法论 (sub-channel key / per-token value 2-bit quantization, compact layout).
 //
-// One launch per layer-step.  CTA (x = 0, unit) attends over the fp16 residual
-// (and appends the new token, and flushes a full key group); CTAs (x >= 1,
-// unit) each attend over one contiguous chunk of packed tokens.  Each CTA
-// writes its partial softmax state (m, l, sum p*v) to the workspace; the last
-// CTA of a unit (atomic arrival counter, self-resetting) merges them.
+// One launch per layer-step, one CTA of 4 warps per work item:
+//   * residual CTAs, n_rc per (sequence, KV head) "unit": 64-token chunks of the
+//     fp16 residual ring, staged by cp.async into swizzled shared memory; the
+//     chunk holding the new token appends it to the ring, chunk 0 packs the
+//     oldest G tokens to 2 bits when the residual is full (same code as
+//     minikv_quant_pack);
+//   * packed CTAs, sized to fill the GPU once: the packed tokens of all units,
+//     cut into 32-token slices, are laid end to end and split evenly into P
+//     contiguous ranges (one per CTA).  Each warp owns a 4-stage TMA-bulk
+//     pipeline (cp.async.bulk + mbarrier) over its slices of the range.
+// Every CTA writes one partial softmax state (m, l, sum p*v) per unit it
+// touched; the last CTA to arrive at a unit (self-resetting atomic counter)
+// merges them into `out`.
 //
-// Packed chunk, per warp and 32-token slice (one key group), heads of one KV
-// head taken four at a time (g <= 4):
-//   scores  S[token, col] = sum_c a[token, c] * b[c, col]          (mma m16n8k16)
-//     a = 1 + code * 2^(p-10): the 2-bit code dropped into an fp16 mantissa at
-//         bit p (6 or 8) by one AND/OR -- no integer->float conversion;
-//     b = q * k_scale * 2^(10-p), split hi + lo in fp16: cols 0..3 carry the hi
-//         parts of heads 0..3, cols 4..7 the lo parts, so one mma gives a
-//         22-bit-accurate product for four heads;
-//     score_h = S[., h] + S[., h+4] - sum_c b_c + sum_c q_c * k_zero_c.
-//   output  O^T[channel, col] = sum_t a'[channel, t] * P'[t, col]    (mma)
-//     a' = the value code in the same mantissa form; P' = p_t * v_scale_t split
-//     hi/lo the same way, moved from the score fragment layout into the B
-//     operand layout with movmatrix; out = (O^T - sum P') * 2^(10-p) + sum p*v_zero.
-// The token order inside a 16-token m-tile is permuted (kPerm) so that both
-// the key-word loads and the value-word loads of a warp hit 32 distinct banks.
+// Slice math (per warp, 32 tokens = 2 m-tiles of 16, g <= 4 query heads):
+//   codes -> fp16 SUBNORMALS: one AND puts a 2-bit code at mantissa bit p in
+//     {4, 6, 8} of both halves of a 32-bit word, i.e. the value code * 2^(p-24)
+//     (mma.sync consumes fp16 subnormals exactly);
+//   scores  S[tok, col] = sum_c code_c 2^(p_c-24) b_c,   b_c = q_c s_c 2^(8-p_c)
+//     split hi + lo in fp16 (HMUL2 / HFMA2): columns 0..3 hold the hi parts of
+//     heads 0..3, columns 4..7 the lo parts; the accumulator starts at the
+//     zero-point term sum_c q_c z_c, itself one mma per 16 channels (A = the
+//     key-zero row broadcast to all 16 rows, B = q);
+//   output  O^T[ch, col] = sum_t code_{t,ch} 2^(p-24) P'[t, col],  P' = p_t * v_scale_t
+//     (hi/lo), moved from the score fragment layout into the B layout by
+//     movmatrix; out_ch = (O^T[ch,h] + O^T[ch,h+4]) 2^(24-p) + sum_t p_t v_zero_t.
+// A 16-token m-tile takes its tokens in the order perm8 so that both the
+// key-word and the value-word shared loads of a warp hit 32 distinct banks.
 #include <math.h>
 
 #include "common.cuh"
@@ -33,23 +40,34 @@ namespace minikv {
 
 namespace {
 
-constexpr int kTile = 128;   // packed tokens per shared-memory stage (4 warps x 32)
-constexpr int kStages = 3;
 constexpr int kThreads = 128;
-constexpr int kPartStride = 132;   // floats per (unit, split, head): y[128], m, l
+constexpr int kSlice = 32;         // packed tokens per warp work item
+constexpr int kWarpStages = 4;
+constexpr int kResChunk = 64;      // residual tokens per residual CTA
+constexpr int kPartStride = 132;   // floats per (unit, slot, head): y[128], m, l
+constexpr int kMaxPackedCtas = 4096;
 
-struct __align__(16) Tile {
-    uint32_t kc[kTile * 8];
-    uint32_t vc[kTile * 8];
-    uint16_t ks[4 * kD];
-    uint16_t kz[4 * kD];
-    uint16_t vs[kTile];
-    uint16_t vz[kTile];
+struct __align__(16) SliceBuf {
+    uint32_t kc[kSlice * 8];   // key codes, token-major
+    uint32_t vc[kSlice * 8];   // value codes
+    uint16_t ks[kD];           // key scales of the slice's group
+    uint16_t kz[kD];           // key zeros of the slice's group
+    uint16_t vs[kSlice];       // value scales
+    uint16_t vz[kSlice];       // value zeros
 };
+constexpr uint32_t kSliceBytes = sizeof(SliceBuf);
+static_assert(kSliceBytes == 2688, "slice buffer layout");
 
 struct __align__(16) Smem {
-    Tile tile[kStages];
-    uint64_t full[kStages];
+    union {
+        SliceBuf st[4][kWarpStages];
+        struct {
+            uint16_t k[kResChunk * kD];   // XOR-swizzled rows (see swz)
+            uint16_t v[kResChunk * kD];
+        } res;
+    };
+    uint16_t qn[8][kD];      // query rows of the current unit (rows >= g are zero)
+    uint64_t full[4][kWarpStages];
     float wm[4][4], wl[4][4];
     float wy[4][4][kD];
     int flag;
@@ -68,23 +86,38 @@ struct Args {
     int *err;
     int Hkv, g, G, cap, ring;
     int n_q, r, res_start, flush;
-    int chunk, S;
+    int units, n_rc, spu, P, S_max;   // schedule: slices per unit, packed CTAs, partial slots per unit
+    int Ns;                           // total slices (< 2^31)
     float scale_log2;
 };
 
-// row permutation inside an 8-row half of an m-tile (see file comment)
-__device__ __forceinline__ int perm8(int r) {
-    return (0x57461320u >> (4 * r)) & 0xf;   // {0,2,1,3,6,4,7,5}
+// element offset of (row, col) in a [rows][128] fp16 tile; 16-byte chunks are
+// XOR-swizzled by row so ldmatrix reads of 8 rows hit distinct banks
+__device__ __forceinline__ int swz(int row, int col) {
+    return row * kD + ((((col >> 3) ^ (row & 7))) << 3) + (col & 7);
 }
 
-template <int S>
-__device__ __forceinline__ uint32_t shiftr(uint32_t x) {
-    if constexpr (S >= 0) return x >> S;
-    else return x << (-S);
+// column of element `col` of query row h in the swizzled sm.qn rows
+__device__ __forceinline__ int qn_col(int h, int col) { return (((col >> 3) ^ h) << 3) | (col & 7); }
+
+// token order inside an 8-row half of an m-tile: {0,2,1,3,6,4,7,5}
+__device__ __forceinline__ int perm8(int r) { return (0x57461320u >> (4 * r)) & 0xf; }
+
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+    return y;
 }
 
-__device__ __forceinline__ uint32_t magic(uint32_t x, uint32_t mask) {
-    return (x & mask) | 0x3C003C00u;   // fp16 1.0 in both halves + the code bits
+__device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("mul.rn.f16x2 %0, %1, %2;\n" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+__device__ __forceinline__ uint32_t hfma2(uint32_t a, uint32_t b, uint32_t c) {
+    uint32_t d;
+    asm("fma.rn.f16x2 %0, %1, %2, %3;\n" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
 }
 
 __device__ __forceinline__ float warp_sum_g(float x) {   // over lanes with equal t (xor 4, 8, 16)
@@ -100,12 +133,48 @@ __device__ __forceinline__ float warp_max_g(float x) {
     return x;
 }
 
-// Write this CTA's partial state for `unit`, split `split`, then let the last
-// arriving CTA of the unit merge all splits into `out`.
-__device__ void finish_unit(const Args &a, Smem &sm, int unit, int split, const float *m_h, const float *l_h,
-                            const float (*y_h)[kD]) {
+// word << 4 and word >> 6 as integer multiplies (IMAD / IMAD.HI), which issue
+// on the FMA pipe and leave the busier integer ALU to the masks
+__device__ __forceinline__ uint32_t shl4(uint32_t x) {
+    uint32_t y;
+    asm("mul.lo.u32 %0, %1, 16;\n" : "=r"(y) : "r"(x));
+    return y;
+}
+__device__ __forceinline__ uint32_t shr6(uint32_t x) {
+    uint32_t y;
+    asm("mul.hi.u32 %0, %1, 67108864;\n" : "=r"(y) : "r"(x));
+    return y;
+}
+
+// Code pair i (i = 0..7) of a 32-bit word of 16 codes -> fp16x2 subnormals
+// (code_i, code_{i+8}) at mantissa bit p_i: i -> p = 4,6,4,6,8,4,6,8.
+// x = word, x1 = word >> 6, x2 = word << 4.
+constexpr uint32_t kM4 = 0x00300030u, kM6 = 0x00C000C0u, kM8 = 0x03000300u;
+template <int I>
+__device__ __forceinline__ uint32_t code_pair(uint32_t x, uint32_t x1, uint32_t x2) {
+    if constexpr (I == 0) return x2 & kM4;
+    else if constexpr (I == 1) return x2 & kM6;
+    else if constexpr (I == 2) return x & kM4;
+    else if constexpr (I == 3) return x & kM6;
+    else if constexpr (I == 4) return x & kM8;
+    else if constexpr (I == 5) return x1 & kM4;
+    else if constexpr (I == 6) return x1 & kM6;
+    else return x1 & kM8;
+}
+// 2^(8 - p_i) and 2^(24 - p_i)
+__host__ __device__ constexpr float pair_wq(int i) {
+    return (i == 4 || i == 7) ? 1.f : ((i == 1 || i == 3 || i == 6) ? 4.f : 16.f);
+}
+__host__ __device__ constexpr float pair_wo(int i) { return pair_wq(i) * 65536.f; }
+
+// ---------------------------------------------------------------- partials
+
+// Write this CTA's partial state for `unit` into slot `slot`, then let the
+// last arriving CTA of the unit (S_u arrivals) merge all slots into `out`.
+__device__ void finish_unit(const Args &a, Smem &sm, int unit, int slot, int S_u, const float *m_h,
+                            const float *l_h, const float (*y_h)[kD]) {
     const int tid = threadIdx.x;
-    float *base = a.part + ((size_t)unit * a.S + split) * 4 * kPartStride;
+    float *base = a.part + ((size_t)unit * a.S_max + slot) * 4 * kPartStride;
     for (int h = 0; h < a.g; ++h) {
         base[h * kPartStride + tid] = y_h[h][tid];
         if (tid == 0) {
@@ -115,32 +184,76 @@ __device__ void finish_unit(const Args &a, Smem &sm, int unit, int split, const 
     }
     __threadfence();
     __syncthreads();
-    if (tid == 0) sm.flag = (atomicInc(&a.counters[unit], (unsigned)(a.S - 1)) == (unsigned)(a.S - 1));
+    if (tid == 0) sm.flag = (atomicInc(&a.counters[unit], (unsigned)(S_u - 1)) == (unsigned)(S_u - 1));
     __syncthreads();
     if (!sm.flag) return;
     __threadfence();
-    const float *ub = a.part + (size_t)unit * a.S * 4 * kPartStride;
+    const float *ub = a.part + (size_t)unit * a.S_max * 4 * kPartStride;
     const int b = unit / a.Hkv, kvh = unit % a.Hkv;
     const int Hq = a.Hkv * a.g;
     for (int h = 0; h < a.g; ++h) {
         float M = -INFINITY;
-        for (int s = 0; s < a.S; ++s) M = fmaxf(M, __ldcg(ub + (s * 4 + h) * kPartStride + 128));
+        for (int s = 0; s < S_u; ++s) M = fmaxf(M, __ldcg(ub + (s * 4 + h) * kPartStride + 128));
         float L = 0.f, Y = 0.f;
-        for (int s = 0; s < a.S; ++s) {
+        for (int s = 0; s < S_u; ++s) {
             const float *p = ub + (s * 4 + h) * kPartStride;
-            float ms = __ldcg(p + 128);
-            float f = (ms == -INFINITY) ? 0.f : exp2f(ms - M);
+            const float ms = __ldcg(p + 128);
+            const float f = (ms == -INFINITY) ? 0.f : ex2(ms - M);
             L += f * __ldcg(p + 129);
             Y += f * __ldcg(p + tid);
         }
-        a.out[((size_t)b * Hq + kvh * a.g + h) * kD + tid] = f2h(Y / L);
+        a.out[((size_t)b * Hq + kvh * a.g + h) * kD + tid] = f2h(__fdividef(Y, L));
     }
 }
 
-// ---------------------------------------------------------------- residual CTA
+// Merge the four warps' states (sm.wm / wl / wy) and hand the CTA partial on.
+__device__ void merge_warps_and_finish(const Args &a, Smem &sm, int unit, int slot, int S_u) {
+    const int tid = threadIdx.x;
+    __syncthreads();
+    float mh[4], lh[4], yh[4];
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+        const float M = fmaxf(fmaxf(sm.wm[0][h], sm.wm[1][h]), fmaxf(sm.wm[2][h], sm.wm[3][h]));
+        float L = 0.f, Y = 0.f;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+            const float f = (sm.wm[w][h] == -INFINITY) ? 0.f : ex2(sm.wm[w][h] - M);
+            L += f * sm.wl[w][h];
+            Y += f * sm.wy[w][h][tid];
+        }
+        mh[h] = M;
+        lh[h] = L;
+        yh[h] = Y;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int h = 0; h < 4; ++h) sm.wy[0][h][tid] = yh[h];
+    finish_unit(a, sm, unit, slot, S_u, mh, lh, sm.wy[0]);
+}
 
-__device__ void residual_cta(const Args &a, Smem &sm, int unit) {
+// packed CTA c covers slices [c*Ns/P, (c+1)*Ns/P); the CTA holding slice x
+__device__ __forceinline__ int cta_of_slice(long long x, int P, int Ns) {
+    return (int)(((x + 1) * P - 1) / Ns);
+}
+__device__ __forceinline__ void unit_slots(const Args &a, int unit, int &first, int &S_u) {
+    if (a.spu == 0) {
+        first = 0;
+        S_u = a.n_rc;
+        return;
+    }
+    first = cta_of_slice((long long)unit * a.spu, a.P, a.Ns);
+    const int last = cta_of_slice((long long)(unit + 1) * a.spu - 1, a.P, a.Ns);
+    S_u = a.n_rc + last - first + 1;
+}
+
+// ------------------------------------------------------------- residual CTAs
+
+// Residual chunk rc of a unit: logical residual tokens [64 rc, 64 rc + 64) in
+// fp16; warp w takes 16 of them as one m-tile.  Scores use q (exact in fp16)
+// as the B operand; outputs the same hi/lo P as the packed path.
+__device__ void residual_chunk_cta(const Args &a, Smem &sm, int unit, int rc) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int g_ = lane >> 2, t_ = lane & 3;
     const int b = unit / a.Hkv, kvh = unit % a.Hkv;
     const int Hq = a.Hkv * a.g;
     const uint16_t *knew = a.k_new + (size_t)unit * kD;
@@ -148,402 +261,500 @@ __device__ void residual_cta(const Args &a, Smem &sm, int unit) {
     uint16_t *kres = a.k_res + (size_t)unit * a.ring * kD;
     uint16_t *vres = a.v_res + (size_t)unit * a.ring * kD;
     const int r = a.r;
+    const int i0 = rc * kResChunk;
+    const int n = min(kResChunk, r - i0);
     auto slot = [&](int i) { int s = a.res_start + i; return s >= a.ring ? s - a.ring : s; };
     auto krow = [&](int i) -> const uint16_t * { return i == r - 1 ? knew : kres + (size_t)slot(i) * kD; };
     auto vrow = [&](int i) -> const uint16_t * { return i == r - 1 ? vnew : vres + (size_t)slot(i) * kD; };
 
-    // append: the new token goes to ring slot of logical index r-1
-    if (tid < 16) {
-        reinterpret_cast<uint4 *>(kres + (size_t)slot(r - 1) * kD)[tid] = reinterpret_cast<const uint4 *>(knew)[tid];
-    } else if (tid < 32) {
-        reinterpret_cast<uint4 *>(vres + (size_t)slot(r - 1) * kD)[tid - 16] =
-            reinterpret_cast<const uint4 *>(vnew)[tid - 16];
-    }
-
-    // shared scratch (the stage buffers are unused by this CTA)
-    float *qs = reinterpret_cast<float *>(&sm.tile[0]);     // [4][128]
-    float *sc = qs + 4 * kD;                                  // [4][ring]
-    for (int i = tid; i < a.g * kD; i += kThreads) {
-        int h = i / kD, c = i % kD;
-        qs[i] = h2f(a.q[((size_t)b * Hq + kvh * a.g + h) * kD + c]);
-    }
-    __syncthreads();
-    // scores: warp per token, lane per 4 channels
-    for (int i = warp; i < r; i += 4) {
-        uint2 raw = *reinterpret_cast<const uint2 *>(krow(i) + 4 * lane);
-        float k0 = h2f(raw.x & 0xffff), k1 = h2f(raw.x >> 16), k2 = h2f(raw.y & 0xffff), k3 = h2f(raw.y >> 16);
-        for (int h = 0; h < a.g; ++h) {
-            const float *qh = qs + h * kD + 4 * lane;
-            float d = qh[0] * k0 + qh[1] * k1 + qh[2] * k2 + qh[3] * k3;
-            for (int o = 16; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
-            if (lane == 0) sc[h * a.ring + i] = d * a.scale_log2;
-        }
-    }
-    __syncthreads();
-    // softmax per head (warp h)
-    if (warp < a.g) {
-        float *s = sc + warp * a.ring;
-        float m = -INFINITY;
-        for (int i = lane; i < r; i += 32) m = fmaxf(m, s[i]);
-        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        float l = 0.f;
-        for (int i = lane; i < r; i += 32) {
-            float p = exp2f(s[i] - m);
-            s[i] = p;
-            l += p;
-        }
-        for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
-        if (lane == 0) {
-            sm.wm[0][warp] = m;
-            sm.wl[0][warp] = l;
-        }
-    }
-    __syncthreads();
-    // values: thread per channel
-    for (int h = 0; h < a.g; ++h) sm.wy[0][h][tid] = 0.f;
     {
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
-        for (int i = 0; i < r; ++i) {
-            float v = h2f(vrow(i)[tid]);
-#pragma unroll
-            for (int h = 0; h < 4; ++h)
-                if (h < a.g) acc[h] += sc[h * a.ring + i] * v;
+        const int ch = tid & 15;
+        int s0 = a.res_start + i0 + (tid >> 4);
+        if (s0 >= a.ring) s0 -= a.ring;
+#pragma unroll 2
+        for (int row = tid >> 4; row < kResChunk; row += 8) {
+            const bool ok = row < n;
+            const bool newest = i0 + row == r - 1;
+            const uint16_t *ks = newest ? knew : kres + (size_t)s0 * kD;
+            const uint16_t *vs = newest ? vnew : vres + (size_t)s0 * kD;
+            const uint32_t so = (uint32_t)swz(row, ch * 8) * 2u;
+            cp_async16(smem_addr(sm.res.k) + so, (ok ? ks : kres) + ch * 8, ok);
+            cp_async16(smem_addr(sm.res.v) + so, (ok ? vs : vres) + ch * 8, ok);
+            s0 += 8;
+            if (s0 >= a.ring) s0 -= a.ring;
         }
-        for (int h = 0; h < a.g; ++h) sm.wy[0][h][tid] = acc[h];
     }
-    __syncthreads();
-
-    if (a.flush) {
-        // the oldest G residual tokens become key group n_q/G and G value tokens
-        const size_t tok0 = (size_t)unit * a.cap + a.n_q;
-        pack_key_group(krow, a.G, a.k_codes_w + tok0 * 8,
-                       a.k_scale_w + ((size_t)unit * (a.cap / a.G) + a.n_q / a.G) * kD,
-                       a.k_zero_w + ((size_t)unit * (a.cap / a.G) + a.n_q / a.G) * kD);
-        pack_value_tokens(vrow, a.G, kD, a.v_codes_w + tok0 * 8, a.v_scale_w + tok0, a.v_zero_w + tok0);
+    cp_async_commit();
+    if (i0 <= r - 1 && r - 1 < i0 + n) {   // append the new token to the ring
+        if (tid < 16)
+            reinterpret_cast<uint4 *>(kres + (size_t)slot(r - 1) * kD)[tid] = reinterpret_cast<const uint4 *>(knew)[tid];
+        else if (tid < 32)
+            reinterpret_cast<uint4 *>(vres + (size_t)slot(r - 1) * kD)[tid - 16] =
+                reinterpret_cast<const uint4 *>(vnew)[tid - 16];
     }
-    finish_unit(a, sm, unit, 0, sm.wm[0], sm.wl[0], sm.wy[0]);
-}
-
-// ------------------------------------------------------------------ packed CTA
-
-__device__ void issue_tile(const Args &a, Smem &sm, int stage, int unit, int t0, int n) {
-    Tile &T = sm.tile[stage];
-    const size_t tok = (size_t)unit * a.cap + t0;
-    const int gfirst = t0 / a.G, glast = (t0 + n - 1) / a.G;
-    const int ng = glast - gfirst + 1;
-    const uint32_t bytes = n * 32u * 2u + ng * kD * 2u * 2u + n * 2u * 2u;
-    mbar_arrive_expect_tx(&sm.full[stage], bytes);
-    bulk_g2s(T.kc, a.k_codes + tok * 8, n * 32u, &sm.full[stage]);
-    bulk_g2s(T.vc, a.v_codes + tok * 8, n * 32u, &sm.full[stage]);
-    const size_t grow = (size_t)unit * (a.cap / a.G) + gfirst;
-    bulk_g2s(T.ks, a.k_scale + grow * kD, ng * kD * 2u, &sm.full[stage]);
-    bulk_g2s(T.kz, a.k_zero + grow * kD, ng * kD * 2u, &sm.full[stage]);
-    bulk_g2s(T.vs, a.v_scale + tok, n * 2u, &sm.full[stage]);
-    bulk_g2s(T.vz, a.v_zero + tok, n * 2u, &sm.full[stage]);
-}
-
-__device__ void packed_cta(const Args &a, Smem &sm, int unit, int chunk_idx) {
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int g_ = lane >> 2, t_ = lane & 3;
-    const int b = unit / a.Hkv, kvh = unit % a.Hkv;
-    const int Hq = a.Hkv * a.g;
-    const int c0 = chunk_idx * a.chunk;
-    const int c1 = min(c0 + a.chunk, a.n_q);
-    const int ntiles = (c1 - c0 + kTile - 1) / kTile;
-
-    if (tid == 0) {
-        for (int s = 0; s < kStages; ++s) mbar_init(&sm.full[s], 1);
-        fence_mbar_init();
-    }
-    __syncthreads();
-    if (tid == 0)
-        for (int s = 0; s < kStages && s < ntiles; ++s) issue_tile(a, sm, s, unit, c0 + s * kTile, min(kTile, c1 - c0 - s * kTile));
-
-    // q * 2^(10-p) for the B-operand channels of this lane (head g_ & 3)
-    const int hq = g_ & 3;
-    const bool lo_col = g_ >= 4;
-    float qw[8][4];
+    // B operand: column g_ < 4 is query head g_ (channels in natural order), columns 4..7 are 0
+    uint32_t bq[8][2];
     {
-        const bool live = hq < a.g;
-        const uint16_t *qp = a.q + ((size_t)b * Hq + kvh * a.g + (live ? hq : 0)) * kD;
+        const int hq = g_ & 3;
+        const bool live = (g_ < 4) && (hq < a.g);
+        const uint32_t *qp =
+            reinterpret_cast<const uint32_t *>(a.q + ((size_t)b * Hq + kvh * a.g + (live ? hq : 0)) * kD);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-            const int c00 = 16 * (2 * t_ + (kk >> 2)) + 2 * (kk & 3);
-            qw[kk][0] = live ? h2f(qp[c00]) * 16.f : 0.f;
-            qw[kk][1] = live ? h2f(qp[c00 + 8]) * 16.f : 0.f;
-            qw[kk][2] = live ? h2f(qp[c00 + 1]) * 4.f : 0.f;
-            qw[kk][3] = live ? h2f(qp[c00 + 9]) * 4.f : 0.f;
+            bq[kk][0] = live ? qp[8 * kk + t_] : 0u;
+            bq[kk][1] = live ? qp[8 * kk + t_ + 4] : 0u;
         }
     }
-    // running state: heads hA = 2*(t_&1) + e, e = 0, 1
-    float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f}, pz[2] = {0.f, 0.f}, ps[2] = {0.f, 0.f};
+    cp_async_wait<0>();
+    __syncthreads();
+
+    const int hA = 2 * (t_ & 1);
+    float m_w[2] = {-INFINITY, -INFINITY}, l_w[2] = {0.f, 0.f};
     float acc[8][4];
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
-    const int hA = 2 * (t_ & 1);
-    const int pg = perm8(g_);
-    const int p2t = perm8(2 * t_), p2t1 = perm8(2 * t_ + 1);
-
-    for (int it = 0; it < ntiles; ++it) {
-        const int stage = it % kStages;
-        const int t0 = c0 + it * kTile;
-        const int n = min(kTile, c1 - t0);
-        bool ok = mbar_wait(&sm.full[stage], (it / kStages) & 1);
-        Tile &T = sm.tile[stage];
-        if (ok && 32 * warp < n) {
-            // ---- key group setup: B fragments and the per-head constant
-            const int grp = (t0 + 32 * warp) / a.G - t0 / a.G;
-            const uint16_t *ksr = T.ks + grp * kD, *kzr = T.kz + grp * kD;
-            uint32_t bk[8][2];
-            float part_b = 0.f, qz6 = 0.f, qz8 = 0.f;
+    if (16 * warp < n) {
+        float s[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                const int c00 = 16 * (2 * t_ + (kk >> 2)) + 2 * (kk & 3);
-                float x0 = qw[kk][0] * h2f(ksr[c00]), x1 = qw[kk][1] * h2f(ksr[c00 + 8]);
-                float x2 = qw[kk][2] * h2f(ksr[c00 + 1]), x3 = qw[kk][3] * h2f(ksr[c00 + 9]);
-                uint32_t h01 = pack_half2(x0, x1), h23 = pack_half2(x2, x3);
-                if (lo_col) {
-                    float2 f01 = unpack_half2(h01), f23 = unpack_half2(h23);
-                    h01 = pack_half2(x0 - f01.x, x1 - f01.y);
-                    h23 = pack_half2(x2 - f23.x, x3 - f23.y);
-                }
-                bk[kk][0] = h01;
-                bk[kk][1] = h23;
-                float2 u = unpack_half2(h01), v = unpack_half2(h23);
-                part_b += (u.x + u.y) + (v.x + v.y);
-                qz6 += qw[kk][0] * h2f(kzr[c00]) + qw[kk][1] * h2f(kzr[c00 + 8]);
-                qz8 += qw[kk][2] * h2f(kzr[c00 + 1]) + qw[kk][3] * h2f(kzr[c00 + 9]);
-            }
-            float cst = (lo_col ? 0.f : (qz6 * 0.0625f + qz8 * 0.25f)) - part_b;
-            cst += __shfl_xor_sync(0xffffffffu, cst, 1);
-            cst += __shfl_xor_sync(0xffffffffu, cst, 2);
-            cst += __shfl_xor_sync(0xffffffffu, cst, 16);
-            const float cA = __shfl_sync(0xffffffffu, cst, 4 * hA);
-            const float cB = __shfl_sync(0xffffffffu, cst, 4 * (hA + 1));
-
-            // ---- scores for the two m-tiles
-            float x[2][4];
-#pragma unroll
-            for (int mt = 0; mt < 2; ++mt) {
-                const int rowg = 32 * warp + 16 * mt + pg;
-                const uint2 ka = *reinterpret_cast<const uint2 *>(&T.kc[rowg * 8 + 2 * t_]);
-                const uint2 kb = *reinterpret_cast<const uint2 *>(&T.kc[(rowg + 8) * 8 + 2 * t_]);
-                float s[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t wa = (kk < 4) ? ka.x : ka.y, wb = (kk < 4) ? kb.x : kb.y;
-                    uint32_t sa, sb;
-                    switch (kk & 3) {
-                        case 0: sa = shiftr<-6>(wa); sb = shiftr<-6>(wb); break;
-                        case 1: sa = shiftr<-2>(wa); sb = shiftr<-2>(wb); break;
-                        case 2: sa = shiftr<2>(wa); sb = shiftr<2>(wb); break;
-                        default: sa = shiftr<6>(wa); sb = shiftr<6>(wb); break;
-                    }
-                    uint32_t af[4] = {magic(sa, 0x00C000C0u), magic(sb, 0x00C000C0u), magic(sa, 0x03000300u),
-                                      magic(sb, 0x03000300u)};
-                    mma16816(s, af, bk[kk][0], bk[kk][1]);
-                }
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    float v = s[i] + __shfl_xor_sync(0xffffffffu, s[i], 2);
-                    x[mt][i] = (v + ((i & 1) ? cB : cA)) * a.scale_log2;
-                }
-            }
-            // ---- online softmax update (per head e = 0, 1)
-            float alpha[2];
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                float mx = fmaxf(fmaxf(x[0][e], x[0][e + 2]), fmaxf(x[1][e], x[1][e + 2]));
-                mx = warp_max_g(mx);
-                const float mn = fmaxf(m_run[e], mx);
-                alpha[e] = exp2f(m_run[e] - mn);
-                m_run[e] = mn;
-                l_run[e] *= alpha[e];
-                pz[e] *= alpha[e];
-                ps[e] *= alpha[e];
-            }
-#pragma unroll
-            for (int nu = 0; nu < 8; ++nu) {
-                acc[nu][0] *= alpha[0];
-                acc[nu][1] *= alpha[1];
-                acc[nu][2] *= alpha[0];
-                acc[nu][3] *= alpha[1];
-            }
-            // ---- P' = p * v_scale (hi on lanes t<2, lo on t>=2), then O^T += V'^T P'
-#pragma unroll
-            for (int mt = 0; mt < 2; ++mt) {
-                const int base = 32 * warp + 16 * mt;
-                uint32_t prow[2];
-#pragma unroll
-                for (int hr = 0; hr < 2; ++hr) {   // row g (hr=0) and row g+8 (hr=1)
-                    const int tok = base + 8 * hr + pg;
-                    const float vsc = h2f(T.vs[tok]), vzr = h2f(T.vz[tok]);
-                    const float p0 = exp2f(x[mt][2 * hr] - m_run[0]);
-                    const float p1 = exp2f(x[mt][2 * hr + 1] - m_run[1]);
-                    l_run[0] += p0;
-                    l_run[1] += p1;
-                    pz[0] += p0 * vzr;
-                    pz[1] += p1 * vzr;
-                    const float y0 = p0 * vsc, y1 = p1 * vsc;
-                    uint32_t hv = pack_half2(y0, y1);
-                    if (t_ >= 2) {
-                        float2 f = unpack_half2(hv);
-                        hv = pack_half2(y0 - f.x, y1 - f.y);
-                    }
-                    float2 f = unpack_half2(hv);
-                    ps[0] += f.x;
-                    ps[1] += f.y;
-                    prow[hr] = hv;
-                }
-                const uint32_t bv0 = movmatrix_t(prow[0]), bv1 = movmatrix_t(prow[1]);
-                const uint32_t wA = T.vc[(base + p2t) * 8 + g_], wB = T.vc[(base + p2t1) * 8 + g_];
-                const uint32_t wC = T.vc[(base + 8 + p2t) * 8 + g_], wD = T.vc[(base + 8 + p2t1) * 8 + g_];
-                const uint32_t lo1 = __byte_perm(wA, wB, 0x5410), hi1 = __byte_perm(wA, wB, 0x7632);
-                const uint32_t lo2 = __byte_perm(wC, wD, 0x5410), hi2 = __byte_perm(wC, wD, 0x7632);
-#pragma unroll
-                for (int pr = 0; pr < 4; ++pr) {
-                    uint32_t s1, s2, s3, s4;
-                    switch (pr) {
-                        case 0: s1 = shiftr<-6>(lo1); s2 = shiftr<-6>(hi1); s3 = shiftr<-6>(lo2); s4 = shiftr<-6>(hi2); break;
-                        case 1: s1 = shiftr<-2>(lo1); s2 = shiftr<-2>(hi1); s3 = shiftr<-2>(lo2); s4 = shiftr<-2>(hi2); break;
-                        case 2: s1 = shiftr<2>(lo1); s2 = shiftr<2>(hi1); s3 = shiftr<2>(lo2); s4 = shiftr<2>(hi2); break;
-                        default: s1 = shiftr<6>(lo1); s2 = shiftr<6>(hi1); s3 = shiftr<6>(lo2); s4 = shiftr<6>(hi2); break;
-                    }
-                    uint32_t a6[4] = {magic(s1, 0x00C000C0u), magic(s2, 0x00C000C0u), magic(s3, 0x00C000C0u),
-                                      magic(s4, 0x00C000C0u)};
-                    mma16816(acc[2 * pr], a6, bv0, bv1);
-                    uint32_t a8[4] = {magic(s1, 0x03000300u), magic(s2, 0x03000300u), magic(s3, 0x03000300u),
-                                      magic(s4, 0x03000300u)};
-                    mma16816(acc[2 * pr + 1], a8, bv0, bv1);
-                }
-            }
+        for (int kk = 0; kk < 8; ++kk) {
+            uint32_t kf[4];
+            ldmatrix_x4(kf, smem_addr(sm.res.k + swz(16 * warp + (lane & 7) + 8 * ((lane >> 3) & 1),
+                                                      16 * kk + 8 * (lane >> 4))));
+            mma16816(s, kf, bq[kk][0], bq[kk][1]);
         }
-        const int timed_out = __syncthreads_or(!ok);
-        if (timed_out) {
-            if (tid == 0 && a.err) atomicExch(a.err, 1);
-            break;
-        }
-        if (tid == 0 && it + kStages < ntiles)
-            issue_tile(a, sm, stage, unit, t0 + kStages * kTile, min(kTile, c1 - t0 - kStages * kTile));
-    }
-
-    // ---- warp epilogue: y[channel][head] = (acc - sum P') * 2^(10-p) + sum p*zero
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-        l_run[e] = warp_sum_g(l_run[e]);
-        pz[e] = warp_sum_g(pz[e]);
-        ps[e] = warp_sum_g(ps[e]);
-    }
-#pragma unroll
-    for (int nu = 0; nu < 8; ++nu) {
-        const float w = (nu & 1) ? 4.f : 16.f;
+        float x[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            float y = (acc[nu][i] - ps[i & 1]) * w;
-            y += __shfl_xor_sync(0xffffffffu, y, 2);
-            acc[nu][i] = y + pz[i & 1];
+            const float v = s[i] + __shfl_xor_sync(0xffffffffu, s[i], 2);
+            const int row = 16 * warp + g_ + 8 * (i >> 1);
+            x[i] = row < n ? v * a.scale_log2 : -INFINITY;
+        }
+#pragma unroll
+        for (int e = 0; e < 2; ++e) m_w[e] = warp_max_g(fmaxf(x[e], x[e + 2]));
+        uint32_t prow[2];
+#pragma unroll
+        for (int hr = 0; hr < 2; ++hr) {
+            const float p0 = ex2(x[2 * hr] - m_w[0]), p1 = ex2(x[2 * hr + 1] - m_w[1]);
+            l_w[0] += p0;
+            l_w[1] += p1;
+            const uint32_t hv = pack_half2(p0, p1);
+            const float2 f = unpack_half2(hv);
+            const uint32_t lv = pack_half2(p0 - f.x, p1 - f.y);
+            prow[hr] = (t_ >= 2) ? lv : hv;
+        }
+        const uint32_t bv0 = movmatrix_t(prow[0]), bv1 = movmatrix_t(prow[1]);
+#pragma unroll
+        for (int nu = 0; nu < 8; ++nu) {
+            uint32_t va[4];
+            ldmatrix_x4_t(va, smem_addr(sm.res.v + swz(16 * warp + (lane & 7) + 8 * (lane >> 4),
+                                                        16 * nu + 8 * ((lane >> 3) & 1))));
+            mma16816(acc[nu], va, bv0, bv1);
         }
     }
+#pragma unroll
+    for (int e = 0; e < 2; ++e) l_w[e] = warp_sum_g(l_w[e]);
+#pragma unroll
+    for (int nu = 0; nu < 8; ++nu)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[nu][i] += __shfl_xor_sync(0xffffffffu, acc[nu][i], 2);
     if (t_ < 2) {
 #pragma unroll
         for (int nu = 0; nu < 8; ++nu) {
-            const int ch = 16 * g_ + nu;
+            const int ch = 16 * nu + g_;
             sm.wy[warp][hA][ch] = acc[nu][0];
             sm.wy[warp][hA + 1][ch] = acc[nu][1];
             sm.wy[warp][hA][ch + 8] = acc[nu][2];
             sm.wy[warp][hA + 1][ch + 8] = acc[nu][3];
         }
         if (g_ == 0) {
-            sm.wm[warp][hA] = m_run[0];
-            sm.wm[warp][hA + 1] = m_run[1];
-            sm.wl[warp][hA] = l_run[0];
-            sm.wl[warp][hA + 1] = l_run[1];
+            sm.wm[warp][hA] = m_w[0];
+            sm.wm[warp][hA + 1] = m_w[1];
+            sm.wl[warp][hA] = l_w[0];
+            sm.wl[warp][hA + 1] = l_w[1];
         }
+    }
+    if (a.flush && rc == 0) {
+        // the oldest G residual tokens become key group n_q/G and G value tokens
+        const size_t tok0 = (size_t)unit * a.cap + a.n_q;
+        const size_t grow = (size_t)unit * (a.cap / a.G) + a.n_q / a.G;
+        pack_key_group(krow, a.G, a.k_codes_w + tok0 * 8, a.k_scale_w + grow * kD, a.k_zero_w + grow * kD);
+        pack_value_tokens(vrow, a.G, kD, a.v_codes_w + tok0 * 8, a.v_scale_w + tok0, a.v_zero_w + tok0);
+    }
+    int first, S_u;
+    unit_slots(a, unit, first, S_u);
+    merge_warps_and_finish(a, sm, unit, rc, S_u);
+}
+
+// ------------------------------------------------------------------ packed CTA
+
+// Queue the bulk copies of the slice at (unit u, token t0) into this warp's
+// stage (called by one lane).
+__device__ __forceinline__ void issue_slice(const Args &a, Smem &sm, int warp, int stage, int u, int t0) {
+    SliceBuf &S = sm.st[warp][stage];
+    uint64_t *bar = &sm.full[warp][stage];
+    const size_t tok = (size_t)u * a.cap + t0;
+    const size_t grow = (size_t)u * (a.cap / a.G) + t0 / a.G;
+    mbar_arrive_expect_tx(bar, kSliceBytes);
+    bulk_g2s(S.kc, a.k_codes + tok * 8, kSlice * 32, bar);
+    bulk_g2s(S.vc, a.v_codes + tok * 8, kSlice * 32, bar);
+    bulk_g2s(S.ks, a.k_scale + grow * kD, kD * 2, bar);
+    bulk_g2s(S.kz, a.k_zero + grow * kD, kD * 2, bar);
+    bulk_g2s(S.vs, a.v_scale + tok, kSlice * 2, bar);
+    bulk_g2s(S.vz, a.v_zero + tok, kSlice * 2, bar);
+}
+
+// A warp's position in the flat slice list, kept as (unit, slice in unit) so
+// that stepping needs no division.
+struct Cursor {
+    int u, j;
+    __device__ __forceinline__ void step(int n, int spu) {
+        j += n;
+        while (j >= spu) {
+            j -= spu;
+            ++u;
+        }
+    }
+};
+
+// q * 2^(8-p) for the key B operand of this lane: head g_ & 3, the channel
+// pair of chunk KK, slot SIG (see code_pair)
+template <int KK, int SIG>
+__device__ __forceinline__ uint32_t qw_pair(const uint16_t *qh, int t_) {
+    constexpr int i = 2 * (KK & 3) + SIG;
+    const int c = 16 * (2 * t_ + (KK >> 2)) + i;
+    constexpr float w = pair_wq(i);
+    return pack_half2(h2f(qh[c]) * w, h2f(qh[c + 8]) * w);
+}
+
+__device__ void packed_cta(const Args &a, Smem &sm, int c) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int g_ = lane >> 2, t_ = lane & 3;
+    const int Hq = a.Hkv * a.g;
+    const int cs = (int)((long long)c * a.Ns / a.P), ce = (int)((long long)(c + 1) * a.Ns / a.P);
+
+    if (tid == 0) {
+        for (int w = 0; w < 4; ++w)
+            for (int s = 0; s < kWarpStages; ++s) mbar_init(&sm.full[w][s], 1);
+        fence_mbar_init();
     }
     __syncthreads();
-    // ---- merge the 4 warps (thread = channel)
-    float mh[4], lh[4];
-    for (int h = 0; h < 4; ++h) {
-        float M = fmaxf(fmaxf(sm.wm[0][h], sm.wm[1][h]), fmaxf(sm.wm[2][h], sm.wm[3][h]));
-        float L = 0.f, Y = 0.f;
-        for (int w = 0; w < 4; ++w) {
-            float f = (sm.wm[w][h] == -INFINITY) ? 0.f : exp2f(sm.wm[w][h] - M);
-            L += f * sm.wl[w][h];
-            Y += f * sm.wy[w][h][tid];
+    // this warp's slices: cs + warp + 4k; `nxt` is the next one to queue
+    Cursor nxt{(cs + warp) / a.spu, (cs + warp) % a.spu};
+    int nxt_x = cs + warp;
+    if (lane == 0)
+        for (int k = 0; k < kWarpStages && nxt_x < ce; ++k) {
+            issue_slice(a, sm, warp, k, nxt.u, nxt.j * kSlice);
+            nxt.step(4, a.spu);
+            nxt_x += 4;
         }
-        mh[h] = M;
-        lh[h] = L;
+
+    const int hA = 2 * (t_ & 1);
+    const int pg = perm8(g_);
+    const int p2t = perm8(2 * t_), p2t1 = perm8(2 * t_ + 1);
+    const uint32_t lo_neg = (g_ >= 4) ? 0xBC00BC00u : 0u;   // fp16x2 (-1, -1) on lo columns, (0, 0) on hi
+    int k = 0;   // this warp's slice counter over the whole range
+    bool ok = true;
+
+    int seg = cs;
+    while (seg < ce) {
+        const int unit = seg / a.spu;
+        const int seg_end = min(ce, (unit + 1) * a.spu);
+        const int b = unit / a.Hkv, kvh = unit % a.Hkv;
+        const uint16_t *qbase = a.q + ((size_t)b * Hq + kvh * a.g) * kD;
+        // query rows of this unit for the zero-point mma (rows >= g zero), 16-byte
+        // chunks XOR-swizzled by row so the ldmatrix of 8 rows is conflict-free
+        for (int e = tid; e < 8 * 16; e += kThreads) {
+            const int h = e / 16, ch = e % 16;
+            uint4 v = make_uint4(0, 0, 0, 0);
+            if (h < a.g) v = reinterpret_cast<const uint4 *>(qbase + (size_t)h * kD)[ch];
+            *reinterpret_cast<uint4 *>(&sm.qn[h][qn_col(h, 8 * ch)]) = v;
+        }
+        uint32_t qw[8][2];
+        {
+            const int hq = g_ & 3;
+            const bool live = hq < a.g;
+            const uint16_t *qh = qbase + (size_t)(live ? hq : 0) * kD;
+#define QW(KK)                                      \
+    qw[KK][0] = live ? qw_pair<KK, 0>(qh, t_) : 0u; \
+    qw[KK][1] = live ? qw_pair<KK, 1>(qh, t_) : 0u;
+            QW(0) QW(1) QW(2) QW(3) QW(4) QW(5) QW(6) QW(7)
+#undef QW
+        }
         __syncthreads();
-        sm.wy[0][h][tid] = Y;   // wy[0][h] is only read by this thread for this h
-        __syncthreads();
+
+        float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f}, pz[2] = {0.f, 0.f};
+        float acc[8][4];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
+
+        for (int x = cs + warp + 4 * k; ok && x < seg_end; x += 4, ++k) {
+            const int stage = k % kWarpStages;
+            ok = mbar_wait(&sm.full[warp][stage], (k / kWarpStages) & 1);
+            if (!ok) break;
+            const SliceBuf &S = sm.st[warp][stage];
+
+            // ---- key B operand: b = q s 2^(8-p), hi (columns 0-3) / lo (4-7)
+            uint32_t bk[8][2];
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                const int ch = 16 * (2 * t_ + (kk >> 2)) + 2 * (kk & 3);
+                const uint32_t sa = *reinterpret_cast<const uint32_t *>(&S.ks[ch]);
+                const uint32_t sb = *reinterpret_cast<const uint32_t *>(&S.ks[ch + 8]);
+                const uint32_t s0 = __byte_perm(sa, sb, 0x5410), s1 = __byte_perm(sa, sb, 0x7632);
+                // hi = fl(q s); lo = fl(q s - hi) (exact remainder); a lane keeps one of them
+                const uint32_t h0 = hmul2(qw[kk][0], s0), h1 = hmul2(qw[kk][1], s1);
+                bk[kk][0] = hfma2(qw[kk][0], s0, hmul2(h0, lo_neg));
+                bk[kk][1] = hfma2(qw[kk][1], s1, hmul2(h1, lo_neg));
+            }
+            // ---- zero-point term sum_c q_c z_c: A = the key-zero row in all 16 rows
+            float zc[4] = {0.f, 0.f, 0.f, 0.f}, zd[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int kp = 0; kp < 4; ++kp) {
+                uint32_t za[4], zb[4], qf[4];
+                ldmatrix_x4(za, smem_addr(&S.kz[32 * kp + 8 * (lane >> 4)]));
+                ldmatrix_x4(qf, smem_addr(&sm.qn[lane & 7][qn_col(lane & 7, 32 * kp + 8 * (lane >> 3))]));
+                mma16816(zc, za, qf[0], qf[1]);
+                ldmatrix_x4(zb, smem_addr(&S.kz[32 * kp + 16 + 8 * (lane >> 4)]));
+                mma16816(zd, zb, qf[2], qf[3]);
+            }
+            // ---- scores of the two m-tiles
+            float x_[2][4];
+#pragma unroll
+            for (int mt = 0; mt < 2; ++mt) {
+                const int row = 16 * mt + pg;
+                const uint2 ka = *reinterpret_cast<const uint2 *>(&S.kc[row * 8 + 2 * t_]);
+                const uint2 kb = *reinterpret_cast<const uint2 *>(&S.kc[(row + 8) * 8 + 2 * t_]);
+                float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};   // two chains (words 2t, 2t+1)
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    const uint32_t wa = half ? ka.y : ka.x, wb = half ? kb.y : kb.x;
+                    const uint32_t wa1 = shr6(wa), wa2 = shl4(wa), wb1 = shr6(wb), wb2 = shl4(wb);
+                    float (&s)[4] = half ? s1 : s0;
+#define KSTEP(Q)                                                                                          \
+    {                                                                                                     \
+        const uint32_t af[4] = {code_pair<2 * Q>(wa, wa1, wa2), code_pair<2 * Q>(wb, wb1, wb2),           \
+                                code_pair<2 * Q + 1>(wa, wa1, wa2), code_pair<2 * Q + 1>(wb, wb1, wb2)};  \
+        mma16816(s, af, bk[4 * half + Q][0], bk[4 * half + Q][1]);                                        \
     }
-    finish_unit(a, sm, unit, 1 + chunk_idx, mh, lh, sm.wy[0]);
+                    KSTEP(0) KSTEP(1) KSTEP(2) KSTEP(3)
+#undef KSTEP
+                }
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float v = (s0[i] + s1[i]) * 65536.f + (zc[i] + zd[i]);
+                    x_[mt][i] = (v + __shfl_xor_sync(0xffffffffu, v, 2)) * a.scale_log2;
+                }
+            }
+            // ---- online softmax: rescale only when a head's running max grows
+            float mx0 = fmaxf(fmaxf(x_[0][0], x_[0][2]), fmaxf(x_[1][0], x_[1][2]));
+            float mx1 = fmaxf(fmaxf(x_[0][1], x_[0][3]), fmaxf(x_[1][1], x_[1][3]));
+            mx0 = warp_max_g(mx0);
+            mx1 = warp_max_g(mx1);
+            if (__any_sync(0xffffffffu, mx0 > m_run[0] || mx1 > m_run[1])) {
+                const float n0 = fmaxf(m_run[0], mx0), n1 = fmaxf(m_run[1], mx1);
+                const float al0 = ex2(m_run[0] - n0), al1 = ex2(m_run[1] - n1);
+                m_run[0] = n0;
+                m_run[1] = n1;
+                l_run[0] *= al0;
+                l_run[1] *= al1;
+                pz[0] *= al0;
+                pz[1] *= al1;
+#pragma unroll
+                for (int nu = 0; nu < 8; ++nu) {
+                    acc[nu][0] *= al0;
+                    acc[nu][1] *= al1;
+                    acc[nu][2] *= al0;
+                    acc[nu][3] *= al1;
+                }
+            }
+            // ---- P' = p * v_scale (hi / lo) and O^T += code^T P'
+#pragma unroll
+            for (int mt = 0; mt < 2; ++mt) {
+                const int base = 16 * mt;
+                uint32_t prow[2];
+#pragma unroll
+                for (int hr = 0; hr < 2; ++hr) {
+                    const int tok = base + 8 * hr + pg;
+                    const float vsc = h2f(S.vs[tok]), vzr = h2f(S.vz[tok]);
+                    const float p0 = ex2(x_[mt][2 * hr] - m_run[0]);
+                    const float p1 = ex2(x_[mt][2 * hr + 1] - m_run[1]);
+                    l_run[0] += p0;
+                    l_run[1] += p1;
+                    pz[0] = fmaf(p0, vzr, pz[0]);
+                    pz[1] = fmaf(p1, vzr, pz[1]);
+                    const float y0 = p0 * vsc, y1 = p1 * vsc;
+                    const uint32_t hv = pack_half2(y0, y1);
+                    const float2 f = unpack_half2(hv);
+                    const uint32_t lv = pack_half2(y0 - f.x, y1 - f.y);
+                    prow[hr] = (t_ >= 2) ? lv : hv;
+                }
+                const uint32_t bv0 = movmatrix_t(prow[0]), bv1 = movmatrix_t(prow[1]);
+                const uint32_t wA = S.vc[(base + p2t) * 8 + g_], wB = S.vc[(base + p2t1) * 8 + g_];
+                const uint32_t wC = S.vc[(base + 8 + p2t) * 8 + g_], wD = S.vc[(base + 8 + p2t1) * 8 + g_];
+                const uint32_t l1 = __byte_perm(wA, wB, 0x5410), h1 = __byte_perm(wA, wB, 0x7632);
+                const uint32_t l2 = __byte_perm(wC, wD, 0x5410), h2 = __byte_perm(wC, wD, 0x7632);
+                const uint32_t l1a = shr6(l1), l1b = shl4(l1), h1a = shr6(h1), h1b = shl4(h1);
+                const uint32_t l2a = shr6(l2), l2b = shl4(l2), h2a = shr6(h2), h2b = shl4(h2);
+#define VSTEP(NU)                                                                          \
+    {                                                                                      \
+        const uint32_t af[4] = {code_pair<NU>(l1, l1a, l1b), code_pair<NU>(h1, h1a, h1b),  \
+                                code_pair<NU>(l2, l2a, l2b), code_pair<NU>(h2, h2a, h2b)}; \
+        mma16816(acc[NU], af, bv0, bv1);                                                   \
+    }
+                VSTEP(0) VSTEP(1) VSTEP(2) VSTEP(3) VSTEP(4) VSTEP(5) VSTEP(6) VSTEP(7)
+#undef VSTEP
+            }
+            __syncwarp();
+            if (lane == 0 && nxt_x < ce) {
+                issue_slice(a, sm, warp, stage, nxt.u, nxt.j * kSlice);
+                nxt.step(4, a.spu);
+                nxt_x += 4;
+            }
+        }
+        if (!ok && lane == 0 && a.err) atomicExch(a.err, 1);
+
+        // ---- warp epilogue: y[head][channel] = (O^T_hi + O^T_lo) 2^(24-p) + sum p * v_zero
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            l_run[e] = warp_sum_g(l_run[e]);
+            pz[e] = warp_sum_g(pz[e]);
+        }
+#define VOUT(NU)                                                                      \
+    _Pragma("unroll") for (int i = 0; i < 4; ++i) {                                   \
+        const float y = acc[NU][i] + __shfl_xor_sync(0xffffffffu, acc[NU][i], 2);     \
+        acc[NU][i] = y * pair_wo(NU) + pz[i & 1];                                     \
+    }
+        VOUT(0) VOUT(1) VOUT(2) VOUT(3) VOUT(4) VOUT(5) VOUT(6) VOUT(7)
+#undef VOUT
+        if (t_ < 2) {
+#pragma unroll
+            for (int nu = 0; nu < 8; ++nu) {
+                const int ch = 16 * g_ + nu;
+                sm.wy[warp][hA][ch] = acc[nu][0];
+                sm.wy[warp][hA + 1][ch] = acc[nu][1];
+                sm.wy[warp][hA][ch + 8] = acc[nu][2];
+                sm.wy[warp][hA + 1][ch + 8] = acc[nu][3];
+            }
+            if (g_ == 0) {
+                sm.wm[warp][hA] = m_run[0];
+                sm.wm[warp][hA + 1] = m_run[1];
+                sm.wl[warp][hA] = l_run[0];
+                sm.wl[warp][hA + 1] = l_run[1];
+            }
+        }
+        int first, S_u;
+        unit_slots(a, unit, first, S_u);
+        merge_warps_and_finish(a, sm, unit, a.n_rc + (c - first), S_u);
+        seg = seg_end;
+    }
 }
 
-__global__ void __launch_bounds__(kThreads) decode_kernel(const Args a) {
+__global__ void __launch_bounds__(kThreads, 4) decode_kernel(const Args a) {
     extern __shared__ __align__(128) unsigned char smem_raw[];
     Smem &sm = *reinterpret_cast<Smem *>(smem_raw);
-    const int unit = blockIdx.y;
-    if (blockIdx.x == 0) residual_cta(a, sm, unit);
-    else packed_cta(a, sm, unit, blockIdx.x - 1);
+    // packed CTAs first: they carry most of the work; the short residual CTAs fill in behind them
+    if ((int)blockIdx.x < a.P) packed_cta(a, sm, blockIdx.x);
+    else {
+        const int i = blockIdx.x - a.P;
+        residual_chunk_cta(a, sm, i / a.n_rc, i % a.n_rc);
+    }
 }
 
-int g_num_sms = 0;
+int g_slots = 0;   // resident decode CTAs on the device (SMs x CTAs per SM)
+bool g_attr_done = false;
+
+// the kernel's shared memory is above the 48 KB default: opt in once
+int ensure_attr() {
+    if (!g_attr_done) {
+        if (cudaFuncSetAttribute(decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(Smem)) !=
+            cudaSuccess)
+            return check_launch("decode_attn: cudaFuncSetAttribute");
+        g_attr_done = true;
+    }
+    return MINIKV_OK;
+}
+
+int resident_slots() {
+    if (g_slots == 0) {
+        int dev = 0, sms = 148, per = 4;
+        if (ensure_attr() == MINIKV_OK && cudaGetDevice(&dev) == cudaSuccess) {
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, decode_kernel, kThreads, sizeof(Smem)) !=
+                    cudaSuccess || per < 1)
+                per = 4;
+        }
+        cudaGetLastError();
+        g_slots = (sms > 0 ? sms : 148) * per;
+    }
+    return g_slots;
+}
+
+struct Plan {
+    int units, n_rc, spu, P, S_max, Ns;
+};
+
+Plan plan(const minikv_cache *c) {
+    Plan p;
+    p.units = c->B * c->Hkv;
+    p.n_rc = (c->n_res + 1 + kResChunk - 1) / kResChunk;
+    p.spu = c->n_packed / kSlice;
+    p.Ns = p.units * p.spu;   // the caller bounds units * cap below 2^31
+    p.P = 0;
+    if (p.Ns > 0) {
+        // three of every four resident slots run packed CTAs, all in one wave; the
+        // short residual CTAs queue behind them in the fourth
+        const int slots = resident_slots();
+        long long P = (3LL * slots) / 4;
+        const long long most = (p.Ns + 3) / 4;   // at least 4 slices per CTA
+        if (P > most) P = most;
+        if (P > kMaxPackedCtas) P = kMaxPackedCtas;
+        if (P < 1) P = 1;
+        p.P = (int)P;
+    }
+    // partial slots per unit: the residual chunks plus the most packed CTAs any unit meets
+    int per_unit = 0;
+    for (int u = 0; p.Ns > 0 && u < p.units; ++u) {
+        const long long lo = (long long)u * p.spu, hi = lo + p.spu - 1;
+        const int first = (int)(((lo + 1) * p.P - 1) / p.Ns), last = (int)(((hi + 1) * p.P - 1) / p.Ns);
+        if (last - first + 1 > per_unit) per_unit = last - first + 1;
+    }
+    p.S_max = p.n_rc + per_unit;
+    return p;
+}
 
 }  // namespace
-
-// Number of CTAs the launch splits a unit's packed tokens into.
-static void plan_chunks(int units, int n_q, int &n_chunks, int &chunk) {
-    if (g_num_sms == 0) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev);
-        if (g_num_sms <= 0) g_num_sms = 148;
-    }
-    n_chunks = 0;
-    chunk = kTile;
-    if (n_q <= 0) return;
-    const int target = 2 * 4 * g_num_sms;        // about two waves at 4 CTAs per SM
-    int want = target / units - 1;
-    if (want < 1) want = 1;
-    const int max_chunks = (n_q + kTile - 1) / kTile;
-    n_chunks = want < max_chunks ? want : max_chunks;
-    chunk = (n_q + n_chunks - 1) / n_chunks;
-    chunk = (chunk + 31) / 32 * 32;
-    n_chunks = (n_q + chunk - 1) / chunk;
-}
-
-size_t decode_workspace_bytes(int B, int Hkv, int max_tokens) {
-    const size_t units = (size_t)B * Hkv;
-    const size_t S = 1 + (size_t)(max_tokens + kTile - 1) / kTile;
-    return ((units * 4 + 255) / 256) * 256 + units * S * 4 * kPartStride * 4;
-}
 
 // Bytes of the workspace prefix that holds the per-unit arrival counters.
 size_t decode_counter_bytes(int B, int Hkv) { return (((size_t)B * Hkv * 4 + 255) / 256) * 256; }
 
+size_t decode_workspace_bytes(int B, int Hkv, int max_tokens) {
+    const size_t units = (size_t)B * Hkv;
+    const int res_max = max_tokens < 1024 ? max_tokens : 1024;   // the ring holds at most 1024 tokens
+    const size_t n_rc = (res_max + kResChunk - 1) / kResChunk + 1;
+    // every packed CTA holds at least 3 slices (the plan gives each about 4 or more)
+    const size_t spu = (size_t)max_tokens / kSlice + 1;
+    size_t per_unit = spu / 3 + 2;
+    if (per_unit > (size_t)kMaxPackedCtas) per_unit = kMaxPackedCtas;
+    return decode_counter_bytes(B, Hkv) + units * (n_rc + per_unit) * 4 * kPartStride * 4;
+}
+
 // Workspace bytes the next decode call on this cache state will use.
 size_t decode_call_workspace_bytes(const minikv_cache *c) {
-    const int units = c->B * c->Hkv;
-    int n_chunks, chunk;
-    plan_chunks(units, c->n_packed, n_chunks, chunk);
-    return decode_counter_bytes(c->B, c->Hkv) + (size_t)units * (1 + n_chunks) * 4 * kPartStride * 4;
+    const Plan p = plan(c);
+    return decode_counter_bytes(c->B, c->Hkv) + (size_t)p.units * p.S_max * 4 * kPartStride * 4;
 }
 
 int decode_launch(minikv_cache *c, const uint16_t *q, const uint16_t *k_new, const uint16_t *v_new, int Hq,
                   float sm_scale, uint16_t *out, void *ws, size_t ws_bytes, cudaStream_t stream) {
-    const int units = c->B * c->Hkv;
     const int g = Hq / c->Hkv;
     const int ring = c->R + c->G;
     const int r = c->n_res + 1;
     const int flush = (r == ring) ? 1 : 0;
     if (flush && c->n_packed + c->G > c->cap)
         return fail(MINIKV_ERR_CAPACITY, "decode_attn: flushing a key group would exceed cap=%d", c->cap);
-    int n_chunks, chunk;
-    plan_chunks(units, c->n_packed, n_chunks, chunk);
-    const int S = 1 + n_chunks;
-    const size_t cnt_bytes = (((size_t)units * 4 + 255) / 256) * 256;
-    const size_t need = cnt_bytes + (size_t)units * S * 4 * kPartStride * 4;
+    const Plan p = plan(c);
+    const size_t cnt_bytes = decode_counter_bytes(c->B, c->Hkv);
+    const size_t need = cnt_bytes + (size_t)p.units * p.S_max * 4 * kPartStride * 4;
     if (ws == nullptr || ws_bytes < need)
         return fail(MINIKV_ERR_INVALID_ARG, "decode_attn: workspace of %zu bytes needed, %zu given", need, ws_bytes);
 
@@ -559,17 +770,13 @@ int decode_launch(minikv_cache *c, const uint16_t *q, const uint16_t *k_new, con
     a.err = nullptr;
     a.Hkv = c->Hkv; a.g = g; a.G = c->G; a.cap = c->cap; a.ring = ring;
     a.n_q = c->n_packed; a.r = r; a.res_start = c->res_start; a.flush = flush;
-    a.chunk = chunk; a.S = S;
+    a.units = p.units; a.n_rc = p.n_rc; a.spu = p.spu; a.P = p.P; a.S_max = p.S_max; a.Ns = p.Ns;
     a.scale_log2 = sm_scale * kLog2e;
 
     const size_t smem = sizeof(Smem);
-    static bool attr_done = false;
-    if (!attr_done) {
-        if (cudaFuncSetAttribute(decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-            return check_launch("decode_attn: cudaFuncSetAttribute");
-        attr_done = true;
-    }
-    dim3 grid(S, units);
+    const int arc = ensure_attr();
+    if (arc) return arc;
+    const int grid = p.units * p.n_rc + p.P;
     decode_kernel<<<grid, kThreads, smem, stream>>>(a);
     int rc = check_launch("decode_attn");
     if (rc) return rc;

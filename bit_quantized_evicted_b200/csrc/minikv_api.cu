@@ -78,6 +78,8 @@ int decode_validate(minikv_cache *c, const uint16_t *q, const uint16_t *k_new, c
     if (Hq / c->Hkv > 4) return fail(MINIKV_ERR_UNSUPPORTED, "decode_attn: more than 4 query heads per KV head");
     if (c->Gv != c->D) return fail(MINIKV_ERR_UNSUPPORTED, "decode_attn: value group Gv=%d (needs Gv = D)", c->Gv);
     if ((size_t)c->B * c->Hkv > 65535) return fail(MINIKV_ERR_UNSUPPORTED, "decode_attn: B*Hkv above 65535");
+    if ((size_t)c->B * c->Hkv * (c->cap / 32) >= (1u << 31))
+        return fail(MINIKV_ERR_UNSUPPORTED, "decode_attn: B*Hkv*cap/32 must stay below 2^31");
     if (c->n_res + 1 == c->R + c->G && c->n_packed + c->G > c->cap)
         return fail(MINIKV_ERR_CAPACITY, "decode_attn: flushing a key group would exceed cap=%d", c->cap);
     return MINIKV_OK;
@@ -189,6 +191,8 @@ int minikv_decode_attn(minikv_cache *c, const uint16_t *q, const uint16_t *k_new
     if (Hq / c->Hkv > 4) return fail(MINIKV_ERR_UNSUPPORTED, "decode_attn: more than 4 query heads per KV head");
     if (c->Gv != c->D) return fail(MINIKV_ERR_UNSUPPORTED, "decode_attn: value group Gv=%d (needs Gv = D)", c->Gv);
     if ((size_t)c->B * c->Hkv > 65535) return fail(MINIKV_ERR_UNSUPPORTED, "decode_attn: B*Hkv above 65535");
+    if ((size_t)c->B * c->Hkv * (c->cap / 32) >= (1u << 31))
+        return fail(MINIKV_ERR_UNSUPPORTED, "decode_attn: B*Hkv*cap/32 must stay below 2^31");
     return decode_launch(c, q, k_new, v_new, Hq, sm_scale, out, ws, ws_bytes, static_cast<cudaStream_t>(stream));
 }
 

@@ -15,7 +15,8 @@ import os
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libminikv.so")
+# MINIKV_LIB points the binding at another build of the library
+LIB_PATH = os.environ.get("MINIKV_LIB", os.path.join(_PKG, "libminikv.so"))
 HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "minikv.h")
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CAPACITY, ERR_CUDA = 0, -1, -2, -3, -4
