@@ -87,6 +87,7 @@ struct Args {
     int Hkv, g, G, cap, ring;
     int n_q, r, res_start, flush;
     int units, n_rc, spu, P, S_max;   // schedule: slices per unit, packed CTAs, partial slots per unit
+    int groups_cap, lg2G;             // cap / G and log2(G)
     int Ns;                           // total slices (< 2^31)
     float scale_log2;
 };
@@ -387,13 +388,14 @@ __device__ void residual_chunk_cta(const Args &a, Smem &sm, int unit, int rc) {
 
 // ------------------------------------------------------------------ packed CTA
 
-// Queue the bulk copies of the slice at (unit u, token t0) into this warp's
-// stage (called by one lane).
-__device__ __forceinline__ void issue_slice(const Args &a, Smem &sm, int warp, int stage, int u, int t0) {
+// Queue the bulk copies of the slice at (unit u, slice j) into this warp's
+// stage.  Called by one lane; no division: G is a power of two.
+__device__ __forceinline__ void issue_slice(const Args &a, Smem &sm, int warp, int stage, int u, int j) {
     SliceBuf &S = sm.st[warp][stage];
     uint64_t *bar = &sm.full[warp][stage];
+    const int t0 = j * kSlice;
     const size_t tok = (size_t)u * a.cap + t0;
-    const size_t grow = (size_t)u * (a.cap / a.G) + t0 / a.G;
+    const size_t grow = (size_t)u * a.groups_cap + (t0 >> a.lg2G);
     mbar_arrive_expect_tx(bar, kSliceBytes);
     bulk_g2s(S.kc, a.k_codes + tok * 8, kSlice * 32, bar);
     bulk_g2s(S.vc, a.v_codes + tok * 8, kSlice * 32, bar);
@@ -426,6 +428,31 @@ __device__ __forceinline__ uint32_t qw_pair(const uint16_t *qh, int t_) {
     return pack_half2(h2f(qh[c]) * w, h2f(qh[c + 8]) * w);
 }
 
+// packed fp32 pairs (two lanes of work per instruction)
+__device__ __forceinline__ unsigned long long f2pack(float lo, float hi) {
+    unsigned long long r;
+    asm("mov.b64 %0, {%1, %2};\n" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2unpack(unsigned long long x, float &lo, float &hi) {
+    asm("mov.b64 {%0, %1}, %2;\n" : "=f"(lo), "=f"(hi) : "l"(x));
+}
+__device__ __forceinline__ unsigned long long fadd2(unsigned long long a, unsigned long long b) {
+    unsigned long long d;
+    asm("add.rn.f32x2 %0, %1, %2;\n" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ unsigned long long fmul2(unsigned long long a, unsigned long long b) {
+    unsigned long long d;
+    asm("mul.rn.f32x2 %0, %1, %2;\n" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ unsigned long long ffma2(unsigned long long a, unsigned long long b, unsigned long long c) {
+    unsigned long long d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;\n" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
 __device__ void packed_cta(const Args &a, Smem &sm, int c) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g_ = lane >> 2, t_ = lane & 3;
@@ -443,7 +470,7 @@ __device__ void packed_cta(const Args &a, Smem &sm, int c) {
     int nxt_x = cs + warp;
     if (lane == 0)
         for (int k = 0; k < kWarpStages && nxt_x < ce; ++k) {
-            issue_slice(a, sm, warp, k, nxt.u, nxt.j * kSlice);
+            issue_slice(a, sm, warp, k, nxt.u, nxt.j);
             nxt.step(4, a.spu);
             nxt_x += 4;
         }
@@ -452,6 +479,7 @@ __device__ void packed_cta(const Args &a, Smem &sm, int c) {
     const int pg = perm8(g_);
     const int p2t = perm8(2 * t_), p2t1 = perm8(2 * t_ + 1);
     const uint32_t lo_neg = (g_ >= 4) ? 0xBC00BC00u : 0u;   // fp16x2 (-1, -1) on lo columns, (0, 0) on hi
+    const bool lo_row = t_ >= 2;
     int k = 0;   // this warp's slice counter over the whole range
     bool ok = true;
 
@@ -482,7 +510,9 @@ __device__ void packed_cta(const Args &a, Smem &sm, int c) {
         }
         __syncthreads();
 
-        float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f}, pz[2] = {0.f, 0.f};
+        // running state of heads hA, hA+1: max (log2 units), sum p, sum p*v_zero
+        float m_run[2] = {-INFINITY, -INFINITY};
+        unsigned long long l2 = f2pack(0.f, 0.f), pz2 = f2pack(0.f, 0.f);
         float acc[8][4];
 #pragma unroll
         for (int i = 0; i < 8; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
@@ -493,21 +523,8 @@ __device__ void packed_cta(const Args &a, Smem &sm, int c) {
             if (!ok) break;
             const SliceBuf &S = sm.st[warp][stage];
 
-            // ---- key B operand: b = q s 2^(8-p), hi (columns 0-3) / lo (4-7)
-            uint32_t bk[8][2];
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                const int ch = 16 * (2 * t_ + (kk >> 2)) + 2 * (kk & 3);
-                const uint32_t sa = *reinterpret_cast<const uint32_t *>(&S.ks[ch]);
-                const uint32_t sb = *reinterpret_cast<const uint32_t *>(&S.ks[ch + 8]);
-                const uint32_t s0 = __byte_perm(sa, sb, 0x5410), s1 = __byte_perm(sa, sb, 0x7632);
-                // hi = fl(q s); lo = fl(q s - hi) (exact remainder); a lane keeps one of them
-                const uint32_t h0 = hmul2(qw[kk][0], s0), h1 = hmul2(qw[kk][1], s1);
-                bk[kk][0] = hfma2(qw[kk][0], s0, hmul2(h0, lo_neg));
-                bk[kk][1] = hfma2(qw[kk][1], s1, hmul2(h1, lo_neg));
-            }
             // ---- zero-point term sum_c q_c z_c: A = the key-zero row in all 16 rows
-            float zc[4] = {0.f, 0.f, 0.f, 0.f}, zd[4] = {0.f, 0.f, 0.f, 0.f};
+            float zc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int kp = 0; kp < 4; ++kp) {
                 uint32_t za[4], zb[4], qf[4];
@@ -515,56 +532,78 @@ __device__ void packed_cta(const Args &a, Smem &sm, int c) {
                 ldmatrix_x4(qf, smem_addr(&sm.qn[lane & 7][qn_col(lane & 7, 32 * kp + 8 * (lane >> 3))]));
                 mma16816(zc, za, qf[0], qf[1]);
                 ldmatrix_x4(zb, smem_addr(&S.kz[32 * kp + 16 + 8 * (lane >> 4)]));
-                mma16816(zd, zb, qf[2], qf[3]);
+                mma16816(zc, zb, qf[2], qf[3]);
             }
-            // ---- scores of the two m-tiles
-            float x_[2][4];
-#pragma unroll
-            for (int mt = 0; mt < 2; ++mt) {
-                const int row = 16 * mt + pg;
-                const uint2 ka = *reinterpret_cast<const uint2 *>(&S.kc[row * 8 + 2 * t_]);
-                const uint2 kb = *reinterpret_cast<const uint2 *>(&S.kc[(row + 8) * 8 + 2 * t_]);
-                float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};   // two chains (words 2t, 2t+1)
+            // ---- scores: both m-tiles, one k-chunk at a time; B operand made just in time
+            float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
+            {
+                const uint2 ka0 = *reinterpret_cast<const uint2 *>(&S.kc[pg * 8 + 2 * t_]);
+                const uint2 kb0 = *reinterpret_cast<const uint2 *>(&S.kc[(pg + 8) * 8 + 2 * t_]);
+                const uint2 ka1 = *reinterpret_cast<const uint2 *>(&S.kc[(pg + 16) * 8 + 2 * t_]);
+                const uint2 kb1 = *reinterpret_cast<const uint2 *>(&S.kc[(pg + 24) * 8 + 2 * t_]);
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
-                    const uint32_t wa = half ? ka.y : ka.x, wb = half ? kb.y : kb.x;
-                    const uint32_t wa1 = shr6(wa), wa2 = shl4(wa), wb1 = shr6(wb), wb2 = shl4(wb);
-                    float (&s)[4] = half ? s1 : s0;
-#define KSTEP(Q)                                                                                          \
-    {                                                                                                     \
-        const uint32_t af[4] = {code_pair<2 * Q>(wa, wa1, wa2), code_pair<2 * Q>(wb, wb1, wb2),           \
-                                code_pair<2 * Q + 1>(wa, wa1, wa2), code_pair<2 * Q + 1>(wb, wb1, wb2)};  \
-        mma16816(s, af, bk[4 * half + Q][0], bk[4 * half + Q][1]);                                        \
+                    const uint32_t a0 = half ? ka0.y : ka0.x, b0 = half ? kb0.y : kb0.x;
+                    const uint32_t a1 = half ? ka1.y : ka1.x, b1 = half ? kb1.y : kb1.x;
+                    const uint32_t a0r = shr6(a0), a0l = shl4(a0), b0r = shr6(b0), b0l = shl4(b0);
+                    const uint32_t a1r = shr6(a1), a1l = shl4(a1), b1r = shr6(b1), b1l = shl4(b1);
+#define KSTEP(Q)                                                                                               \
+    {                                                                                                          \
+        const int kk = 4 * half + Q;                                                                           \
+        const int ch = 16 * (2 * t_ + half) + 2 * Q;                                                           \
+        const uint32_t sa = *reinterpret_cast<const uint32_t *>(&S.ks[ch]);                                    \
+        const uint32_t sb = *reinterpret_cast<const uint32_t *>(&S.ks[ch + 8]);                                \
+        const uint32_t e0 = __byte_perm(sa, sb, 0x5410), e1 = __byte_perm(sa, sb, 0x7632);                     \
+        const uint32_t bk0 = hfma2(qw[kk][0], e0, hmul2(hmul2(qw[kk][0], e0), lo_neg));                        \
+        const uint32_t bk1 = hfma2(qw[kk][1], e1, hmul2(hmul2(qw[kk][1], e1), lo_neg));                        \
+        const uint32_t f0[4] = {code_pair<2 * Q>(a0, a0r, a0l), code_pair<2 * Q>(b0, b0r, b0l),                \
+                                code_pair<2 * Q + 1>(a0, a0r, a0l), code_pair<2 * Q + 1>(b0, b0r, b0l)};       \
+        mma16816(s0, f0, bk0, bk1);                                                                            \
+        const uint32_t f1[4] = {code_pair<2 * Q>(a1, a1r, a1l), code_pair<2 * Q>(b1, b1r, b1l),                \
+                                code_pair<2 * Q + 1>(a1, a1r, a1l), code_pair<2 * Q + 1>(b1, b1r, b1l)};       \
+        mma16816(s1, f1, bk0, bk1);                                                                            \
     }
                     KSTEP(0) KSTEP(1) KSTEP(2) KSTEP(3)
 #undef KSTEP
                 }
+            }
+            // ---- x = score * scale - mr (log2 units, relative to the running max mr;
+            //      0 stands in until a first max is known)
+            const float mr0 = (m_run[0] == -INFINITY) ? 0.f : m_run[0];
+            const float mr1 = (m_run[1] == -INFINITY) ? 0.f : m_run[1];
+            float x_[2][4];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const float v = (s0[i] + s1[i]) * 65536.f + (zc[i] + zd[i]);
-                    x_[mt][i] = (v + __shfl_xor_sync(0xffffffffu, v, 2)) * a.scale_log2;
-                }
+            for (int i = 0; i < 4; ++i) {
+                const float v0 = fmaf(zc[i], 1.f / 65536.f, s0[i]), v1 = fmaf(zc[i], 1.f / 65536.f, s1[i]);
+                const float w0 = v0 + __shfl_xor_sync(0xffffffffu, v0, 2);
+                const float w1 = v1 + __shfl_xor_sync(0xffffffffu, v1, 2);
+                x_[0][i] = fmaf(w0, a.scale_log2 * 65536.f, (i & 1) ? -mr1 : -mr0);
+                x_[1][i] = fmaf(w1, a.scale_log2 * 65536.f, (i & 1) ? -mr1 : -mr0);
             }
             // ---- online softmax: rescale only when a head's running max grows
             float mx0 = fmaxf(fmaxf(x_[0][0], x_[0][2]), fmaxf(x_[1][0], x_[1][2]));
             float mx1 = fmaxf(fmaxf(x_[0][1], x_[0][3]), fmaxf(x_[1][1], x_[1][3]));
-            mx0 = warp_max_g(mx0);
-            mx1 = warp_max_g(mx1);
+            mx0 = warp_max_g(mx0) + mr0;   // slice max, absolute
+            mx1 = warp_max_g(mx1) + mr1;
             if (__any_sync(0xffffffffu, mx0 > m_run[0] || mx1 > m_run[1])) {
                 const float n0 = fmaxf(m_run[0], mx0), n1 = fmaxf(m_run[1], mx1);
-                const float al0 = ex2(m_run[0] - n0), al1 = ex2(m_run[1] - n1);
+                const float al0 = ex2(m_run[0] - n0), al1 = ex2(m_run[1] - n1);   // 0 on the first slice
+                const float d0 = n0 - mr0, d1 = n1 - mr1;                            // shift of the reference
                 m_run[0] = n0;
                 m_run[1] = n1;
-                l_run[0] *= al0;
-                l_run[1] *= al1;
-                pz[0] *= al0;
-                pz[1] *= al1;
+                l2 = fmul2(l2, f2pack(al0, al1));
+                pz2 = fmul2(pz2, f2pack(al0, al1));
 #pragma unroll
                 for (int nu = 0; nu < 8; ++nu) {
                     acc[nu][0] *= al0;
                     acc[nu][1] *= al1;
                     acc[nu][2] *= al0;
                     acc[nu][3] *= al1;
+                }
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    x_[0][i] -= (i & 1) ? d1 : d0;
+                    x_[1][i] -= (i & 1) ? d1 : d0;
                 }
             }
             // ---- P' = p * v_scale (hi / lo) and O^T += code^T P'
@@ -576,37 +615,38 @@ __device__ void packed_cta(const Args &a, Smem &sm, int c) {
                 for (int hr = 0; hr < 2; ++hr) {
                     const int tok = base + 8 * hr + pg;
                     const float vsc = h2f(S.vs[tok]), vzr = h2f(S.vz[tok]);
-                    const float p0 = ex2(x_[mt][2 * hr] - m_run[0]);
-                    const float p1 = ex2(x_[mt][2 * hr + 1] - m_run[1]);
-                    l_run[0] += p0;
-                    l_run[1] += p1;
-                    pz[0] = fmaf(p0, vzr, pz[0]);
-                    pz[1] = fmaf(p1, vzr, pz[1]);
-                    const float y0 = p0 * vsc, y1 = p1 * vsc;
+                    const unsigned long long p2 = f2pack(ex2(x_[mt][2 * hr]), ex2(x_[mt][2 * hr + 1]));
+                    l2 = fadd2(l2, p2);
+                    pz2 = ffma2(p2, f2pack(vzr, vzr), pz2);
+                    const unsigned long long y2 = fmul2(p2, f2pack(vsc, vsc));
+                    float y0, y1;
+                    f2unpack(y2, y0, y1);
                     const uint32_t hv = pack_half2(y0, y1);
                     const float2 f = unpack_half2(hv);
-                    const uint32_t lv = pack_half2(y0 - f.x, y1 - f.y);
-                    prow[hr] = (t_ >= 2) ? lv : hv;
+                    float r0, r1;
+                    f2unpack(fadd2(y2, f2pack(-f.x, -f.y)), r0, r1);
+                    const uint32_t lv = pack_half2(r0, r1);
+                    prow[hr] = lo_row ? lv : hv;
                 }
                 const uint32_t bv0 = movmatrix_t(prow[0]), bv1 = movmatrix_t(prow[1]);
                 const uint32_t wA = S.vc[(base + p2t) * 8 + g_], wB = S.vc[(base + p2t1) * 8 + g_];
                 const uint32_t wC = S.vc[(base + 8 + p2t) * 8 + g_], wD = S.vc[(base + 8 + p2t1) * 8 + g_];
                 const uint32_t l1 = __byte_perm(wA, wB, 0x5410), h1 = __byte_perm(wA, wB, 0x7632);
-                const uint32_t l2 = __byte_perm(wC, wD, 0x5410), h2 = __byte_perm(wC, wD, 0x7632);
+                const uint32_t l2w = __byte_perm(wC, wD, 0x5410), h2 = __byte_perm(wC, wD, 0x7632);
                 const uint32_t l1a = shr6(l1), l1b = shl4(l1), h1a = shr6(h1), h1b = shl4(h1);
-                const uint32_t l2a = shr6(l2), l2b = shl4(l2), h2a = shr6(h2), h2b = shl4(h2);
-#define VSTEP(NU)                                                                          \
-    {                                                                                      \
-        const uint32_t af[4] = {code_pair<NU>(l1, l1a, l1b), code_pair<NU>(h1, h1a, h1b),  \
-                                code_pair<NU>(l2, l2a, l2b), code_pair<NU>(h2, h2a, h2b)}; \
-        mma16816(acc[NU], af, bv0, bv1);                                                   \
+                const uint32_t l2a = shr6(l2w), l2b = shl4(l2w), h2a = shr6(h2), h2b = shl4(h2);
+#define VSTEP(NU)                                                                             \
+    {                                                                                         \
+        const uint32_t af[4] = {code_pair<NU>(l1, l1a, l1b), code_pair<NU>(h1, h1a, h1b),     \
+                                code_pair<NU>(l2w, l2a, l2b), code_pair<NU>(h2, h2a, h2b)};   \
+        mma16816(acc[NU], af, bv0, bv1);                                                      \
     }
                 VSTEP(0) VSTEP(1) VSTEP(2) VSTEP(3) VSTEP(4) VSTEP(5) VSTEP(6) VSTEP(7)
 #undef VSTEP
             }
             __syncwarp();
             if (lane == 0 && nxt_x < ce) {
-                issue_slice(a, sm, warp, stage, nxt.u, nxt.j * kSlice);
+                issue_slice(a, sm, warp, stage, nxt.u, nxt.j);
                 nxt.step(4, a.spu);
                 nxt_x += 4;
             }
@@ -614,6 +654,9 @@ __device__ void packed_cta(const Args &a, Smem &sm, int c) {
         if (!ok && lane == 0 && a.err) atomicExch(a.err, 1);
 
         // ---- warp epilogue: y[head][channel] = (O^T_hi + O^T_lo) 2^(24-p) + sum p * v_zero
+        float l_run[2], pz[2];
+        f2unpack(l2, l_run[0], l_run[1]);
+        f2unpack(pz2, pz[0], pz[1]);
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
             l_run[e] = warp_sum_g(l_run[e]);
@@ -770,6 +813,8 @@ int decode_launch(minikv_cache *c, const uint16_t *q, const uint16_t *k_new, con
     a.err = nullptr;
     a.Hkv = c->Hkv; a.g = g; a.G = c->G; a.cap = c->cap; a.ring = ring;
     a.n_q = c->n_packed; a.r = r; a.res_start = c->res_start; a.flush = flush;
+    a.groups_cap = c->cap / c->G;
+    a.lg2G = 31 - __builtin_clz((unsigned)c->G);
     a.units = p.units; a.n_rc = p.n_rc; a.spu = p.spu; a.P = p.P; a.S_max = p.S_max; a.Ns = p.Ns;
     a.scale_log2 = sm_scale * kLog2e;
 

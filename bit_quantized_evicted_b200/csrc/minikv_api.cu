@@ -42,7 +42,7 @@ static int check_cache_shape(int B, int Hkv, int D, int G, int Gv, int R, int ca
     if (B < 1 || Hkv < 1 || G < 1 || Gv < 1 || R < 0 || cap < 0)
         return fail(MINIKV_ERR_INVALID_ARG, "cache shape: B=%d Hkv=%d G=%d Gv=%d R=%d cap=%d", B, Hkv, G, Gv, R, cap);
     if (D != kD) return fail(MINIKV_ERR_UNSUPPORTED, "head size D=%d (only 128)", D);
-    if (G % 32 != 0 || G > 128) return fail(MINIKV_ERR_UNSUPPORTED, "key group G=%d (32, 64, 96 or 128)", G);
+    if (!(G == 32 || G == 64 || G == 128)) return fail(MINIKV_ERR_UNSUPPORTED, "key group G=%d (32, 64 or 128)", G);
     if (!(Gv == 16 || Gv == 32 || Gv == 64 || Gv == 128))
         return fail(MINIKV_ERR_UNSUPPORTED, "value group Gv=%d (16, 32, 64 or 128)", Gv);
     if (cap % G != 0) return fail(MINIKV_ERR_INVALID_ARG, "cap=%d is not a multiple of G=%d", cap, G);

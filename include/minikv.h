@@ -48,7 +48,7 @@ extern "C" {
 
 #define MINIKV_OK                0
 #define MINIKV_ERR_INVALID_ARG  -1  /* null pointer, bad shape, W > keep, ... */
-#define MINIKV_ERR_UNSUPPORTED  -2  /* D != 128, G not a multiple of 32, ...  */
+#define MINIKV_ERR_UNSUPPORTED  -2  /* D != 128, G not 32/64/128, ...        */
 #define MINIKV_ERR_CAPACITY     -3  /* the packed cache would exceed `cap`     */
 #define MINIKV_ERR_CUDA         -4  /* a CUDA launch or attribute call failed  */
 
@@ -169,7 +169,8 @@ MINIKV_API int minikv_topk_evict(const float *scores, const uint16_t *k, const u
  *       the next (its arrival counters return to zero).  Calls that share one
  *       ws must not overlap on the GPU.
  * Errors: INVALID_ARG (null, Hq % Hkv, ws too small), CAPACITY (a flush would
- * exceed cap), UNSUPPORTED (D != 128, Gv != D, G not a multiple of 32).
+ * exceed cap), UNSUPPORTED (D != 128, Gv != D, G not 32/64/128, more than 4
+ * query heads per KV head).
  */
 MINIKV_API int minikv_decode_attn(minikv_cache *c, const uint16_t *q, const uint16_t *k_new,
                        const uint16_t *v_new, int Hq, float sm_scale, uint16_t *out,
