@@ -445,8 +445,11 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--layers", type=int, default=DECODE["layers"],
                     help="decode layers (fewer only for small profiling runs; the workload has 32)")
+    ap.add_argument("--prefill-layers", type=int, default=PREFILL["layers"],
+                    help="prefill layers (fewer only for small profiling runs; the workload has 32)")
     args = ap.parse_args()
     DECODE["layers"] = args.layers
+    PREFILL["layers"] = args.prefill_layers
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     if args.impl == "reference":

@@ -246,6 +246,34 @@ void oracle_prefill_attention(const uint16_t *q, const uint16_t *k, const uint16
     free(kd); free(vd); free(p); free(qi);
 }
 
+/* O1 for selected query rows only: rows[n] in [0, T); out [nrows, D] fp64.
+ * Row i is the same computation as in oracle_prefill_attention. */
+void oracle_prefill_attention_rows(const uint16_t *q, const uint16_t *k, const uint16_t *v, int T, int D,
+                                   double tau, const int32_t *rows, int nrows, double *out)
+{
+    double *p = (double *)malloc(sizeof(double) * (size_t)T + 8);
+    double *qi = (double *)malloc(sizeof(double) * (size_t)D + 8);
+    for (int n = 0; n < nrows; ++n) {
+        int i = rows[n];
+        for (int c = 0; c < D; ++c) qi[c] = oracle_half_to_double(q[(long)i * D + c]);
+        double m = -INFINITY;
+        for (int j = 0; j <= i; ++j) {
+            double s = 0.0;
+            for (int c = 0; c < D; ++c) s += qi[c] * oracle_half_to_double(k[(long)j * D + c]);
+            p[j] = tau * s;
+            if (p[j] > m) m = p[j];
+        }
+        double l = 0.0;
+        for (int j = 0; j <= i; ++j) { p[j] = exp(p[j] - m); l += p[j]; }
+        for (int c = 0; c < D; ++c) {
+            double acc = 0.0;
+            for (int j = 0; j <= i; ++j) acc += p[j] * oracle_half_to_double(v[(long)j * D + c]);
+            out[(long)n * D + c] = acc / l;
+        }
+    }
+    free(p); free(qi);
+}
+
 /* ------------------------------------------- O2: observation-window scores */
 
 /* One KV head.  q: [g, T, D] fp16 (the g query heads that read this KV head),

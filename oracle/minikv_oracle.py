@@ -61,6 +61,7 @@ _SIGS = {
     "oracle_pack_tokens": (None, [_P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P]),
     "oracle_dequant_tokens": (None, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P]),
     "oracle_prefill_attention": (None, [_P, _P, _P, _I, _I, _D, _P]),
+    "oracle_prefill_attention_rows": (None, [_P, _P, _P, _I, _I, _D, _P, _I, _P]),
     "oracle_window_scores": (None, [_P, _P, _I, _I, _I, _I, _D, _P]),
     "oracle_select": (_I, [_P, _I, _I, _I, _P]),
     "oracle_decode_attention": (None, [_P, _I, _P, _P, _P, _P, _P, _P, _I, _P, _P, _I, _I, _I, _I, _D, _P]),
@@ -171,6 +172,16 @@ def prefill_attention(q, k, v, tau: float) -> np.ndarray:
     return o
 
 
+def prefill_attention_rows(q, k, v, rows, tau: float) -> np.ndarray:
+    """O1 for the listed query rows of one head: -> [len(rows), D] fp64."""
+    qb, kb, vb = _h(q), _h(k), _h(v)
+    T, D = qb.shape
+    r = np.ascontiguousarray(rows, dtype=np.int32)
+    out = np.zeros((r.size, D))
+    lib().oracle_prefill_attention_rows(_ptr(qb), _ptr(kb), _ptr(vb), T, D, tau, _ptr(r), r.size, _ptr(out))
+    return out
+
+
 def window_scores(q_group, k, W: int, tau: float) -> np.ndarray:
     """O2 for one KV head: q_group [g, T, D], k [T, D] fp16 -> s [T] fp64."""
     qb, kb = _h(q_group), _h(k)
@@ -257,6 +268,14 @@ class SliceCache:
         if self.r == self.R + self.G:
             self.flush()
         return out
+
+    def advance(self, k_new, v_new) -> None:
+        """O9 without the attention: append the new token and flush if due
+        (bookkeeping for steps whose output is not checked)."""
+        self.res_k.append(_h(k_new).ravel().copy())
+        self.res_v.append(_h(v_new).ravel().copy())
+        if self.r == self.R + self.G:
+            self.flush()
 
     def flush(self) -> None:
         """Pack the oldest G residual tokens as the next key group and G value tokens."""

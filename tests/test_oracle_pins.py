@@ -215,6 +215,31 @@ def test_prefill_attention_matches_torch_fp64(oracle):
     assert np.array_equal(o[0], v[0].astype(np.float64))       # row 0 sees only key 0
 
 
+def test_prefill_rows_match_full_rows(oracle):
+    T, D = 90, 128
+    q = synth.normal_fp16((T, D), 27).numpy()
+    k = synth.keys_fp16((T, D), 28).numpy()
+    v = synth.normal_fp16((T, D), 29).numpy()
+    rows = np.array([0, 1, 44, 89, 7])
+    full = oracle.prefill_attention(q, k, v, TAU)
+    assert np.array_equal(oracle.prefill_attention_rows(q, k, v, rows, TAU), full[rows])
+
+
+def test_decode_advance_equals_step_bookkeeping(oracle):
+    D, N = 128, 100
+    k = synth.keys_fp16((N + 40, D), 71).numpy()
+    v = synth.normal_fp16((N + 40, D), 72).numpy()
+    q = synth.normal_fp16((1, D), 73).numpy()
+    a = oracle.SliceCache.from_kept(k[:N], v[:N], R=32, G=32, Gv=128)
+    b = oracle.SliceCache.from_kept(k[:N], v[:N], R=32, G=32, Gv=128)
+    for i in range(40):
+        a.step(q, k[N + i], v[N + i], TAU)
+        b.advance(k[N + i], v[N + i])
+    for key in ("k_codes", "k_scale", "k_zero", "v_codes", "v_scale", "v_zero"):
+        assert np.array_equal(getattr(a, key), getattr(b, key))
+    assert np.array_equal(np.array(a.res_k), np.array(b.res_k))
+
+
 def test_prefill_attention_equal_keys_is_running_mean(oracle):
     T, D = 40, 128
     q = synth.normal_fp16((T, D), 24).numpy()
