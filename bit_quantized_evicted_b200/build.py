@@ -15,7 +15,7 @@ CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libminikv.so")
 SOURCES = ["minikv_api.cu", "pack.cu", "prefill.cu", "topk.cu", "decode.cu", "decode_static.cu"]
-HEADERS = ["common.cuh"]
+HEADERS = ["common.cuh", "tc.cuh"]
 NVCC = os.environ.get("NVCC", "nvcc")
 FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -29,6 +29,31 @@ __device__ __forceinline__ float2 unpack_half2(uint32_t x) {
     return __half22float2(h);
 }
 
+// Packed fp32 pairs (lo in bits 0..31): one f32x2 instruction per two lanes of work.
+__device__ __forceinline__ unsigned long long f2pack(float lo, float hi) {
+    unsigned long long r;
+    asm("mov.b64 %0, {%1, %2};\n" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2unpack(unsigned long long x, float &lo, float &hi) {
+    asm("mov.b64 {%0, %1}, %2;\n" : "=f"(lo), "=f"(hi) : "l"(x));
+}
+__device__ __forceinline__ unsigned long long fadd2(unsigned long long a, unsigned long long b) {
+    unsigned long long d;
+    asm("add.rn.f32x2 %0, %1, %2;\n" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ unsigned long long fmul2(unsigned long long a, unsigned long long b) {
+    unsigned long long d;
+    asm("mul.rn.f32x2 %0, %1, %2;\n" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ unsigned long long ffma2(unsigned long long a, unsigned long long b, unsigned long long c) {
+    unsigned long long d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;\n" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
 // D (16x8 fp32) += A (16x16 fp16, row) * B (16x8 fp16, col).
 // Fragment ownership, g = lane/4, t = lane%4:
 //   A: a[0]={(g,2t),(g,2t+1)} a[1]={(g+8,2t),(g+8,2t+1)} a[2]={(g,2t+8),(g,2t+9)} a[3]={(g+8,2t+8),(g+8,2t+9)}

@@ -150,6 +150,8 @@ int minikv_select_prefill(const uint16_t *q, const uint16_t *k, const uint16_t *
     if (B < 1 || Hq < 1 || Hkv < 1 || T < 1 || Hq % Hkv)
         return fail(MINIKV_ERR_INVALID_ARG, "select_prefill: B=%d Hq=%d Hkv=%d T=%d", B, Hq, Hkv, T);
     if (D != kD) return fail(MINIKV_ERR_UNSUPPORTED, "select_prefill: D=%d (only 128)", D);
+    if (!(sm_scale > 0.f) || !(sm_scale < INFINITY))
+        return fail(MINIKV_ERR_INVALID_ARG, "select_prefill: sm_scale must be positive and finite");
     if (W < 1 || W > T) return fail(MINIKV_ERR_INVALID_ARG, "select_prefill: W=%d must be in [1, T=%d]", W, T);
     if ((Hq / Hkv) * W > 512) return fail(MINIKV_ERR_UNSUPPORTED, "select_prefill: (Hq/Hkv)*W above 512");
     if ((size_t)B * Hq > 65535 || (size_t)B * Hkv > 65535)

@@ -13,15 +13,19 @@
 // rows, fp16 mma.sync with fp32 accumulation, K/V double-buffered by cp.async
 // in XOR-swizzled shared memory.  Kernel 2 (window_score_kernel): one CTA per
 // 64 keys of one KV head; S^T = K Q_w^T on the tensor cores, then column sums.
+#include <cudaTypedefs.h>
 #include <math.h>
 
+#include <mutex>
+
 #include "common.cuh"
+#include "tc.cuh"
 
 namespace minikv {
 
 namespace {
 
-constexpr int kBM = 64, kBN = 64;
+constexpr int kBN = 64;   // keys per window-score CTA
 
 // element offset of (row, col) in a [rows][128] fp16 tile, 16-byte chunks
 // XOR-swizzled by row so ldmatrix row reads hit distinct banks
@@ -41,181 +45,288 @@ __device__ __forceinline__ void load_tile(uint16_t *tile, const uint16_t *g, int
     }
 }
 
+// ---------------------------------------------------------------- kernel 1
+//
+// One CTA = one 128-row query tile of one (sequence, query head); 6 warps:
+//   warp 0      TMA producer: the Q tile once, then K_j / V_j into 2 stages;
+//   warp 1      TMEM owner and the single thread issuing tcgen05.mma;
+//   warps 2..5  softmax: thread = query row = TMEM lane (warp w reads lanes
+//               32*(w%4) .. +31), plus the O rescale and the epilogue.
+// Tensor memory (512 columns): S_0, S_1 fp32 [128 x 128] at 0 / 128; O fp32 at
+// 256; P_0, P_1 (fp16 pairs, the A operand of P V) at 384 / 448.
+// Issue order S_0, S_1, PV_0, S_2, PV_1, ... lets the tensor pipe compute
+// PV_{j-1} and S_{j+1} while the softmax warps work on S_j.
+// The running max is lazy: a row's reference max moves only when a new score
+// exceeds it by more than 2^8 (p <= 256 stays exact enough in fp16), so O is
+// rescaled rarely; l and O always refer to the same reference.
+constexpr int kTileM = 128, kTileN = 128;
+constexpr int kFaThreads = 192;
+constexpr uint32_t kColS = 0, kColO = 256, kColP = 384;
+constexpr float kLazyMax = 8.f;
+
+struct FaSmem {
+    uint16_t q[2][kTileM * 64];        // K-blocks of 64 fp16, 128-byte swizzle
+    uint16_t k[2][2][kTileN * 64];     // [stage][K-block]
+    uint16_t v[2][2][kTileN * 64];     // [stage][64-wide d block]: MN-major B of P V
+    uint64_t q_full, k_full[2], k_empty[2], v_full[2], v_empty[2];
+    uint64_t s_full[2], s_empty[2], p_full[2], o_done;
+    uint32_t tmem_base;
+    int abort;
+};
+
 struct FaArgs {
-    const uint16_t *q, *k, *v;
-    uint16_t *o;
     float *lse2;   // [B, Hq, W] window rows, log2 domain
-    int Hq, Hkv, T, W;
+    int Hq, Hkv, T, W, nqt;
     float scale_log2;
 };
 
-__global__ void __launch_bounds__(128) fa_fwd_kernel(const FaArgs a) {
-    extern __shared__ __align__(128) unsigned char smem_raw[];
-    uint16_t *sQ = reinterpret_cast<uint16_t *>(smem_raw);
-    uint16_t *sK = sQ + kBM * kD;          // [2][64][128]
-    uint16_t *sV = sK + 2 * kBN * kD;      // [2][64][128]
+// Bounded wait shared by a CTA: once any wait times out, every later wait
+// returns false at once so all roles reach the final barrier.
+__device__ __forceinline__ bool fa_wait(FaSmem &s, uint64_t *bar, uint32_t parity) {
+    if (*reinterpret_cast<volatile int *>(&s.abort)) return false;
+    if (mbar_wait(bar, parity)) return true;
+    *reinterpret_cast<volatile int *>(&s.abort) = 1;
+    return false;
+}
 
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;\n" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__global__ void __launch_bounds__(kFaThreads, 1)
+    fa_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
+                 const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_o, const FaArgs a) {
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    FaSmem &s = *reinterpret_cast<FaSmem *>(smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u));
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int g = lane >> 2, t = lane & 3;
-    const int nqt = (a.T + kBM - 1) / kBM;
-    const int qt = nqt - 1 - blockIdx.x;    // heaviest tiles first
-    const int bh = blockIdx.y;
+
+    // heads outer, query tiles (heaviest first) inner: the CTAs resident at
+    // one time share one head's K / V in L2
+    const int bh = blockIdx.x / a.nqt;
+    const int qt = a.nqt - 1 - (int)(blockIdx.x % a.nqt);
     const int b = bh / a.Hq, h = bh % a.Hq;
-    const int kvh = h / (a.Hq / a.Hkv);
-    const uint16_t *qg = a.q + (size_t)bh * a.T * kD;
-    const uint16_t *kg = a.k + ((size_t)b * a.Hkv + kvh) * a.T * kD;
-    const uint16_t *vg = a.v + ((size_t)b * a.Hkv + kvh) * a.T * kD;
-    const int q0 = qt * kBM;
+    const int kvh = b * a.Hkv + h / (a.Hq / a.Hkv);
     const int nkb = qt + 1;   // causal: key blocks 0..qt
 
-    load_tile(sQ, qg, q0, kBM, a.T);
-    cp_async_commit();
-    load_tile(sK, kg, 0, kBN, a.T);
-    load_tile(sV, vg, 0, kBN, a.T);
-    cp_async_commit();
-
-    uint32_t qf[8][4];
-    float oacc[16][4];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) oacc[i][0] = oacc[i][1] = oacc[i][2] = oacc[i][3] = 0.f;
-    float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f}, lr[2] = {0.f, 0.f};
-    const int row_g = q0 + 16 * warp + g;   // this lane's rows: row_g and row_g + 8
-
-    for (int kb = 0; kb < nkb; ++kb) {
-        cp_async_wait<0>();
-        __syncthreads();
-        if (kb + 1 < nkb) {
-            load_tile(sK + ((kb + 1) & 1) * kBN * kD, kg, (kb + 1) * kBN, kBN, a.T);
-            load_tile(sV + ((kb + 1) & 1) * kBN * kD, vg, (kb + 1) * kBN, kBN, a.T);
-            cp_async_commit();
+    if (tid == 0) {
+        mbar_init(&s.q_full, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&s.k_full[i], 1);
+            mbar_init(&s.k_empty[i], 1);
+            mbar_init(&s.v_full[i], 1);
+            mbar_init(&s.v_empty[i], 1);
+            mbar_init(&s.s_full[i], 1);
+            mbar_init(&s.s_empty[i], 128);
+            mbar_init(&s.p_full[i], 128);
         }
-        if (kb == 0) {
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                const int r = 16 * warp + (lane & 7) + 8 * ((lane >> 3) & 1);
-                const int c = 16 * kk + 8 * (lane >> 4);
-                ldmatrix_x4(qf[kk], smem_addr(sQ + swz(r, c)));
+        mbar_init(&s.o_done, 1);
+        s.abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) tc::tmem_alloc(&s.tmem_base, 512);
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = s.tmem_base;
+
+    if (warp == 0) {
+        // ---------------- producer
+        if (lane == 0) {
+            tc::prefetch_map(&map_q);
+            tc::prefetch_map(&map_k);
+            tc::prefetch_map(&map_v);
+            mbar_arrive_expect_tx(&s.q_full, 2 * kTileM * 128);
+            tc::tma_load_3d(s.q[0], &map_q, 0, qt * kTileM, bh, &s.q_full);
+            tc::tma_load_3d(s.q[1], &map_q, 64, qt * kTileM, bh, &s.q_full);
+            for (int j = 0; j < nkb; ++j) {
+                const int st = j & 1;
+                if (j >= 2 && !fa_wait(s, &s.k_empty[st], ((j - 2) >> 1) & 1)) break;
+                mbar_arrive_expect_tx(&s.k_full[st], 2 * kTileN * 128);
+                tc::tma_load_3d(s.k[st][0], &map_k, 0, j * kTileN, kvh, &s.k_full[st]);
+                tc::tma_load_3d(s.k[st][1], &map_k, 64, j * kTileN, kvh, &s.k_full[st]);
+                if (j >= 2 && !fa_wait(s, &s.v_empty[st], ((j - 2) >> 1) & 1)) break;
+                mbar_arrive_expect_tx(&s.v_full[st], 2 * kTileN * 128);
+                tc::tma_load_3d(s.v[st][0], &map_v, 0, j * kTileN, kvh, &s.v_full[st]);
+                tc::tma_load_3d(s.v[st][1], &map_v, 64, j * kTileN, kvh, &s.v_full[st]);
             }
         }
-        const uint16_t *Kb = sK + (kb & 1) * kBN * kD;
-        const uint16_t *Vb = sV + (kb & 1) * kBN * kD;
-        // S = Q K^T: 16 rows x 64 keys per warp
-        float s[8][4];
+        __syncwarp();
+    } else if (warp == 1) {
+        // ---------------- MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t id_s = tc::idesc_f16(kTileM, kTileN, false, false);
+            constexpr uint32_t id_pv = tc::idesc_f16(kTileM, kD, false, true);
+            bool ok = fa_wait(s, &s.q_full, 0);
+            for (int j = 0; ok && j <= nkb; ++j) {
+                if (j < nkb) {
+                    const int st = j & 1;
+                    if (!fa_wait(s, &s.k_full[st], (j >> 1) & 1)) break;
+                    if (j >= 2 && !fa_wait(s, &s.s_empty[st], ((j - 2) >> 1) & 1)) break;
+                    tc::fence_after_sync();
 #pragma unroll
-        for (int nt = 0; nt < 8; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-#pragma unroll
-            for (int np = 0; np < 4; ++np) {   // pairs of 8-key n-tiles
-                uint32_t bf[4];
-                const int r = 16 * np + (lane & 7) + 8 * (lane >> 4);
-                const int c = 16 * kk + 8 * ((lane >> 3) & 1);
-                ldmatrix_x4(bf, smem_addr(Kb + swz(r, c)));
-                mma16816(s[2 * np], qf[kk], bf[0], bf[1]);
-                mma16816(s[2 * np + 1], qf[kk], bf[2], bf[3]);
-            }
-        }
-        // online softmax (log2 domain), causal mask on the diagonal block
-        const bool diag = (kb == qt);
-        float mx[2] = {-INFINITY, -INFINITY};
-#pragma unroll
-        for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                float x = s[nt][i] * a.scale_log2;
-                if (diag) {
-                    const int key = kb * kBN + 8 * nt + 2 * t + (i & 1);
-                    const int row = row_g + 8 * (i >> 1);
-                    if (key > row) x = -INFINITY;
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const uint64_t ad = tc::sdesc_sw128(smem_addr(s.q[kk >> 2]) + (kk & 3) * 32, 16, 1024);
+                        const uint64_t bd = tc::sdesc_sw128(smem_addr(s.k[st][kk >> 2]) + (kk & 3) * 32, 16, 1024);
+                        tc::mma_ss(tmem + kColS + st * kTileN, ad, bd, id_s, kk > 0);
+                    }
+                    tc::commit(&s.s_full[st]);
+                    tc::commit(&s.k_empty[st]);
                 }
-                s[nt][i] = x;
-                mx[i >> 1] = fmaxf(mx[i >> 1], x);
-            }
-        float alpha[2];
+                if (j >= 1) {
+                    const int i = j - 1, st = i & 1;
+                    if (!fa_wait(s, &s.p_full[st], (i >> 1) & 1)) break;
+                    if (!fa_wait(s, &s.v_full[st], (i >> 1) & 1)) break;
+                    tc::fence_after_sync();
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-            mx[e] = fmaxf(mx[e], __shfl_xor_sync(0xffffffffu, mx[e], 1));
-            mx[e] = fmaxf(mx[e], __shfl_xor_sync(0xffffffffu, mx[e], 2));
-            const float mn = fmaxf(m[e], mx[e]);
-            alpha[e] = exp2f(m[e] - mn);
-            m[e] = mn;
-            l[e] *= alpha[e];
-            lr[e] *= alpha[e];
-        }
-        uint32_t pf[4][4];   // P as the A operand of P V: 4 k-chunks of 16 keys
-        float ls[2] = {0.f, 0.f}, lrs[2] = {0.f, 0.f};
-#pragma unroll
-        for (int nt = 0; nt < 8; ++nt) {
-            const float p0 = exp2f(s[nt][0] - m[0]), p1 = exp2f(s[nt][1] - m[0]);
-            const float p2 = exp2f(s[nt][2] - m[1]), p3 = exp2f(s[nt][3] - m[1]);
-            const uint32_t h01 = pack_half2(p0, p1), h23 = pack_half2(p2, p3);
-            const float2 f01 = unpack_half2(h01), f23 = unpack_half2(h23);
-            ls[0] += p0 + p1;
-            ls[1] += p2 + p3;
-            lrs[0] += f01.x + f01.y;
-            lrs[1] += f23.x + f23.y;
-            pf[nt >> 1][(nt & 1) * 2 + 0] = h01;
-            pf[nt >> 1][(nt & 1) * 2 + 1] = h23;
-        }
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-            ls[e] += __shfl_xor_sync(0xffffffffu, ls[e], 1);
-            ls[e] += __shfl_xor_sync(0xffffffffu, ls[e], 2);
-            lrs[e] += __shfl_xor_sync(0xffffffffu, lrs[e], 1);
-            lrs[e] += __shfl_xor_sync(0xffffffffu, lrs[e], 2);
-            l[e] += ls[e];
-            lr[e] += lrs[e];
-        }
-#pragma unroll
-        for (int dt = 0; dt < 16; ++dt) {
-            oacc[dt][0] *= alpha[0];
-            oacc[dt][1] *= alpha[0];
-            oacc[dt][2] *= alpha[1];
-            oacc[dt][3] *= alpha[1];
-        }
-        // O += P V
-#pragma unroll
-        for (int kc = 0; kc < 4; ++kc) {
-            // pf[kc] holds {n-tile 2kc rows g / g+8, n-tile 2kc+1 rows g / g+8}; reorder to A layout
-            const uint32_t af[4] = {pf[kc][0], pf[kc][1], pf[kc][2], pf[kc][3]};
-#pragma unroll
-            for (int dp = 0; dp < 8; ++dp) {   // pairs of 8-wide d tiles
-                uint32_t bf[4];
-                const int r = 16 * kc + (lane & 7) + 8 * ((lane >> 3) & 1);
-                const int c = 16 * dp + 8 * (lane >> 4);
-                ldmatrix_x4_t(bf, smem_addr(Vb + swz(r, c)));
-                mma16816(oacc[2 * dp], af, bf[0], bf[1]);
-                mma16816(oacc[2 * dp + 1], af, bf[2], bf[3]);
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const uint64_t bd = tc::sdesc_sw128(smem_addr(s.v[st][0]) + kk * 2048, 2 * kTileN * 64, 1024);
+                        tc::mma_ts(tmem + kColO, tmem + kColP + st * 64 + kk * 8, bd, id_pv, (i > 0) || (kk > 0));
+                    }
+                    tc::commit(&s.o_done);
+                    tc::commit(&s.v_empty[st]);
+                }
             }
         }
-    }
-
-    // epilogue: O / l_rounded -> fp16 via shared memory; window-row LSE
-    __syncthreads();
-    const float inv0 = 1.f / lr[0], inv1 = 1.f / lr[1];
+        __syncwarp();
+    } else {
+        // ---------------- softmax warps
+        const int r = 32 * (warp & 3) + lane;   // row within the tile = TMEM lane
+        const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
+        const float sc = a.scale_log2;
+        float m_ref = -INFINITY;
+        // l: sum of the fp32 probabilities (for the log-sum-exp); lr: sum of
+        // their fp16 roundings, the weights P V actually applied (normalises O,
+        // so each output row is a convex combination of value rows)
+        unsigned long long l2a = 0ull, l2b = 0ull, lr2a = 0ull, lr2b = 0ull;
+        bool ok = true;
+        for (int j = 0; j < nkb; ++j) {
+            const int st = j & 1;
+            ok = __all_sync(0xffffffffu, fa_wait(s, &s.s_full[st], (j >> 1) & 1));
+            if (!ok) break;
+            tc::fence_after_sync();
+            uint32_t x[128];
 #pragma unroll
-    for (int dt = 0; dt < 16; ++dt) {
-        const int rr = 16 * warp + g;
-        const int c = 8 * dt + 2 * t;
-        *reinterpret_cast<uint32_t *>(sQ + swz(rr, c)) = pack_half2(oacc[dt][0] * inv0, oacc[dt][1] * inv0);
-        *reinterpret_cast<uint32_t *>(sQ + swz(rr + 8, c)) = pack_half2(oacc[dt][2] * inv1, oacc[dt][3] * inv1);
-    }
-    if (t == 0) {
+            for (int c = 0; c < 4; ++c)
+                tc::tmem_ld32(tmem + lane_off + kColS + st * kTileN + 32 * c,
+                              *reinterpret_cast<uint32_t(*)[32]>(&x[32 * c]));
+            tc::wait_ld();
+            tc::fence_before_sync();
+            tc::mbar_arrive(&s.s_empty[st]);
+            if (j == qt) {   // diagonal block: key c > row r is in the future
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-            const int row = row_g + 8 * e;
-            if (row < a.T && row >= a.T - a.W)
-                a.lse2[(size_t)bh * a.W + (row - (a.T - a.W))] = m[e] + log2f(l[e]);
+                for (int c = 0; c < 128; ++c)
+                    if (c > r) x[c] = __float_as_uint(-INFINITY);
+            }
+            float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < 128; c += 8) {
+                mx0 = fmax3(mx0, __uint_as_float(x[c]), __uint_as_float(x[c + 1]));
+                mx1 = fmax3(mx1, __uint_as_float(x[c + 2]), __uint_as_float(x[c + 3]));
+                mx2 = fmax3(mx2, __uint_as_float(x[c + 4]), __uint_as_float(x[c + 5]));
+                mx3 = fmax3(mx3, __uint_as_float(x[c + 6]), __uint_as_float(x[c + 7]));
+            }
+            const float mxs = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sc;
+            float alpha = 1.f;
+            const bool grow = mxs > m_ref + kLazyMax;
+            if (grow) {
+                alpha = ex2(m_ref - mxs);
+                m_ref = mxs;
+                const unsigned long long al2 = f2pack(alpha, alpha);
+                l2a = fmul2(l2a, al2);
+                l2b = fmul2(l2b, al2);
+                lr2a = fmul2(lr2a, al2);
+                lr2b = fmul2(lr2b, al2);
+            }
+            const unsigned long long sc2 = f2pack(sc, sc), nm2 = f2pack(-m_ref, -m_ref);
+            uint32_t p[64];
+#pragma unroll
+            for (int c = 0; c < 64; ++c) {
+                float e0, e1;
+                f2unpack(ffma2(f2pack(__uint_as_float(x[2 * c]), __uint_as_float(x[2 * c + 1])), sc2, nm2), e0, e1);
+                const float p0 = ex2(e0), p1 = ex2(e1);
+                p[c] = pack_half2(p0, p1);
+                const float2 pr = unpack_half2(p[c]);
+                if (c & 1) {
+                    l2b = fadd2(l2b, f2pack(p0, p1));
+                    lr2b = fadd2(lr2b, f2pack(pr.x, pr.y));
+                } else {
+                    l2a = fadd2(l2a, f2pack(p0, p1));
+                    lr2a = fadd2(lr2a, f2pack(pr.x, pr.y));
+                }
+            }
+            tc::tmem_st32(tmem + lane_off + kColP + st * 64, *reinterpret_cast<uint32_t(*)[32]>(&p[0]));
+            tc::tmem_st32(tmem + lane_off + kColP + st * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&p[32]));
+            tc::wait_st();
+            if (j > 0) {
+                ok = __all_sync(0xffffffffu, fa_wait(s, &s.o_done, (j - 1) & 1));
+                if (!ok) break;
+                tc::fence_after_sync();
+                if (__any_sync(0xffffffffu, grow)) {   // O of this warp's rows *= alpha
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        uint32_t o[32];
+                        tc::tmem_ld32(tmem + lane_off + kColO + 32 * c, o);
+                        tc::wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+                        tc::tmem_st32(tmem + lane_off + kColO + 32 * c, o);
+                    }
+                    tc::wait_st();
+                }
+            }
+            tc::fence_before_sync();
+            tc::mbar_arrive(&s.p_full[st]);
+        }
+        // ---------------- epilogue: O / l -> fp16 -> swizzled smem (the Q tile) -> TMA store
+        if (ok) ok = __all_sync(0xffffffffu, fa_wait(s, &s.o_done, (nkb - 1) & 1));
+        if (ok) {
+            tc::fence_after_sync();
+            float la, lb, ra, rb;
+            f2unpack(fadd2(l2a, l2b), la, lb);
+            f2unpack(fadd2(lr2a, lr2b), ra, rb);
+            const float l = la + lb;
+            const float inv = 1.f / (ra + rb);
+            const int row = qt * kTileM + r;
+            if (row < a.T && row >= a.T - a.W) a.lse2[(size_t)bh * a.W + (row - (a.T - a.W))] = m_ref + log2f(l);
+            unsigned char *qbytes = reinterpret_cast<unsigned char *>(s.q);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                uint32_t o[32];
+                tc::tmem_ld32(tmem + lane_off + kColO + 32 * c, o);
+                tc::wait_ld();
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {   // 16-byte chunk: d = 32c + 8u .. +7
+                    const int d = 32 * c + 8 * u;
+                    const int kb = d >> 6, ch = (d & 63) >> 3;
+                    uint4 w;
+                    w.x = pack_half2(__uint_as_float(o[8 * u + 0]) * inv, __uint_as_float(o[8 * u + 1]) * inv);
+                    w.y = pack_half2(__uint_as_float(o[8 * u + 2]) * inv, __uint_as_float(o[8 * u + 3]) * inv);
+                    w.z = pack_half2(__uint_as_float(o[8 * u + 4]) * inv, __uint_as_float(o[8 * u + 5]) * inv);
+                    w.w = pack_half2(__uint_as_float(o[8 * u + 6]) * inv, __uint_as_float(o[8 * u + 7]) * inv);
+                    *reinterpret_cast<uint4 *>(qbytes + kb * (kTileM * 128) + r * 128 + ((ch ^ (r & 7)) << 4)) = w;
+                }
+            }
+            tc::fence_proxy_async_smem();
+        }
+        asm volatile("bar.sync 1, 128;\n" ::: "memory");
+        if (ok && warp == 2 && lane == 0) {
+            tc::tma_store_3d(&map_o, s.q[0], 0, qt * kTileM, bh);
+            tc::tma_store_3d(&map_o, s.q[1], 64, qt * kTileM, bh);
+            tc::bulk_commit_group();
+            tc::bulk_wait_all();
         }
     }
+    tc::fence_before_sync();
     __syncthreads();
-    uint16_t *og = a.o + (size_t)bh * a.T * kD;
-    for (int e = tid; e < kBM * 16; e += 128) {
-        const int r = e >> 4, ch = e & 15;
-        if (q0 + r < a.T)
-            *reinterpret_cast<uint4 *>(og + (size_t)(q0 + r) * kD + ch * 8) =
-                *reinterpret_cast<const uint4 *>(sQ + swz(r, ch * 8));
-    }
+    tc::fence_after_sync();
+    if (warp == 1) tc::tmem_dealloc(tmem, 512);
 }
 
 // ---------------------------------------------------------------- kernel 2
@@ -229,7 +340,7 @@ struct ScoreArgs {
 };
 
 __global__ void __launch_bounds__(128) window_score_kernel(const ScoreArgs a) {
-    extern __shared__ __align__(128) unsigned char smem_raw[];
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
     const int gq = a.Hq / a.Hkv;
     const int nrows = gq * a.W;                       // window rows of this KV head
     const int nrows8 = (nrows + 7) / 8 * 8;
@@ -317,27 +428,57 @@ __global__ void __launch_bounds__(128) window_score_kernel(const ScoreArgs a) {
 bool g_attr_fa = false;
 size_t g_attr_score = 0;
 
+std::mutex g_encode_mu;
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+// [planes][rows][128] fp16, 128-byte swizzled boxes of 64 x 128 rows
+int make_map(CUtensorMap *m, const void *base, int rows, int planes, const char *what) {
+    {
+        std::lock_guard<std::mutex> lk(g_encode_mu);
+        if (!g_encode) {
+            cudaDriverEntryPointQueryResult qr;
+            void *fn = nullptr;
+            if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &qr) != cudaSuccess ||
+                qr != cudaDriverEntryPointSuccess || !fn)
+                return fail(MINIKV_ERR_CUDA, "select_prefill: cuTensorMapEncodeTiled unavailable");
+            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+        }
+    }
+    cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)rows, (cuuint64_t)planes};
+    cuuint64_t strides[2] = {(cuuint64_t)kD * 2, (cuuint64_t)rows * kD * 2};
+    cuuint32_t box[3] = {64, 128, 1}, estr[3] = {1, 1, 1};
+    const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void *>(base), dims, strides, box,
+                                estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(MINIKV_ERR_CUDA, "select_prefill: tensor map for %s (CUresult %d)", what, (int)r);
+    return 0;
+}
+
 }  // namespace
 
 size_t prefill_workspace_bytes(int B, int Hq, int W) { return ((size_t)B * Hq * W * 4 + 255) / 256 * 256; }
 
 int prefill_launch(const uint16_t *q, const uint16_t *k, const uint16_t *v, int B, int Hq, int Hkv, int T, int W,
                    float sm_scale, uint16_t *o, float *scores, void *ws, cudaStream_t stream) {
+    CUtensorMap mq, mk, mv, mo;
+    int rc;
+    if ((rc = make_map(&mq, q, T, B * Hq, "q")) || (rc = make_map(&mk, k, T, B * Hkv, "k")) ||
+        (rc = make_map(&mv, v, T, B * Hkv, "v")) || (rc = make_map(&mo, o, T, B * Hq, "o")))
+        return rc;
     FaArgs fa;
-    fa.q = q; fa.k = k; fa.v = v; fa.o = o;
     fa.lse2 = static_cast<float *>(ws);
     fa.Hq = Hq; fa.Hkv = Hkv; fa.T = T; fa.W = W;
+    fa.nqt = (T + kTileM - 1) / kTileM;
     fa.scale_log2 = sm_scale * kLog2e;
-    const size_t fa_smem = (size_t)(kBM + 4 * kBN) * kD * 2;
+    const size_t fa_smem = sizeof(FaSmem) + 1024;
     if (!g_attr_fa) {
-        if (cudaFuncSetAttribute(fa_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fa_smem) !=
+        if (cudaFuncSetAttribute(fa_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fa_smem) !=
             cudaSuccess)
             return check_launch("select_prefill: attribute");
         g_attr_fa = true;
     }
-    const int nqt = (T + kBM - 1) / kBM;
-    fa_fwd_kernel<<<dim3(nqt, B * Hq), 128, fa_smem, stream>>>(fa);
-    int rc = check_launch("select_prefill: flash attention");
+    fa_tc_kernel<<<(unsigned)(fa.nqt * B * Hq), kFaThreads, fa_smem, stream>>>(mq, mk, mv, mo, fa);
+    rc = check_launch("select_prefill: flash attention");
     if (rc) return rc;
 
     ScoreArgs sa;

@@ -118,13 +118,15 @@ MINIKV_API int minikv_quant_pack(minikv_cache *c, const uint16_t *k, const uint1
  *   scores [B, Hkv, T] fp32: scores[j] = sum over the Hq/Hkv query heads of the
  *       KV head and over the last W rows i in [T-W, T) of the softmax
  *       probability P[i, j] (0 where j > i).
- * Pass 1 is a causal flash-attention forward that also records the row
+ * Pass 1 is a causal flash-attention forward on the tcgen05 tensor cores
+ * (128-row query tiles, operands brought in by TMA) that also records the row
  * log-sum-exp of the window rows in `ws`; pass 2 (the second kernel) recomputes
  * the window rows' probabilities from it and sums them per key.
+ *   sm_scale > 0 (the usual 1/sqrt(D)).
  *   ws: device scratch of minikv_workspace_size(MINIKV_OP_SELECT_PREFILL, ...)
  *       bytes, no initial contents required.
- * Errors: INVALID_ARG (null, W < 1, W > T, Hq % Hkv, ws too small),
- * UNSUPPORTED (D != 128).
+ * Errors: INVALID_ARG (null, W < 1, W > T, Hq % Hkv, sm_scale <= 0, ws too
+ * small), UNSUPPORTED (D != 128), CUDA (tensor-map encoding or launch failed).
  */
 MINIKV_API int minikv_select_prefill(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                           int B, int Hq, int Hkv, int T, int D, int W, float sm_scale,

@@ -62,16 +62,22 @@ def test_quant_pack_bitexact(B, H, N, G, Gv, R, cap):
 
 # ------------------------------------------------------- select prefill
 
-@pytest.mark.parametrize("B,Hq,Hkv,T,W", [
+@pytest.mark.parametrize("B,Hq,Hkv,T,W,kind", [(c + ("plain",))[:6] for c in [
     (1, 4, 4, 512, 32),      # tiny single layer
     (1, 8, 2, 300, 17),      # GQA, ragged tail
     (2, 2, 1, 130, 130),     # window = whole prompt
     (1, 1, 1, 1, 1),
     (1, 4, 1, 200, 32),      # g = 4
-])
-def test_select_prefill_vs_oracle(B, Hq, Hkv, T, W):
+    (1, 2, 1, 1000, 32),     # 8 query tiles, key-block stages reused
+    (2, 4, 2, 2100, 64),     # 17 tiles, ragged last tile
+    (1, 2, 2, 1500, 32, "ramp"),   # key norms growing with position: the running max moves late
+]])
+def test_select_prefill_vs_oracle(B, Hq, Hkv, T, W, kind):
     q = synth.normal_fp16((B, Hq, T, 128), synth.seed_of(7, T, synth.T_Q), DEV)
     k, v = _kv(B, Hkv, T, 7 + T)
+    if kind == "ramp":
+        ramp = 1.0 + 4.0 * torch.arange(T, device=DEV, dtype=torch.float32) / T
+        k = (k.float() * ramp[None, None, :, None]).half()
     o, scores = mk.select_prefill(q, k, v, W)
     torch.cuda.synchronize()
     outs, sref = prefill_reference(q, k, v, W, TAU)
