@@ -47,29 +47,33 @@ __device__ __forceinline__ void load_tile(uint16_t *tile, const uint16_t *g, int
 
 // ---------------------------------------------------------------- kernel 1
 //
-// One CTA = one 128-row query tile of one (sequence, query head); 6 warps:
-//   warp 0      TMA producer: the Q tile once, then K_j / V_j into 2 stages;
+// One CTA = one 128-row query tile of one (sequence, query head); 7 warps:
+//   warp 0      TMA producer of the Q tile, then K_j into 3 stages;
 //   warp 1      TMEM owner and the single thread issuing tcgen05.mma;
-//   warps 2..5  softmax: thread = query row = TMEM lane (warp w reads lanes
+//   warp 2      TMA producer of V_j into 2 stages;
+//   warps 3..6  softmax: thread = query row = TMEM lane (warp w reads lanes
 //               32*(w%4) .. +31), plus the O rescale and the epilogue.
 // Tensor memory (512 columns): S_0, S_1 fp32 [128 x 128] at 0 / 128; O fp32 at
 // 256; P_0, P_1 (fp16 pairs, the A operand of P V) at 384 / 448.
-// Issue order S_0, S_1, PV_0, S_2, PV_1, ... lets the tensor pipe compute
-// PV_{j-1} and S_{j+1} while the softmax warps work on S_j.
+// Issue order S_0, S_1, then (PV_j interleaved with S_{j+2}) as soon as P_j
+// is written.  MMAs into one accumulator wait for each other (about 200 cycles
+// each on B200), so two independent chains in flight roughly double the
+// tensor-pipe throughput; meanwhile the softmax warps work on S_{j+1}.
 // The running max is lazy: a row's reference max moves only when a new score
 // exceeds it by more than 2^8 (p <= 256 stays exact enough in fp16), so O is
 // rescaled rarely; l and O always refer to the same reference.
 constexpr int kTileM = 128, kTileN = 128;
-constexpr int kFaThreads = 192;
+constexpr int kKStages = 3, kVStages = 2;
+constexpr int kFaThreads = 224;
 constexpr uint32_t kColS = 0, kColO = 256, kColP = 384;
 constexpr float kLazyMax = 8.f;
 
 struct FaSmem {
     uint16_t q[2][kTileM * 64];        // K-blocks of 64 fp16, 128-byte swizzle
-    uint16_t k[2][2][kTileN * 64];     // [stage][K-block]
-    uint16_t v[2][2][kTileN * 64];     // [stage][64-wide d block]: MN-major B of P V
-    uint64_t q_full, k_full[2], k_empty[2], v_full[2], v_empty[2];
-    uint64_t s_full[2], s_empty[2], p_full[2], o_done;
+    uint16_t k[kKStages][2][kTileN * 64];   // [stage][K-block]
+    uint16_t v[kVStages][2][kTileN * 64];   // [stage][64-wide d block]: MN-major B of P V
+    uint64_t q_full, k_full[kKStages], k_empty[kKStages], v_full[kVStages], v_empty[kVStages];
+    uint64_t s_full[2], p_full[2], o_done[2];
     uint32_t tmem_base;
     int abort;
 };
@@ -117,16 +121,19 @@ __global__ void __launch_bounds__(kFaThreads, 1)
 
     if (tid == 0) {
         mbar_init(&s.q_full, 1);
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < kKStages; ++i) {
             mbar_init(&s.k_full[i], 1);
             mbar_init(&s.k_empty[i], 1);
+        }
+        for (int i = 0; i < kVStages; ++i) {
             mbar_init(&s.v_full[i], 1);
             mbar_init(&s.v_empty[i], 1);
-            mbar_init(&s.s_full[i], 1);
-            mbar_init(&s.s_empty[i], 128);
-            mbar_init(&s.p_full[i], 128);
         }
-        mbar_init(&s.o_done, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&s.s_full[i], 1);
+            mbar_init(&s.p_full[i], 128);
+            mbar_init(&s.o_done[i], 1);
+        }
         s.abort = 0;
         fence_mbar_init();
     }
@@ -146,15 +153,23 @@ __global__ void __launch_bounds__(kFaThreads, 1)
             tc::tma_load_3d(s.q[0], &map_q, 0, qt * kTileM, bh, &s.q_full);
             tc::tma_load_3d(s.q[1], &map_q, 64, qt * kTileM, bh, &s.q_full);
             for (int j = 0; j < nkb; ++j) {
-                const int st = j & 1;
-                if (j >= 2 && !fa_wait(s, &s.k_empty[st], ((j - 2) >> 1) & 1)) break;
-                mbar_arrive_expect_tx(&s.k_full[st], 2 * kTileN * 128);
-                tc::tma_load_3d(s.k[st][0], &map_k, 0, j * kTileN, kvh, &s.k_full[st]);
-                tc::tma_load_3d(s.k[st][1], &map_k, 64, j * kTileN, kvh, &s.k_full[st]);
-                if (j >= 2 && !fa_wait(s, &s.v_empty[st], ((j - 2) >> 1) & 1)) break;
-                mbar_arrive_expect_tx(&s.v_full[st], 2 * kTileN * 128);
-                tc::tma_load_3d(s.v[st][0], &map_v, 0, j * kTileN, kvh, &s.v_full[st]);
-                tc::tma_load_3d(s.v[st][1], &map_v, 64, j * kTileN, kvh, &s.v_full[st]);
+                const int ks = j % kKStages;
+                if (j >= kKStages && !fa_wait(s, &s.k_empty[ks], (j / kKStages - 1) & 1)) break;
+                mbar_arrive_expect_tx(&s.k_full[ks], 2 * kTileN * 128);
+                tc::tma_load_3d(s.k[ks][0], &map_k, 0, j * kTileN, kvh, &s.k_full[ks]);
+                tc::tma_load_3d(s.k[ks][1], &map_k, 64, j * kTileN, kvh, &s.k_full[ks]);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 2) {
+        // ---------------- V producer (its own thread: a V slot frees later than a K slot)
+        if (lane == 0) {
+            for (int j = 0; j < nkb; ++j) {
+                const int vs = j % kVStages;
+                if (j >= kVStages && !fa_wait(s, &s.v_empty[vs], (j / kVStages - 1) & 1)) break;
+                mbar_arrive_expect_tx(&s.v_full[vs], 2 * kTileN * 128);
+                tc::tma_load_3d(s.v[vs][0], &map_v, 0, j * kTileN, kvh, &s.v_full[vs]);
+                tc::tma_load_3d(s.v[vs][1], &map_v, 64, j * kTileN, kvh, &s.v_full[vs]);
             }
         }
         __syncwarp();
@@ -163,34 +178,51 @@ __global__ void __launch_bounds__(kFaThreads, 1)
         if (lane == 0) {
             constexpr uint32_t id_s = tc::idesc_f16(kTileM, kTileN, false, false);
             constexpr uint32_t id_pv = tc::idesc_f16(kTileM, kD, false, true);
-            bool ok = fa_wait(s, &s.q_full, 0);
-            for (int j = 0; ok && j <= nkb; ++j) {
-                if (j < nkb) {
-                    const int st = j & 1;
-                    if (!fa_wait(s, &s.k_full[st], (j >> 1) & 1)) break;
-                    if (j >= 2 && !fa_wait(s, &s.s_empty[st], ((j - 2) >> 1) & 1)) break;
-                    tc::fence_after_sync();
+            auto s_desc = [&](int ks, int kk, uint64_t &ad, uint64_t &bd) {
+                ad = tc::sdesc_sw128(smem_addr(s.q[kk >> 2]) + (kk & 3) * 32, 16, 1024);
+                bd = tc::sdesc_sw128(smem_addr(s.k[ks][kk >> 2]) + (kk & 3) * 32, 16, 1024);
+            };
+            auto issue_s = [&](int j) {   // S_j alone (the first two blocks)
+                const int st = j & 1, ks = j % kKStages;
+                if (!fa_wait(s, &s.k_full[ks], (j / kKStages) & 1)) return false;
+                tc::fence_after_sync();
 #pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {
-                        const uint64_t ad = tc::sdesc_sw128(smem_addr(s.q[kk >> 2]) + (kk & 3) * 32, 16, 1024);
-                        const uint64_t bd = tc::sdesc_sw128(smem_addr(s.k[st][kk >> 2]) + (kk & 3) * 32, 16, 1024);
+                for (int kk = 0; kk < 8; ++kk) {
+                    uint64_t ad, bd;
+                    s_desc(ks, kk, ad, bd);
+                    tc::mma_ss(tmem + kColS + st * kTileN, ad, bd, id_s, kk > 0);
+                }
+                tc::commit(&s.s_full[st]);
+                tc::commit(&s.k_empty[ks]);
+                return true;
+            };
+            bool ok = fa_wait(s, &s.q_full, 0) && issue_s(0) && (nkb < 2 || issue_s(1));
+            // P_j V_j and S_{j+2} (same S / P / K / V slot st) go out interleaved:
+            // two independent accumulator chains keep the tensor pipe busy.
+            // The commit after the pair therefore also tells the softmax of
+            // block j+2 that P_j V_j is complete.
+            for (int j = 0; ok && j < nkb; ++j) {
+                const int st = j & 1, vs = j % kVStages, ks = (j + 2) % kKStages;
+                const bool s_next = j + 2 < nkb;
+                if (!fa_wait(s, &s.p_full[st], (j >> 1) & 1)) break;
+                if (!fa_wait(s, &s.v_full[vs], (j / kVStages) & 1)) break;
+                if (s_next && !fa_wait(s, &s.k_full[ks], ((j + 2) / kKStages) & 1)) break;
+                tc::fence_after_sync();
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint64_t vd = tc::sdesc_sw128(smem_addr(s.v[vs][0]) + kk * 2048, 2 * kTileN * 64, 1024);
+                    tc::mma_ts(tmem + kColO, tmem + kColP + st * 64 + kk * 8, vd, id_pv, (j > 0) || (kk > 0));
+                    if (s_next) {
+                        uint64_t ad, bd;
+                        s_desc(ks, kk, ad, bd);
                         tc::mma_ss(tmem + kColS + st * kTileN, ad, bd, id_s, kk > 0);
                     }
-                    tc::commit(&s.s_full[st]);
-                    tc::commit(&s.k_empty[st]);
                 }
-                if (j >= 1) {
-                    const int i = j - 1, st = i & 1;
-                    if (!fa_wait(s, &s.p_full[st], (i >> 1) & 1)) break;
-                    if (!fa_wait(s, &s.v_full[st], (i >> 1) & 1)) break;
-                    tc::fence_after_sync();
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {
-                        const uint64_t bd = tc::sdesc_sw128(smem_addr(s.v[st][0]) + kk * 2048, 2 * kTileN * 64, 1024);
-                        tc::mma_ts(tmem + kColO, tmem + kColP + st * 64 + kk * 8, bd, id_pv, (i > 0) || (kk > 0));
-                    }
-                    tc::commit(&s.o_done);
-                    tc::commit(&s.v_empty[st]);
+                tc::commit(&s.o_done[st]);
+                tc::commit(&s.v_empty[vs]);
+                if (s_next) {
+                    tc::commit(&s.s_full[st]);
+                    tc::commit(&s.k_empty[ks]);
                 }
             }
         }
@@ -217,8 +249,6 @@ __global__ void __launch_bounds__(kFaThreads, 1)
                 tc::tmem_ld32(tmem + lane_off + kColS + st * kTileN + 32 * c,
                               *reinterpret_cast<uint32_t(*)[32]>(&x[32 * c]));
             tc::wait_ld();
-            tc::fence_before_sync();
-            tc::mbar_arrive(&s.s_empty[st]);
             if (j == qt) {   // diagonal block: key c > row r is in the future
 #pragma unroll
                 for (int c = 0; c < 128; ++c)
@@ -264,28 +294,28 @@ __global__ void __launch_bounds__(kFaThreads, 1)
             tc::tmem_st32(tmem + lane_off + kColP + st * 64, *reinterpret_cast<uint32_t(*)[32]>(&p[0]));
             tc::tmem_st32(tmem + lane_off + kColP + st * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&p[32]));
             tc::wait_st();
-            if (j > 0) {
-                ok = __all_sync(0xffffffffu, fa_wait(s, &s.o_done, (j - 1) & 1));
+            // O of this warp's rows *= alpha, once P_{j-1} V_{j-1} has landed in O.
+            // (P_j over P_{j-2} needs no wait: S_j's commit covered P_{j-2} V_{j-2}.)
+            if (j > 0 && __any_sync(0xffffffffu, grow)) {
+                ok = __all_sync(0xffffffffu, fa_wait(s, &s.o_done[(j - 1) & 1], ((j - 1) >> 1) & 1));
                 if (!ok) break;
                 tc::fence_after_sync();
-                if (__any_sync(0xffffffffu, grow)) {   // O of this warp's rows *= alpha
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        uint32_t o[32];
-                        tc::tmem_ld32(tmem + lane_off + kColO + 32 * c, o);
-                        tc::wait_ld();
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t o[32];
+                    tc::tmem_ld32(tmem + lane_off + kColO + 32 * c, o);
+                    tc::wait_ld();
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-                        tc::tmem_st32(tmem + lane_off + kColO + 32 * c, o);
-                    }
-                    tc::wait_st();
+                    for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+                    tc::tmem_st32(tmem + lane_off + kColO + 32 * c, o);
                 }
+                tc::wait_st();
             }
             tc::fence_before_sync();
             tc::mbar_arrive(&s.p_full[st]);
         }
         // ---------------- epilogue: O / l -> fp16 -> swizzled smem (the Q tile) -> TMA store
-        if (ok) ok = __all_sync(0xffffffffu, fa_wait(s, &s.o_done, (nkb - 1) & 1));
+        if (ok) ok = __all_sync(0xffffffffu, fa_wait(s, &s.o_done[(nkb - 1) & 1], ((nkb - 1) >> 1) & 1));
         if (ok) {
             tc::fence_after_sync();
             float la, lb, ra, rb;
@@ -316,7 +346,7 @@ __global__ void __launch_bounds__(kFaThreads, 1)
             tc::fence_proxy_async_smem();
         }
         asm volatile("bar.sync 1, 128;\n" ::: "memory");
-        if (ok && warp == 2 && lane == 0) {
+        if (ok && warp == 3 && lane == 0) {
             tc::tma_store_3d(&map_o, s.q[0], 0, qt * kTileM, bh);
             tc::tma_store_3d(&map_o, s.q[1], 64, qt * kTileM, bh);
             tc::bulk_commit_group();
