@@ -39,16 +39,40 @@ if ROOT not in sys.path:
 
 METRIC = "decode attn tokens/s and HBM GB/s (% of peak) over 2-bit KV; prefill select ms"
 
-DECODE = dict(workload="mistral7b_gqa_decode", layers=32, batch=16, q_heads=32, kv_heads=8, head_dim=128,
-              context=32768, keep_pct=20, G=32, Gv=128, R=128)
-PREFILL = dict(workload="llama2_7b_prefill_select", layers=32, batch=1, q_heads=32, kv_heads=32, head_dim=128,
-               prompt=4096, W=32, keep_pct=15, G=32, Gv=128, R=128)
+# Decode workloads (--workload); the first is the default bench line.  keep_pct
+# "pyramid" is the layer-discriminative budget: 30% of the context at layer 0
+# falling linearly to 5% at the last layer.
+DECODE_PRESETS = {
+    "mistral7b_gqa_decode": dict(workload="mistral7b_gqa_decode", layers=32, batch=16, q_heads=32, kv_heads=8,
+                                 head_dim=128, context=32768, keep_pct=20, G=32, Gv=128, R=128),
+    "llama2_13b_decode": dict(workload="llama2_13b_decode", layers=40, batch=8, q_heads=40, kv_heads=40,
+                              head_dim=128, context=16384, keep_pct=15, G=32, Gv=128, R=128),
+    "pyramid_44k_decode": dict(workload="pyramid_44k_decode", layers=32, batch=4, q_heads=32, kv_heads=32,
+                               head_dim=128, context=44000, keep_pct="pyramid", G=32, Gv=128, R=128),
+    # every token kept, only quantized (the KIVI-like point of the method): 32K context
+    "quant_only_32k_decode": dict(workload="quant_only_32k_decode", layers=32, batch=16, q_heads=32, kv_heads=8,
+                                  head_dim=128, context=32768, keep_pct=100, G=32, Gv=128, R=128),
+}
+PREFILL_PRESETS = {
+    "llama2_7b_prefill_select": dict(workload="llama2_7b_prefill_select", layers=32, batch=1, q_heads=32,
+                                     kv_heads=32, head_dim=128, prompt=4096, W=32, keep_pct=15, G=32, Gv=128,
+                                     R=128),
+    "pyramid_44k_prefill_select": dict(workload="pyramid_44k_prefill_select", layers=32, batch=4, q_heads=32,
+                                       kv_heads=32, head_dim=128, prompt=44000, W=32, keep_pct="pyramid", G=32,
+                                       Gv=128, R=128),
+}
+DECODE = dict(DECODE_PRESETS["mistral7b_gqa_decode"])
+PREFILL = dict(PREFILL_PRESETS["llama2_7b_prefill_select"])
 
 BYTES_PER_PACKED = 84     # per token and KV head at D=128, G=32, Gv=128: 64 code + 16 key + 4 value scale/zero
 BYTES_PER_RESIDUAL = 512  # fp16 K + V row
 
 
-def keep_of(T, pct):
+def keep_of(T, pct, layer=0, n_layers=32):
+    """Kept tokens of a layer: pct % of T, or the pyramid budget (30% at layer 0
+    down to 5% at the last layer, linear in the layer index, floor in integers)."""
+    if pct == "pyramid":
+        return (T * (30 * (n_layers - 1) - 25 * layer)) // (100 * (n_layers - 1))
     return T * pct // 100
 
 
@@ -178,10 +202,17 @@ def cpu_tokens_per_s(rate):
     return rate * DECODE["batch"] / units_per_step
 
 
-def decode_config(extra=None):
+def decode_keeps():
+    return [keep_of(DECODE["context"], DECODE["keep_pct"], l, DECODE["layers"]) for l in range(DECODE["layers"])]
+
+
+def decode_config(extra=None, step_bytes=None):
     c = {k: v for k, v in DECODE.items()}
-    c["keep"] = keep_of(DECODE["context"], DECODE["keep_pct"])
-    c["l2"] = "inputs larger than L2: 32 distinct layer caches, 2.52 GB read per step"
+    keeps = decode_keeps()
+    c["keep"] = keeps[0] if len(set(keeps)) == 1 else f"{keeps[0]}..{keeps[-1]} (per layer)"
+    gb = (step_bytes or 0) / 1e9
+    c["l2"] = (f"inputs larger than L2: {DECODE['layers']} distinct layer caches, {gb:.2f} GB read per step"
+               if step_bytes else f"inputs larger than L2: {DECODE['layers']} distinct layer caches")
     if extra:
         c.update(extra)
     return c
@@ -219,18 +250,21 @@ def run_reference(args):
 def make_decode_state(torch, mk, synth, device, warmup, steps):
     L, B, Hq, Hkv = DECODE["layers"], DECODE["batch"], DECODE["q_heads"], DECODE["kv_heads"]
     G, Gv, R = DECODE["G"], DECODE["Gv"], DECODE["R"]
-    N = keep_of(DECODE["context"], DECODE["keep_pct"])
+    keeps = decode_keeps()
     total_steps = warmup + 2 * steps + 2
-    cap = ((N + total_steps) // G + 2) * G
-    ws = torch.zeros(mk.workspace_size(mk.OP_DECODE_ATTN, B, Hq, Hkv, cap + R + G), dtype=torch.uint8,
+    cap_max = ((max(keeps) + total_steps) // G + 2) * G
+    ws = torch.zeros(mk.workspace_size(mk.OP_DECODE_ATTN, B, Hq, Hkv, cap_max + R + G), dtype=torch.uint8,
                      device=device)
+    wid = 4 if DECODE["workload"] == "mistral7b_gqa_decode" else 40 + list(DECODE_PRESETS).index(DECODE["workload"])
     caches = []
     for l in range(L):
+        N = keeps[l]
+        cap = ((N + total_steps) // G + 2) * G
         k = torch.empty((B, Hkv, N, 128), dtype=torch.float16, device=device)
         v = torch.empty_like(k)
         for b in range(B):
-            k[b] = synth.keys_fp16((Hkv, N, 128), synth.seed_of(4, l, synth.T_K, 0, b), device)
-            v[b] = synth.normal_fp16((Hkv, N, 128), synth.seed_of(4, l, synth.T_V, 0, b), device)
+            k[b] = synth.keys_fp16((Hkv, N, 128), synth.seed_of(wid, l, synth.T_K, 0, b), device)
+            v[b] = synth.normal_fp16((Hkv, N, 128), synth.seed_of(wid, l, synth.T_V, 0, b), device)
         c = mk.MiniKVCache(B, Hkv, cap, G=G, Gv=Gv, R=R, Hq=Hq, device=device, ws=ws)
         mk.quant_pack(c, k, v)
         caches.append(c)
@@ -243,9 +277,9 @@ def make_decode_state(torch, mk, synth, device, warmup, steps):
     vnin = torch.empty_like(knin)
     for p in range(P):
         for l in range(L):
-            qin[p, l] = synth.normal_fp16((B, Hq, 128), synth.seed_of(4, l, synth.T_QDEC, p), device)
-            knin[p, l] = synth.keys_fp16((B, Hkv, 128), synth.seed_of(4, l, synth.T_KNEW, p), device)
-            vnin[p, l] = synth.normal_fp16((B, Hkv, 128), synth.seed_of(4, l, synth.T_VNEW, p), device)
+            qin[p, l] = synth.normal_fp16((B, Hq, 128), synth.seed_of(wid, l, synth.T_QDEC, p), device)
+            knin[p, l] = synth.keys_fp16((B, Hkv, 128), synth.seed_of(wid, l, synth.T_KNEW, p), device)
+            vnin[p, l] = synth.normal_fp16((B, Hkv, 128), synth.seed_of(wid, l, synth.T_VNEW, p), device)
     out = torch.empty((L, B, Hq, 128), dtype=torch.float16, device=device)
     return caches, ws, qin, knin, vnin, out
 
@@ -255,47 +289,68 @@ def unit_bytes(c):
 
 
 def run_prefill(torch, mk, synth, device):
-    """Prompt rows on the LLaMA2-7B shape: per layer select_prefill, topk_evict
-    and quant_pack, each timed with CUDA events (3 warm-up layers first)."""
+    """Prompt rows of one prefill workload: per layer select_prefill, topk_evict
+    and quant_pack, each timed with CUDA events (3 warm-up layers first).  A
+    layer's q, k, v are generated (untimed) just before its calls."""
     L, B, H, T, W = PREFILL["layers"], PREFILL["batch"], PREFILL["q_heads"], PREFILL["prompt"], PREFILL["W"]
-    keep = keep_of(T, PREFILL["keep_pct"])
-    qs, ks, vs = [], [], []
-    for l in range(L):
-        qs.append(synth.normal_fp16((B, H, T, 128), synth.seed_of(2, l, synth.T_Q), device))
-        ks.append(synth.keys_fp16((B, H, T, 128), synth.seed_of(2, l, synth.T_K), device))
-        vs.append(synth.normal_fp16((B, H, T, 128), synth.seed_of(2, l, synth.T_V), device))
+    keeps = [keep_of(T, PREFILL["keep_pct"], l, 32) for l in range(L)]
+    wid = 2 if PREFILL["workload"] == "llama2_7b_prefill_select" else 50
+    kmax = min(max(keeps), T)
     ws = torch.empty(mk.workspace_size(mk.OP_SELECT_PREFILL, B, H, H, T, 128, W), dtype=torch.uint8, device=device)
-    o = torch.empty_like(qs[0])
+    q = torch.empty((B, H, T, 128), dtype=torch.float16, device=device)
+    k, v, o = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
     sc = torch.empty((B, H, T), dtype=torch.float32, device=device)
-    idx = torch.empty((B, H, keep), dtype=torch.int32, device=device)
-    kk = torch.empty((B, H, keep, 128), dtype=torch.float16, device=device)
-    vk = torch.empty_like(kk)
-    cache = mk.MiniKVCache(B, H, 640, G=PREFILL["G"], Gv=PREFILL["Gv"], R=PREFILL["R"], device=device)
+    idx_buf = torch.empty(B * H * kmax, dtype=torch.int32, device=device)
+    kk_buf = torch.empty(B * H * kmax * 128, dtype=torch.float16, device=device)
+    vk_buf = torch.empty_like(kk_buf)
+    cap = ((kmax + 2 * PREFILL["G"]) // PREFILL["G"] + 1) * PREFILL["G"]
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)   # twice the L2
+
+    def layer(l, e=None):
+        q.copy_(synth.normal_fp16((B, H, T, 128), synth.seed_of(wid, l, synth.T_Q), device))
+        k.copy_(synth.keys_fp16((B, H, T, 128), synth.seed_of(wid, l, synth.T_K), device))
+        v.copy_(synth.normal_fp16((B, H, T, 128), synth.seed_of(wid, l, synth.T_V), device))
+        n = min(keeps[l], T)
+        idx = idx_buf[:B * H * n].view(B, H, n)   # contiguous views of this layer's size
+        kk = kk_buf[:B * H * n * 128].view(B, H, n, 128)
+        vk = vk_buf[:B * H * n * 128].view(B, H, n, 128)
+        cache = mk.MiniKVCache(B, H, cap, G=PREFILL["G"], Gv=PREFILL["Gv"], R=PREFILL["R"], device=device)
+        cache2 = mk.MiniKVCache(B, H, cap, G=PREFILL["G"], Gv=PREFILL["Gv"], R=PREFILL["R"], device=device)
+        flush.zero_()   # evict the freshly generated inputs from L2 before the timed calls
+        torch.cuda.synchronize()
+        if e is not None:
+            e[0].record()
+        mk.select_prefill(q, k, v, W, o=o, scores=sc, ws=ws)
+        if e is not None:
+            e[1].record()
+        mk.topk_evict(sc, k, v, W, keeps[l], idx=idx, k_kept=kk, v_kept=vk)
+        if e is not None:
+            e[2].record()
+        mk.quant_pack(cache, kk, vk)
+        if e is not None:
+            e[3].record()
+        # the fused form of the last two calls (select -> pack with no fp16 copy of the kept rows)
+        mk.evict_pack(cache2, sc, k, v, W, keeps[l], idx=idx)
+        if e is not None:
+            e[4].record()
+        torch.cuda.synchronize()
+
     for l in range(3):
-        mk.select_prefill(qs[l], ks[l], vs[l], W, o=o, scores=sc, ws=ws)
-        mk.topk_evict(sc, ks[l], vs[l], W, keep, idx=idx, k_kept=kk, v_kept=vk)
-        mk.quant_pack(cache, kk, vk)
-    torch.cuda.synchronize()
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(L)]
+        layer(l)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(L)]
     for l in range(L):
-        e = ev[l]
-        e[0].record()
-        mk.select_prefill(qs[l], ks[l], vs[l], W, o=o, scores=sc, ws=ws)
-        e[1].record()
-        mk.topk_evict(sc, ks[l], vs[l], W, keep, idx=idx, k_kept=kk, v_kept=vk)
-        e[2].record()
-        mk.quant_pack(cache, kk, vk)
-        e[3].record()
-    torch.cuda.synchronize()
+        layer(l, ev[l])
     sel = sum(e[0].elapsed_time(e[1]) for e in ev)
     top = sum(e[1].elapsed_time(e[2]) for e in ev)
     pk = sum(e[2].elapsed_time(e[3]) for e in ev)
-    flops = L * (2.0 * T * T * 128 * H + 2.0 * W * T * 128 * H)    # causal QK^T + PV, plus the window pass
-    del qs, ks, vs
-    return {"workload": PREFILL["workload"], "config": {**PREFILL, "keep": keep},
+    fused = sum(e[3].elapsed_time(e[4]) for e in ev)
+    flops = L * (2.0 * T * T * 128 * H * B + 2.0 * W * T * 128 * H * B)    # causal QK^T + PV, plus the window pass
+    del q, k, v, o
+    return {"workload": PREFILL["workload"], "config": {**PREFILL, "keep": keeps[0] if len(set(keeps)) == 1 else
+                                                        f"{keeps[0]}..{keeps[-1]} (per layer)"},
             "select_prefill_ms": sel, "select_prefill_ms_per_layer": sel / L,
             "select_prefill_tflops": flops / (sel * 1e-3) / 1e12,
-            "topk_evict_ms": top, "quant_pack_ms": pk, "layers": L}
+            "topk_evict_ms": top, "quant_pack_ms": pk, "evict_pack_ms": fused, "layers": L}
 
 
 def run_gpu(args):
@@ -401,7 +456,7 @@ def run_gpu(args):
         prefill["tensor_frac_of_bf16_peak"] = prefill["select_prefill_tflops"] / pk["bf16"]
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and DECODE["workload"] == "mistral7b_gqa_decode":
         threads = os.cpu_count() or 1
         rate, n, dt = oracle_decode_rate(args.cpu_seconds, threads)
         cpu = {"value": cpu_tokens_per_s(rate), "unit": "tokens/s", "cores": threads, "kind": "oracle",
@@ -416,7 +471,8 @@ def run_gpu(args):
             "metric": METRIC, "value": tok_s, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "u2+f16 (2-bit codes, fp16 scales/residual, fp32 accumulate)",
-            "data": "synthetic", "config": decode_config({"parallelism": f"replicas x{world}"}),
+            "data": "synthetic",
+            "config": decode_config({"parallelism": f"replicas x{world}"}, step_bytes=alg_bytes / args.steps),
             "hbm_gbs": step_gbs, "hbm_frac_of_peak": step_gbs / pk["hbm"],
             "roofline": {"bound": "hbm", "kernel": "decode_kernel", "achieved": achieved, "peak": pk["hbm"],
                          "unit": "GB/s", "frac": achieved / pk["hbm"], "traffic": traffic,
@@ -443,13 +499,22 @@ def main():
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
-    ap.add_argument("--layers", type=int, default=DECODE["layers"],
-                    help="decode layers (fewer only for small profiling runs; the workload has 32)")
-    ap.add_argument("--prefill-layers", type=int, default=PREFILL["layers"],
-                    help="prefill layers (fewer only for small profiling runs; the workload has 32)")
+    ap.add_argument("--workload", default="mistral7b_gqa_decode", choices=list(DECODE_PRESETS),
+                    help="decode workload (the default one carries the bench line's target)")
+    ap.add_argument("--prefill-workload", default="llama2_7b_prefill_select", choices=list(PREFILL_PRESETS))
+    ap.add_argument("--layers", type=int, default=None,
+                    help="decode layers (fewer only for small profiling runs; default: the workload's)")
+    ap.add_argument("--prefill-layers", type=int, default=None,
+                    help="prefill layers (fewer only for small profiling runs; default: the workload's)")
     args = ap.parse_args()
-    DECODE["layers"] = args.layers
-    PREFILL["layers"] = args.prefill_layers
+    DECODE.clear()
+    DECODE.update(DECODE_PRESETS[args.workload])
+    PREFILL.clear()
+    PREFILL.update(PREFILL_PRESETS[args.prefill_workload])
+    if args.layers is not None:
+        DECODE["layers"] = args.layers
+    if args.prefill_layers is not None:
+        PREFILL["layers"] = args.prefill_layers
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     if args.impl == "reference":

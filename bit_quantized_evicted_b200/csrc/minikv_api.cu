@@ -23,7 +23,9 @@ int check_launch(const char *what) {
     return MINIKV_OK;
 }
 
-int pack_launch(minikv_cache *c, const uint16_t *k, const uint16_t *v, int N, cudaStream_t stream);
+int pack_launch(minikv_cache *c, const uint16_t *k, const uint16_t *v, int N, cudaStream_t stream,
+                const int32_t *idx = nullptr, int T = 0);
+int select_launch(const float *scores, int B, int Hkv, int T, int W, int keep, int32_t *idx, cudaStream_t stream);
 int prefill_launch(const uint16_t *q, const uint16_t *k, const uint16_t *v, int B, int Hq, int Hkv, int T, int W,
                    float sm_scale, uint16_t *o, float *scores, void *ws, cudaStream_t stream);
 size_t prefill_workspace_bytes(int B, int Hq, int W);
@@ -179,6 +181,33 @@ int minikv_topk_evict(const float *scores, const uint16_t *k, const uint16_t *v,
         return fail(MINIKV_ERR_INVALID_ARG, "topk_evict: window W=%d above the budget keep=%d", W, keep);
     if ((size_t)B * Hkv > 65535) return fail(MINIKV_ERR_UNSUPPORTED, "topk_evict: B*Hkv above 65535");
     return topk_launch(scores, k, v, B, Hkv, T, W, keep, idx, k_kept, v_kept, static_cast<cudaStream_t>(stream));
+}
+
+int minikv_evict_pack(const float *scores, const uint16_t *k, const uint16_t *v, int B, int Hkv, int T, int D, int W,
+                      int keep, int32_t *idx, minikv_cache *c, void *stream) {
+    g_err[0] = 0;
+    int rc = check_cache(c);
+    if (rc) return rc;
+    if (!scores || !k || !v || !idx) return fail(MINIKV_ERR_INVALID_ARG, "evict_pack: null pointer");
+    if (!aligned16(k) || !aligned16(v))
+        return fail(MINIKV_ERR_INVALID_ARG, "evict_pack: K/V pointers must be 16-byte aligned");
+    if (B < 1 || Hkv < 1 || T < 1 || W < 0 || keep < 1)
+        return fail(MINIKV_ERR_INVALID_ARG, "evict_pack: B=%d Hkv=%d T=%d W=%d keep=%d", B, Hkv, T, W, keep);
+    if (D != kD) return fail(MINIKV_ERR_UNSUPPORTED, "evict_pack: D=%d (only 128)", D);
+    if (B != c->B || Hkv != c->Hkv)
+        return fail(MINIKV_ERR_INVALID_ARG, "evict_pack: B=%d Hkv=%d but the cache has B=%d Hkv=%d", B, Hkv, c->B,
+                    c->Hkv);
+    if (keep < T && W > keep)
+        return fail(MINIKV_ERR_INVALID_ARG, "evict_pack: window W=%d above the budget keep=%d", W, keep);
+    if ((size_t)B * Hkv > 65535) return fail(MINIKV_ERR_UNSUPPORTED, "evict_pack: B*Hkv above 65535");
+    const int n = keep < T ? keep : T;
+    int n_q = 0;
+    if (n >= c->R) n_q = n - (c->R + (n - c->R) % c->G);
+    if (n_q > c->cap) return fail(MINIKV_ERR_CAPACITY, "evict_pack: %d packed tokens exceed cap=%d", n_q, c->cap);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    rc = select_launch(scores, B, Hkv, T, W, keep, idx, s);
+    if (rc) return rc;
+    return pack_launch(c, k, v, n, s, idx, T);
 }
 
 int minikv_decode_attn(minikv_cache *c, const uint16_t *q, const uint16_t *k_new, const uint16_t *v_new, int Hq,

@@ -8,6 +8,11 @@
 // key group x (G tokens, thread = channel) and the same G value tokens (warp =
 // token); the remaining blocks copy residual tokens into ring slots 0..r-1.
 // Memory-bound: 512 B read and 84 B written per packed token and KV head.
+//
+// minikv_evict_pack runs the same kernel with an index list: compacted token
+// t of a unit is then prompt row idx[t] (the kept positions of
+// minikv_topk_evict), read straight from the prompt K/V, so the kept rows are
+// never written out in fp16 (the fused select -> gather -> pack of the path).
 #include "common.cuh"
 
 namespace minikv {
@@ -16,6 +21,8 @@ namespace {
 
 struct PackArgs {
     const uint16_t *k, *v;
+    const int32_t *idx;   // null: rows are contiguous [unit][N]; else row t = prompt row idx[unit][t] of T
+    int T;
     uint32_t *k_codes, *v_codes;
     uint16_t *k_scale, *k_zero, *v_scale, *v_zero;
     uint16_t *k_res, *v_res;
@@ -26,13 +33,16 @@ constexpr int kResPerBlock = 32;   // residual tokens copied per block
 
 __global__ void __launch_bounds__(128) pack_kernel(const PackArgs a) {
     const int unit = blockIdx.y;
-    const uint16_t *ku = a.k + (size_t)unit * a.N * kD;
-    const uint16_t *vu = a.v + (size_t)unit * a.N * kD;
+    const size_t rows = a.idx ? (size_t)a.T : (size_t)a.N;
+    const uint16_t *ku = a.k + (size_t)unit * rows * kD;
+    const uint16_t *vu = a.v + (size_t)unit * rows * kD;
+    const int32_t *iu = a.idx ? a.idx + (size_t)unit * a.N : nullptr;
+    auto src_row = [&](int t) -> size_t { return iu ? (size_t)iu[t] : (size_t)t; };   // compacted -> source row
     if ((int)blockIdx.x < a.n_groups) {
         const int grp = blockIdx.x;
         const int t0 = grp * a.G;
-        auto krow = [&](int t) { return ku + (size_t)(t0 + t) * kD; };
-        auto vrow = [&](int t) { return vu + (size_t)(t0 + t) * kD; };
+        auto krow = [&](int t) { return ku + src_row(t0 + t) * kD; };
+        auto vrow = [&](int t) { return vu + src_row(t0 + t) * kD; };
         const size_t tok = (size_t)unit * a.cap + t0;
         const size_t grow = (size_t)unit * (a.cap / a.G) + grp;
         pack_key_group(krow, a.G, a.k_codes + tok * 8, a.k_scale + grow * kD, a.k_zero + grow * kD);
@@ -44,7 +54,7 @@ __global__ void __launch_bounds__(128) pack_kernel(const PackArgs a) {
         for (int e = threadIdx.x; e < kResPerBlock * 16; e += 128) {
             const int i = i0 + e / 16, ch = e % 16;
             if (i >= a.r) break;
-            const size_t src = (size_t)(a.n_q + i) * kD;
+            const size_t src = src_row(a.n_q + i) * kD;
             const size_t dst = ((size_t)unit * a.ring + i) * kD;
             reinterpret_cast<uint4 *>(a.k_res + dst)[ch] = reinterpret_cast<const uint4 *>(ku + src)[ch];
             reinterpret_cast<uint4 *>(a.v_res + dst)[ch] = reinterpret_cast<const uint4 *>(vu + src)[ch];
@@ -54,7 +64,10 @@ __global__ void __launch_bounds__(128) pack_kernel(const PackArgs a) {
 
 }  // namespace
 
-int pack_launch(minikv_cache *c, const uint16_t *k, const uint16_t *v, int N, cudaStream_t stream) {
+// idx == nullptr: k, v are [B,Hkv,N,D]; else k, v are [B,Hkv,T,D] and row t of
+// unit u is idx[u][t] (idx [B,Hkv,N], ascending positions < T).
+int pack_launch(minikv_cache *c, const uint16_t *k, const uint16_t *v, int N, cudaStream_t stream,
+                const int32_t *idx, int T) {
     int n_q, r;
     if (N >= c->R) {
         r = c->R + (N - c->R) % c->G;
@@ -67,6 +80,7 @@ int pack_launch(minikv_cache *c, const uint16_t *k, const uint16_t *v, int N, cu
         return fail(MINIKV_ERR_CAPACITY, "quant_pack: %d packed tokens exceed cap=%d", n_q, c->cap);
     PackArgs a;
     a.k = k; a.v = v;
+    a.idx = idx; a.T = T;
     a.k_codes = c->k_codes; a.v_codes = c->v_codes;
     a.k_scale = c->k_scale; a.k_zero = c->k_zero; a.v_scale = c->v_scale; a.v_zero = c->v_zero;
     a.k_res = c->k_res; a.v_res = c->v_res;

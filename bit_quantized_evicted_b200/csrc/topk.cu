@@ -166,12 +166,16 @@ __global__ void __launch_bounds__(128) gather_kernel(const GatherArgs a) {
 
 }  // namespace
 
+int select_launch(const float *scores, int B, int Hkv, int T, int W, int keep, int32_t *idx, cudaStream_t stream) {
+    SelArgs sa{scores, idx, T, W, keep};
+    select_kernel<<<B * Hkv, kSelThreads, 0, stream>>>(sa);
+    return check_launch("topk_evict: select");
+}
+
 int topk_launch(const float *scores, const uint16_t *k, const uint16_t *v, int B, int Hkv, int T, int W, int keep,
                 int32_t *idx, uint16_t *k_kept, uint16_t *v_kept, cudaStream_t stream) {
     const int units = B * Hkv;
-    SelArgs sa{scores, idx, T, W, keep};
-    select_kernel<<<units, kSelThreads, 0, stream>>>(sa);
-    int rc = check_launch("topk_evict: select");
+    int rc = select_launch(scores, B, Hkv, T, W, keep, idx, stream);
     if (rc) return rc;
     const int n = keep < T ? keep : T;
     GatherArgs ga{idx, k, v, k_kept, v_kept, T, n};

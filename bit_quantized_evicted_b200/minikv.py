@@ -42,6 +42,7 @@ _SIGS = {
     "minikv_quant_pack": (_I, [ctypes.POINTER(CacheStruct), _P, _P, _I, _P]),
     "minikv_select_prefill": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P, _Z, _P]),
     "minikv_topk_evict": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _Z, _P]),
+    "minikv_evict_pack": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, ctypes.POINTER(CacheStruct), _P]),
     "minikv_decode_attn": (_I, [ctypes.POINTER(CacheStruct), _P, _P, _P, _I, _F, _P, _P, _Z, _P]),
     "minikv_decode_attn_static": (_I, [ctypes.POINTER(CacheStruct), _P, _P, _P, _I, _F, _P, _P]),
     "minikv_workspace_size": (_Z, [_I, _I, _I, _I, _I, _I, _I]),
@@ -213,6 +214,20 @@ def topk_evict(scores: torch.Tensor, k: torch.Tensor, v: torch.Tensor, W: int, k
         B, Hkv, T, D, W, keep, _dev(idx, torch.int32, "idx"), _dev(k_kept, torch.float16, "k_kept"),
         _dev(v_kept, torch.float16, "v_kept"), None, 0, _stream(stream, k.device)))
     return idx, k_kept, v_kept
+
+
+def evict_pack(cache: MiniKVCache, scores: torch.Tensor, k: torch.Tensor, v: torch.Tensor, W: int, keep: int,
+               idx: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """topk_evict + quant_pack in one call: the kept rows of the prompt k, v
+    [B, Hkv, T, D] go straight into the cache; returns idx [B, Hkv, n]."""
+    B, Hkv, T, D = k.shape
+    n = min(keep, T)
+    if idx is None:
+        idx = torch.empty((B, Hkv, n), dtype=torch.int32, device=k.device)
+    _check(lib().minikv_evict_pack(
+        _dev(scores, torch.float32, "scores"), _dev(k, torch.float16, "k"), _dev(v, torch.float16, "v"),
+        B, Hkv, T, D, W, keep, _dev(idx, torch.int32, "idx"), ctypes.byref(cache.c), _stream(stream, k.device)))
+    return idx
 
 
 def decode_attn(cache: MiniKVCache, q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor,

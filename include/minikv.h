@@ -153,6 +153,27 @@ MINIKV_API int minikv_topk_evict(const float *scores, const uint16_t *k, const u
                       void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * minikv_evict_pack -- minikv_topk_evict followed by minikv_quant_pack in one
+ * call, without the fp16 copy of the kept rows in between.
+ * Source: the same passages as the two calls it fuses (glossary "adaptive KV";
+ * 方法论, the compact 2-bit layout): keep by importance, then quantize what is
+ * kept.
+ *   scores [B, Hkv, T] fp32, k, v [B, Hkv, T, D] fp16 (the prompt), as for
+ *   minikv_topk_evict; idx [B, Hkv, n] int32 receives the kept positions
+ *   (n = min(keep, T), ascending).  The kept rows are read straight from k and
+ *   v and packed into *c exactly as minikv_quant_pack(c, k[idx], v[idx], n)
+ *   would pack them (same codes, scales, zeros and residual, bit for bit);
+ *   the cache state is reset the same way.
+ *   B, Hkv must match the cache.  No workspace.
+ * Errors: INVALID_ARG (null, misaligned, keep < 1, W > keep < T, B/Hkv differ
+ * from the cache), UNSUPPORTED (D != 128, bad cache shape), CAPACITY (the
+ * packed part would exceed cap).
+ */
+MINIKV_API int minikv_evict_pack(const float *scores, const uint16_t *k, const uint16_t *v,
+                      int B, int Hkv, int T, int D, int W, int keep,
+                      int32_t *idx, minikv_cache *c, void *stream);
+
+/*
  * minikv_decode_attn -- one decoding step of one layer over the 2-bit cache.
  * Source: abstract ("specialized CUDA kernels ... compatible with
  * FlashAttention"); summary page, 方法论 (the compact 2-bit layout it reads).

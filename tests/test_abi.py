@@ -120,3 +120,23 @@ def test_workspace_sizes():
     assert mk.workspace_size(mk.OP_SELECT_PREFILL, 1, 32, 32, 4096, 128, 32) == 4096
     assert mk.workspace_size(mk.OP_TOPK_EVICT, 1, 32, 32, 4096, 128, 32) == 0
     assert mk.workspace_size(mk.OP_DECODE_ATTN, 16, 32, 8, 6656 + 160, 128) > 16 * 8 * 4
+
+
+def test_evict_pack_argument_errors():
+    L = mk.lib()
+    c = _bound_cache(B=1, Hkv=2, cap=64)
+    p = 1 << 24
+    # B / Hkv must match the cache
+    assert L.minikv_evict_pack(p, p, p, 1, 3, 512, 128, 32, 96, p, ctypes.byref(c), None) == mk.ERR_INVALID_ARG
+    # window above the budget; empty budget; null index list
+    assert L.minikv_evict_pack(p, p, p, 1, 2, 512, 128, 64, 32, p, ctypes.byref(c), None) == mk.ERR_INVALID_ARG
+    assert L.minikv_evict_pack(p, p, p, 1, 2, 512, 128, 32, 0, p, ctypes.byref(c), None) == mk.ERR_INVALID_ARG
+    assert L.minikv_evict_pack(p, p, p, 1, 2, 512, 128, 32, 96, None, ctypes.byref(c), None) == mk.ERR_INVALID_ARG
+    # D != 128
+    assert L.minikv_evict_pack(p, p, p, 1, 2, 512, 96, 32, 96, p, ctypes.byref(c), None) == mk.ERR_UNSUPPORTED
+    # keep 300 of 512 with R=32, G=32 -> 256 packed > cap 64
+    assert L.minikv_evict_pack(p, p, p, 1, 2, 512, 128, 32, 300, p, ctypes.byref(c), None) == mk.ERR_CAPACITY
+    assert b"cap" in L.minikv_last_error_string()
+    # misaligned K
+    assert L.minikv_evict_pack(p, p + 2, p, 1, 2, 512, 128, 32, 96, p, ctypes.byref(c), None) == mk.ERR_INVALID_ARG
+    assert (c.n_packed, c.n_res, c.res_start) == (0, 0, 0)   # the cache state is untouched on error

@@ -90,6 +90,47 @@ def test_select_prefill_vs_oracle(B, Hq, Hkv, T, W, kind):
     np.testing.assert_allclose(sg.sum(-1), W * g, rtol=1e-4)
 
 
+# ------------------------------------------------------- fused evict + pack
+
+@pytest.mark.parametrize("B,H,T,W,keep,G,R", [
+    (1, 4, 512, 32, 256, 32, 32),     # tiny layer, keep 50%
+    (2, 3, 1000, 16, 150, 32, 48),    # ragged residual
+    (1, 2, 300, 32, 300, 64, 128),    # keep = T: every row, G = 64
+    (1, 2, 64, 32, 32, 32, 32),       # only the window, all residual
+])
+def test_evict_pack_matches_topk_then_pack(B, H, T, W, keep, G, R):
+    """evict_pack == quant_pack(topk_evict(...)) bit for bit, and both == the oracle's pack of its selection."""
+    scores = torch.rand((B, H, T), generator=torch.Generator().manual_seed(T + keep), dtype=torch.float32).to(DEV)
+    k, v = _kv(B, H, T, 500 + T)
+    n = min(keep, T)
+    cap = (n // G + 2) * G
+    idx, kk, vk = mk.topk_evict(scores, k, v, W, keep)
+    ref_cache = mk.MiniKVCache(B, H, cap, G=G, R=R)
+    mk.quant_pack(ref_cache, kk, vk)
+    cache = mk.MiniKVCache(B, H, cap, G=G, R=R)
+    idx2 = mk.evict_pack(cache, scores, k, v, W, keep)
+    torch.cuda.synchronize()
+    assert torch.equal(idx, idx2)
+    assert (cache.n_packed, cache.n_res, cache.res_start) == (ref_cache.n_packed, ref_cache.n_res, 0)
+    a, b = cache.arrays(), ref_cache.arrays()
+    nq = cache.n_packed
+    for name in ("k_codes", "v_codes", "v_scale", "v_zero"):
+        assert torch.equal(a[name][:, :, :nq], b[name][:, :, :nq]), name
+    for name in ("k_scale", "k_zero"):
+        assert torch.equal(a[name][:, :, :nq // G], b[name][:, :, :nq // G]), name
+    kr, vr = cache.residual()
+    kr2, vr2 = ref_cache.residual()
+    assert torch.equal(kr, kr2) and torch.equal(vr, vr2)
+    # and against the oracle: its selection on the same scores, its pack of those rows
+    sn = scores.cpu().numpy().astype(np.float64)
+    for b_ in range(B):
+        for h in range(H):
+            sel = O.select(sn[b_, h], W, keep)
+            assert np.array_equal(idx2[b_, h].cpu().numpy(), sel)
+    ref = pack_reference(kk, vk, R, G, 128)
+    compare_cache(cache, ref)
+
+
 # ------------------------------------------------------------- top-k
 
 def _select_ref(scores_np, W, keep):
