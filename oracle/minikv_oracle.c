@@ -31,6 +31,9 @@
  *   O7  16 codes per little-endian 32-bit word, channel 16w+i at bits 2i..2i+1
  *   O8  dequant x^ = c*scale + zero (exact in fp64)
  *   O9  decode: attend over dequantized packed tokens + fp16 residual, fp64
+ *   O10 decode-time attention mass (H2O-style accumulated score): each step
+ *       adds, per cached token, its softmax probability summed over the query
+ *       heads of the KV head                             [summary, 实验设计]
  *
  * Build: gcc -O2 -std=c11 -ffp-contract=off -fno-fast-math -fPIC -shared
  * (no FMA contraction, SSE2 float arithmetic, IEEE round-to-nearest-even).
@@ -353,12 +356,15 @@ int oracle_select(const double *s, int T, int W, int keep, int32_t *idx)
  * residual.  q: [g, D] fp16.  The cache holds n_q packed tokens (layout of
  * O5-O7) followed by the residual res_k/res_v [r, D] fp16, oldest first.
  * out[h] = sum_t softmax_t(tau * q_h . kappa_t) nu_t over all n_q + r tokens,
- * kappa/nu the dequantized (O8) packed rows and the raw residual rows; fp64. */
-void oracle_decode_attention(const uint16_t *q, int g,
-                             const uint32_t *k_codes, const uint16_t *k_scale, const uint16_t *k_zero,
-                             const uint32_t *v_codes, const uint16_t *v_scale, const uint16_t *v_zero,
-                             int n_q, const uint16_t *res_k, const uint16_t *res_v, int r,
-                             int D, int G, int Gv, double tau, double *out)
+ * kappa/nu the dequantized (O8) packed rows and the raw residual rows; fp64.
+ * If mass is not NULL, O10 as well: mass[t] = sum_h softmax_t(tau * q_h .
+ * kappa_t) for t in [0, n_q + r), packed tokens first, then the residual
+ * oldest first (the order in which the tokens entered the cache). */
+static void decode_attention_impl(const uint16_t *q, int g,
+                                  const uint32_t *k_codes, const uint16_t *k_scale, const uint16_t *k_zero,
+                                  const uint32_t *v_codes, const uint16_t *v_scale, const uint16_t *v_zero,
+                                  int n_q, const uint16_t *res_k, const uint16_t *res_v, int r,
+                                  int D, int G, int Gv, double tau, double *out, double *mass)
 {
     int n = n_q + r;
     double *kh = (double *)malloc(sizeof(double) * ((size_t)n * D + 1));
@@ -369,6 +375,8 @@ void oracle_decode_attention(const uint16_t *q, int g,
         kh[(long)n_q * D + e] = oracle_half_to_double(res_k[e]);
         vh[(long)n_q * D + e] = oracle_half_to_double(res_v[e]);
     }
+    if (mass)
+        for (int t = 0; t < n; ++t) mass[t] = 0.0;
     for (int h = 0; h < g; ++h) {
         double m = -INFINITY;
         for (int t = 0; t < n; ++t) {
@@ -384,6 +392,34 @@ void oracle_decode_attention(const uint16_t *q, int g,
             for (int t = 0; t < n; ++t) acc += p[t] * vh[(long)t * D + c];
             out[(long)h * D + c] = acc / l;
         }
+        if (mass)
+            for (int t = 0; t < n; ++t) mass[t] += p[t] / l;
     }
     free(kh); free(vh); free(p);
+}
+
+void oracle_decode_attention(const uint16_t *q, int g,
+                             const uint32_t *k_codes, const uint16_t *k_scale, const uint16_t *k_zero,
+                             const uint32_t *v_codes, const uint16_t *v_scale, const uint16_t *v_zero,
+                             int n_q, const uint16_t *res_k, const uint16_t *res_v, int r,
+                             int D, int G, int Gv, double tau, double *out)
+{
+    decode_attention_impl(q, g, k_codes, k_scale, k_zero, v_codes, v_scale, v_zero, n_q, res_k, res_v, r,
+                          D, G, Gv, tau, out, NULL);
+}
+
+/* ------------------------------------------- O10: decode attention mass */
+
+/* O9 plus this step's attention mass of every cached token (see
+ * decode_attention_impl): mass [n_q + r] fp64, overwritten.  H2O, the
+ * accumulated-attention eviction the summary's experiments compare against,
+ * ranks tokens by the sum of these per-step masses; the caller accumulates. */
+void oracle_decode_attention_mass(const uint16_t *q, int g,
+                                  const uint32_t *k_codes, const uint16_t *k_scale, const uint16_t *k_zero,
+                                  const uint32_t *v_codes, const uint16_t *v_scale, const uint16_t *v_zero,
+                                  int n_q, const uint16_t *res_k, const uint16_t *res_v, int r,
+                                  int D, int G, int Gv, double tau, double *out, double *mass)
+{
+    decode_attention_impl(q, g, k_codes, k_scale, k_zero, v_codes, v_scale, v_zero, n_q, res_k, res_v, r,
+                          D, G, Gv, tau, out, mass);
 }

@@ -11,11 +11,13 @@ Step names O1..O9 follow the restatement in ``minikv_oracle.c``:
   O1 prefill attention        O2 observation-window scores   O3 select
   O4 gather                   O5 split                       O6 quantize
   O7 bit packing              O8 dequant                     O9 decode step
+  O10 decode-time attention mass (H2O-style accumulated score)
 Sources: the MiniKV abstract (2-bit layer-discriminative KV cache, kernels
 compatible with FlashAttention) and the gptget.net summary of arXiv 2411.18077,
 sections 方法论 / 方法详解 (sub-channel key quantization, per-token value
 quantization, selective flash attention by a second kernel, importance-based
-adaptive KV).
+adaptive KV) and 实验设计 (H2O, the accumulated-attention eviction MiniKV is
+compared with).
 
 Parity pins: every function here is pinned by ``tests/test_oracle_pins.py``
 against fp16 library rounding (numpy), torch fp64 attention, closed forms,
@@ -65,6 +67,8 @@ _SIGS = {
     "oracle_window_scores": (None, [_P, _P, _I, _I, _I, _I, _D, _P]),
     "oracle_select": (_I, [_P, _I, _I, _I, _P]),
     "oracle_decode_attention": (None, [_P, _I, _P, _P, _P, _P, _P, _P, _I, _P, _P, _I, _I, _I, _I, _D, _P]),
+    "oracle_decode_attention_mass": (None, [_P, _I, _P, _P, _P, _P, _P, _P, _I, _P, _P, _I, _I, _I, _I, _D, _P,
+                                            _P]),
 }
 
 
@@ -258,6 +262,36 @@ class SliceCache:
         lib().oracle_decode_attention(_ptr(qb), g, *(_ptr(x) for x in a), self.n_q,
                                       _ptr(rk), _ptr(rv), self.r, self.D, self.G, self.Gv,
                                       tau, _ptr(out))
+        return out
+
+    def attend_mass(self, q, tau: float) -> tuple[np.ndarray, np.ndarray]:
+        """O9 + O10 step 2: q [g, D] fp16 -> (out [g, D], mass [n_q + r]) fp64.
+        mass[t] = sum over the g heads of token t's softmax probability; t runs
+        over the packed tokens, then the residual oldest first, i.e. the order in
+        which the tokens entered this slice."""
+        qb = _h(q)
+        g = qb.shape[0]
+        rk = np.ascontiguousarray(np.array(self.res_k, np.uint16).reshape(self.r, self.D))
+        rv = np.ascontiguousarray(np.array(self.res_v, np.uint16).reshape(self.r, self.D))
+        out = np.zeros((g, self.D))
+        mass = np.zeros(self.n_q + self.r)
+        a = [np.ascontiguousarray(x) for x in (self.k_codes, self.k_scale, self.k_zero,
+                                               self.v_codes, self.v_scale, self.v_zero)]
+        lib().oracle_decode_attention_mass(_ptr(qb), g, *(_ptr(x) for x in a), self.n_q,
+                                           _ptr(rk), _ptr(rv), self.r, self.D, self.G, self.Gv,
+                                           tau, _ptr(out), _ptr(mass))
+        return out, mass
+
+    def step_mass(self, q, k_new, v_new, tau: float, acc: np.ndarray) -> np.ndarray:
+        """O9 + O10: append the new token, attend, add this step's mass to the
+        running score acc[:n_q + r] (indexed by arrival order, which a flush
+        keeps), then flush if due.  Returns out [g, D]."""
+        self.res_k.append(_h(k_new).ravel().copy())
+        self.res_v.append(_h(v_new).ravel().copy())
+        out, mass = self.attend_mass(q, tau)
+        acc[: mass.size] += mass
+        if self.r == self.R + self.G:
+            self.flush()
         return out
 
     def step(self, q, k_new, v_new, tau: float) -> np.ndarray:

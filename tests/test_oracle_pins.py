@@ -4,7 +4,7 @@ Each test ties one oracle step to something other than the oracle itself:
 numpy's fp16 rounding, torch's fp64 attention, a closed form, an invariant or
 brute force on a tiny input.  The steps are those of the MiniKV method as the
 pages name them (abstract; gptget.net summary, 方法论 / 方法详解), restated in
-oracle/minikv_oracle.c as O1..O9.
+oracle/minikv_oracle.c as O1..O10.
 """
 import math
 
@@ -380,3 +380,90 @@ def test_decode_flush_packs_oldest_group(oracle):
     whole = oracle.pack_tokens(k[: 64 + 2 * G], v[: 64 + 2 * G], G, Gv)
     for key in whole:
         assert np.array_equal(getattr(sc, key), whole[key]), key
+
+
+# ------------------------------------------------------ O10 decode mass
+
+def test_decode_mass_matches_dense_softmax(oracle):
+    """Per-token mass = softmax over the dequantized keys (independent numpy
+    dequant, torch fp64 softmax) summed over the group's heads; it sums to g and
+    the attention output is O9's."""
+    D, N, g, G, Gv, R = 128, 300, 3, 32, 64, 32
+    k = synth.keys_fp16((N, D), 71).numpy()
+    v = synth.normal_fp16((N, D), 72).numpy()
+    q = synth.normal_fp16((g, D), 73).numpy()
+    kn = synth.keys_fp16((D,), 74).numpy()
+    vn = synth.normal_fp16((D,), 75).numpy()
+    sc = oracle.SliceCache.from_kept(k, v, R=R, G=G, Gv=Gv)
+    twin = oracle.SliceCache.from_kept(k, v, R=R, G=G, Gv=Gv)
+    nq = sc.n_q
+    kh, _ = _np_dequant(sc, G, Gv)
+    acc = np.zeros(N + 1)
+    out = sc.step_mass(q, kn, vn, TAU, acc)
+    kk = np.vstack([kh, k[nq:].astype(np.float64), kn[None].astype(np.float64)])
+    logits = torch.from_numpy(q.astype(np.float64)) @ torch.from_numpy(kk).T * TAU
+    ref = torch.softmax(logits, dim=-1).sum(0).numpy()
+    assert np.max(np.abs(acc - ref)) < 1e-13
+    assert abs(acc.sum() - g) < 1e-12
+    assert np.array_equal(out, twin.step(q, kn, vn, TAU))
+
+
+def test_decode_mass_single_head_weights_reproduce_output(oracle):
+    """g = 1: the mass is the softmax weight vector, so sum_t mass_t nu_t is the
+    O9 output (values dequantized independently)."""
+    D, N, G, Gv, R = 128, 200, 32, 32, 32
+    k = synth.keys_fp16((N, D), 81).numpy()
+    v = synth.normal_fp16((N, D), 82).numpy()
+    q = synth.normal_fp16((1, D), 83).numpy()
+    sc = oracle.SliceCache.from_kept(k, v, R=R, G=G, Gv=Gv)
+    nq = sc.n_q
+    _, vh = _np_dequant(sc, G, Gv)
+    out, mass = sc.attend_mass(q, TAU)
+    vv = np.vstack([vh, v[nq:].astype(np.float64)])
+    assert np.max(np.abs(mass @ vv - out[0])) < 1e-12
+
+
+def test_decode_mass_zero_query_is_uniform(oracle):
+    D, N, g = 128, 130, 4
+    k = synth.keys_fp16((N, D), 91).numpy()
+    v = synth.normal_fp16((N, D), 92).numpy()
+    sc = oracle.SliceCache.from_kept(k, v, R=32, G=32, Gv=128)
+    _, mass = sc.attend_mass(np.zeros((g, D), np.float16), TAU)
+    assert mass.shape == (N,)
+    assert np.max(np.abs(mass - g / N)) < 1e-15
+
+
+def test_decode_mass_accumulates_by_arrival_order_across_flush(oracle):
+    """Closed form.  Queries see only channel 0; every key has channel 0 = 0
+    except one 'beacon' token appended at step s0 (channel 0 = 30, exact after
+    2-bit packing: its group's channel-0 range is [0, 30], scale 10).  Before the
+    beacon every step is uniform, g/n per token; from then on the beacon takes
+    all but ~n e^-21 of every head's mass.  The beacon is flushed into the packed
+    part midway and must keep its position."""
+    D, G, Gv, R, g = 128, 32, 128, 32, 2
+    N = 64 + R + G - 6                      # r = R+G-6 after the split
+    steps, s0 = 12, 3                       # beacon at arrival position N+3; flush at step 5
+    rng = np.random.default_rng(5)
+    k = f16(rng.standard_normal((N + steps, D)))
+    k[:, 0] = 0
+    k[N + s0, 0] = 30
+    v = f16(rng.standard_normal((N + steps, D)))
+    q = np.zeros((g, D), np.float16)
+    q[:, 0] = 8
+    sc = oracle.SliceCache.from_kept(k[:N], v[:N], R=R, G=G, Gv=Gv)
+    acc = np.zeros(N + steps)
+    flushed = False
+    for s in range(steps):
+        nq = sc.n_q
+        sc.step_mass(q, k[N + s], v[N + s], TAU, acc)
+        flushed |= sc.n_q > nq
+        if s == s0 + 1:
+            assert not flushed
+    assert flushed and sc.n_q > N + s0 - sc.r   # the beacon now sits in the packed part
+    n_after = steps - s0
+    # tokens that arrived before the beacon: the uniform steps, plus at most e^-21 each after it
+    for t in range(N + s0):
+        exp_t = sum(g / (N + s + 1) for s in range(max(0, t - N), s0))
+        assert abs(acc[t] - exp_t) < g * n_after * math.exp(-21) * 1.01, t
+    assert abs(acc[N + s0] - g * n_after) < g * n_after * (N + steps) * math.exp(-21)
+    assert abs(acc.sum() - g * steps) < 1e-9
