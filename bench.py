@@ -253,8 +253,8 @@ def make_decode_state(torch, mk, synth, device, warmup, steps):
     keeps = decode_keeps()
     total_steps = warmup + 2 * steps + 2
     cap_max = ((max(keeps) + total_steps) // G + 2) * G
-    ws = torch.zeros(mk.workspace_size(mk.OP_DECODE_ATTN, B, Hq, Hkv, cap_max + R + G), dtype=torch.uint8,
-                     device=device)
+    op = mk.OP_DECODE_ATTN_MASS if DECODE.get("mass") else mk.OP_DECODE_ATTN
+    ws = torch.zeros(mk.workspace_size(op, B, Hq, Hkv, cap_max + R + G), dtype=torch.uint8, device=device)
     wid = 4 if DECODE["workload"] == "mistral7b_gqa_decode" else 40 + list(DECODE_PRESETS).index(DECODE["workload"])
     caches = []
     for l in range(L):
@@ -267,6 +267,8 @@ def make_decode_state(torch, mk, synth, device, warmup, steps):
             v[b] = synth.normal_fp16((Hkv, N, 128), synth.seed_of(wid, l, synth.T_V, 0, b), device)
         c = mk.MiniKVCache(B, Hkv, cap, G=G, Gv=Gv, R=R, Hq=Hq, device=device, ws=ws)
         mk.quant_pack(c, k, v)
+        # H2O-style running attention mass per token (--mass)
+        c.mass = torch.zeros((B, Hkv, cap + R + G), dtype=torch.float32, device=device) if DECODE.get("mass") else None
         caches.append(c)
         del k, v
     torch.cuda.synchronize()
@@ -285,7 +287,17 @@ def make_decode_state(torch, mk, synth, device, warmup, steps):
 
 
 def unit_bytes(c):
-    return BYTES_PER_PACKED * c.n_packed + BYTES_PER_RESIDUAL * (c.n_res + 1)
+    n = BYTES_PER_PACKED * c.n_packed + BYTES_PER_RESIDUAL * (c.n_res + 1)
+    if c.mass is not None:   # read and write of one fp32 running score per token
+        n += 8 * (c.n_packed + c.n_res + 1)
+    return n
+
+
+def decode_call(mk, c, q, kn, vn, out, ws):
+    if c.mass is not None:
+        mk.decode_attn_mass(c, q, kn, vn, c.mass, out=out, ws=ws)
+    else:
+        mk.decode_attn(c, q, kn, vn, out=out, ws=ws)
 
 
 def run_prefill(torch, mk, synth, device):
@@ -387,7 +399,7 @@ def run_gpu(args):
                 nbytes.append(unit_bytes(caches[l]) * B * DECODE["kv_heads"])
             if ev is not None:
                 ev[l][0].record(stream)
-            mk.decode_attn(caches[l], q_src[p, l], kn_src[p, l], vn_src[p, l], out=out[l], ws=ws)
+            decode_call(mk, caches[l], q_src[p, l], kn_src[p, l], vn_src[p, l], out[l], ws)
             if ev is not None:
                 ev[l][1].record(stream)
 
@@ -439,7 +451,7 @@ def run_gpu(args):
         dk.copy_(hk[p:p + 1], non_blocking=True)
         dv.copy_(hv[p:p + 1], non_blocking=True)
         for l in range(L):
-            mk.decode_attn(caches[l], dq[0, l], dk[0, l], dv[0, l], out=out[l], ws=ws)
+            decode_call(mk, caches[l], dq[0, l], dk[0, l], dv[0, l], out[l], ws)
         hout.copy_(out, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
@@ -456,7 +468,8 @@ def run_gpu(args):
         prefill["tensor_frac_of_bf16_peak"] = prefill["select_prefill_tflops"] / pk["bf16"]
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and DECODE["workload"] == "mistral7b_gqa_decode":
+    if (rank == 0 and world == 1 and not args.no_cpu_baseline and DECODE["workload"] == "mistral7b_gqa_decode"
+            and not DECODE.get("mass")):
         threads = os.cpu_count() or 1
         rate, n, dt = oracle_decode_rate(args.cpu_seconds, threads)
         cpu = {"value": cpu_tokens_per_s(rate), "unit": "tokens/s", "cores": threads, "kind": "oracle",
@@ -466,6 +479,8 @@ def run_gpu(args):
 
     traffic, traffic_note = recorded_traffic(
         "decode_kernel", os.path.join(ROOT, "bit_quantized_evicted_b200", "csrc", "decode.cu"))
+    if DECODE.get("mass"):
+        traffic, traffic_note = None, "no capture of the attention-mass variant (decode_kernel<true> + mass_kernel)"
     if rank == 0:
         line = {
             "metric": METRIC, "value": tok_s, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
@@ -481,7 +496,7 @@ def run_gpu(args):
                          "traffic_source": traffic_note},
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_tok_s, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-            "gpu_launches": L * args.steps,
+            "gpu_launches": L * args.steps * (2 if DECODE.get("mass") else 1),
             "clocks": clk.summary(),
             "prefill": prefill,
         }
@@ -501,6 +516,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--workload", default="mistral7b_gqa_decode", choices=list(DECODE_PRESETS),
                     help="decode workload (the default one carries the bench line's target)")
+    ap.add_argument("--mass", action="store_true",
+                    help="decode with minikv_decode_attn_mass (H2O-style running attention mass per token)")
     ap.add_argument("--prefill-workload", default="llama2_7b_prefill_select", choices=list(PREFILL_PRESETS))
     ap.add_argument("--layers", type=int, default=None,
                     help="decode layers (fewer only for small profiling runs; default: the workload's)")
@@ -513,6 +530,8 @@ def main():
     PREFILL.update(PREFILL_PRESETS[args.prefill_workload])
     if args.layers is not None:
         DECODE["layers"] = args.layers
+    if args.mass:
+        DECODE["mass"] = True
     if args.prefill_layers is not None:
         PREFILL["layers"] = args.prefill_layers
     if args.warmup < 3:

@@ -32,6 +32,13 @@
 //     movmatrix; out_ch = (O^T[ch,h] + O^T[ch,h+4]) 2^(24-p) + sum_t p_t v_zero_t.
 // A 16-token m-tile takes its tokens in the order perm8 so that both the
 // key-word and the value-word shared loads of a warp hit 32 distinct banks.
+//
+// Attention-mass variant (decode_kernel<true>, minikv_decode_attn_mass): every
+// CTA also stores the absolute log2 score of each token it scores, per query
+// head, into a workspace array; the merging CTA of a unit stores the unit's
+// final (max, sum) per head; mass_kernel then adds
+// sum_h 2^(x_h,t - M_h) / L_h to the caller's running score of token t, the
+// H2O-style accumulated attention the MiniKV summary's experiments compare with.
 #include <math.h>
 
 #include "common.cuh"
@@ -84,6 +91,9 @@ struct Args {
     float *part;
     unsigned *counters;
     int *err;
+    float *xs;          // mass variant: absolute log2 scores [unit][g][xs_stride]
+    float *stats;       // mass variant: merged (max, sum) per unit and head [unit][4][2]
+    int xs_stride;
     int Hkv, g, G, cap, ring;
     int n_q, r, res_start, flush;
     int units, n_rc, spu, P, S_max;   // schedule: slices per unit, packed CTAs, partial slots per unit
@@ -172,6 +182,7 @@ __host__ __device__ constexpr float pair_wo(int i) { return pair_wq(i) * 65536.f
 
 // Write this CTA's partial state for `unit` into slot `slot`, then let the
 // last arriving CTA of the unit (S_u arrivals) merge all slots into `out`.
+template <bool kMass>
 __device__ void finish_unit(const Args &a, Smem &sm, int unit, int slot, int S_u, const float *m_h,
                             const float *l_h, const float (*y_h)[kD]) {
     const int tid = threadIdx.x;
@@ -204,10 +215,15 @@ __device__ void finish_unit(const Args &a, Smem &sm, int unit, int slot, int S_u
             Y += f * __ldcg(p + tid);
         }
         a.out[((size_t)b * Hq + kvh * a.g + h) * kD + tid] = f2h(__fdividef(Y, L));
+        if (kMass && tid == 0) {
+            a.stats[(unit * 4 + h) * 2] = M;
+            a.stats[(unit * 4 + h) * 2 + 1] = L;
+        }
     }
 }
 
 // Merge the four warps' states (sm.wm / wl / wy) and hand the CTA partial on.
+template <bool kMass>
 __device__ void merge_warps_and_finish(const Args &a, Smem &sm, int unit, int slot, int S_u) {
     const int tid = threadIdx.x;
     __syncthreads();
@@ -229,7 +245,7 @@ __device__ void merge_warps_and_finish(const Args &a, Smem &sm, int unit, int sl
     __syncthreads();
 #pragma unroll
     for (int h = 0; h < 4; ++h) sm.wy[0][h][tid] = yh[h];
-    finish_unit(a, sm, unit, slot, S_u, mh, lh, sm.wy[0]);
+    finish_unit<kMass>(a, sm, unit, slot, S_u, mh, lh, sm.wy[0]);
 }
 
 // packed CTA c covers slices [c*Ns/P, (c+1)*Ns/P); the CTA holding slice x
@@ -252,6 +268,7 @@ __device__ __forceinline__ void unit_slots(const Args &a, int unit, int &first, 
 // Residual chunk rc of a unit: logical residual tokens [64 rc, 64 rc + 64) in
 // fp16; warp w takes 16 of them as one m-tile.  Scores use q (exact in fp16)
 // as the B operand; outputs the same hi/lo P as the packed path.
+template <bool kMass>
 __device__ void residual_chunk_cta(const Args &a, Smem &sm, int unit, int rc) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g_ = lane >> 2, t_ = lane & 3;
@@ -329,6 +346,11 @@ __device__ void residual_chunk_cta(const Args &a, Smem &sm, int unit, int rc) {
             const float v = s[i] + __shfl_xor_sync(0xffffffffu, s[i], 2);
             const int row = 16 * warp + g_ + 8 * (i >> 1);
             x[i] = row < n ? v * a.scale_log2 : -INFINITY;
+            if (kMass) {   // lanes t_ < 2 hold head hA + (i & 1) of token `row`
+                const int h = hA + (i & 1);
+                if (t_ < 2 && h < a.g && row < n)
+                    a.xs[((size_t)unit * a.g + h) * a.xs_stride + a.n_q + i0 + row] = x[i];
+            }
         }
 #pragma unroll
         for (int e = 0; e < 2; ++e) m_w[e] = warp_max_g(fmaxf(x[e], x[e + 2]));
@@ -383,7 +405,7 @@ __device__ void residual_chunk_cta(const Args &a, Smem &sm, int unit, int rc) {
     }
     int first, S_u;
     unit_slots(a, unit, first, S_u);
-    merge_warps_and_finish(a, sm, unit, rc, S_u);
+    merge_warps_and_finish<kMass>(a, sm, unit, rc, S_u);
 }
 
 // ------------------------------------------------------------------ packed CTA
@@ -429,6 +451,7 @@ __device__ __forceinline__ uint32_t qw_pair(const uint16_t *qh, int t_) {
 }
 
 // packed fp32 pairs (two lanes of work per instruction)
+template <bool kMass>
 __device__ void packed_cta(const Args &a, Smem &sm, int c) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g_ = lane >> 2, t_ = lane & 3;
@@ -556,6 +579,19 @@ __device__ void packed_cta(const Args &a, Smem &sm, int c) {
                 x_[0][i] = fmaf(w0, a.scale_log2 * 65536.f, (i & 1) ? -mr1 : -mr0);
                 x_[1][i] = fmaf(w1, a.scale_log2 * 65536.f, (i & 1) ? -mr1 : -mr0);
             }
+            if (kMass) {   // lanes t_ < 2: head hA + (i & 1), token 16 mt + 8 (i >> 1) + perm8(g_)
+                const int h = hA;
+                if (t_ < 2) {
+                    float *xrow = a.xs + ((size_t)unit * a.g + h) * a.xs_stride + (size_t)(x - unit * a.spu) * kSlice + pg;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        if (h + (i & 1) < a.g) {
+                            const float ref = (i & 1) ? mr1 : mr0;
+                            xrow[(i & 1) * a.xs_stride + 8 * (i >> 1)] = x_[0][i] + ref;
+                            xrow[(i & 1) * a.xs_stride + 16 + 8 * (i >> 1)] = x_[1][i] + ref;
+                        }
+                }
+            }
             // ---- online softmax: rescale only when a head's running max grows
             float mx0 = fmaxf(fmaxf(x_[0][0], x_[0][2]), fmaxf(x_[1][0], x_[1][2]));
             float mx1 = fmaxf(fmaxf(x_[0][1], x_[0][3]), fmaxf(x_[1][1], x_[1][3]));
@@ -663,30 +699,76 @@ __device__ void packed_cta(const Args &a, Smem &sm, int c) {
         }
         int first, S_u;
         unit_slots(a, unit, first, S_u);
-        merge_warps_and_finish(a, sm, unit, a.n_rc + (c - first), S_u);
+        merge_warps_and_finish<kMass>(a, sm, unit, a.n_rc + (c - first), S_u);
         seg = seg_end;
     }
 }
 
+template <bool kMass>
 __global__ void __launch_bounds__(kThreads, 4) decode_kernel(const Args a) {
     extern __shared__ __align__(128) unsigned char smem_raw[];
     Smem &sm = *reinterpret_cast<Smem *>(smem_raw);
     // packed CTAs first: they carry most of the work; the short residual CTAs fill in behind them
-    if ((int)blockIdx.x < a.P) packed_cta(a, sm, blockIdx.x);
+    if ((int)blockIdx.x < a.P) packed_cta<kMass>(a, sm, blockIdx.x);
     else {
         const int i = blockIdx.x - a.P;
-        residual_chunk_cta(a, sm, i / a.n_rc, i % a.n_rc);
+        residual_chunk_cta<kMass>(a, sm, i / a.n_rc, i % a.n_rc);
+    }
+}
+
+// mass[unit][t] += sum_h 2^(xs[unit][h][t] - M_h) / L_h for the n tokens of
+// this step; grid (ceil(n / 1024), units), four consecutive tokens per thread,
+// all G_ score loads issued before any use.  Launched as a programmatic
+// dependent of decode_kernel<true>: its launch overlaps the decode kernel's
+// tail and griddepcontrol.wait holds it until that grid has finished and its
+// writes are visible.  xs rows are 16-byte aligned (xs_stride4 float4s each);
+// entries from n up to the row end hold no score and are never used.
+template <int G_>
+__global__ void __launch_bounds__(256) mass_kernel(const float4 *__restrict__ xs, const float *__restrict__ stats,
+                                                   float *__restrict__ mass, int n, int xs_stride4,
+                                                   long long mass_stride, bool vec) {
+    asm volatile("griddepcontrol.wait;\n" ::: "memory");
+    const int unit = blockIdx.y;
+    const int t4 = blockIdx.x * 256 + threadIdx.x;
+    if (4 * t4 >= n) return;
+    float4 x[G_];
+#pragma unroll
+    for (int h = 0; h < G_; ++h) x[h] = __ldcs(xs + (size_t)(unit * G_ + h) * xs_stride4 + t4);
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll
+    for (int h = 0; h < G_; ++h) {
+        const float M = __ldg(stats + (unit * 4 + h) * 2), iL = 1.f / __ldg(stats + (unit * 4 + h) * 2 + 1);
+        a0 += ex2(x[h].x - M) * iL;
+        a1 += ex2(x[h].y - M) * iL;
+        a2 += ex2(x[h].z - M) * iL;
+        a3 += ex2(x[h].w - M) * iL;
+    }
+    float *m = mass + (size_t)unit * mass_stride + 4 * t4;
+    if (vec && 4 * t4 + 3 < n) {
+        float4 v = *reinterpret_cast<float4 *>(m);
+        v.x += a0;
+        v.y += a1;
+        v.z += a2;
+        v.w += a3;
+        *reinterpret_cast<float4 *>(m) = v;
+    } else {
+        const float a[4] = {a0, a1, a2, a3};
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+            if (4 * t4 + e < n) m[e] += a[e];
     }
 }
 
 int g_slots = 0;   // resident decode CTAs on the device (SMs x CTAs per SM)
 bool g_attr_done = false;
 
-// the kernel's shared memory is above the 48 KB default: opt in once
+// the kernels' shared memory is above the 48 KB default: opt in once
 int ensure_attr() {
     if (!g_attr_done) {
-        if (cudaFuncSetAttribute(decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(Smem)) !=
-            cudaSuccess)
+        if (cudaFuncSetAttribute(decode_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)sizeof(Smem)) != cudaSuccess ||
+            cudaFuncSetAttribute(decode_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)sizeof(Smem)) != cudaSuccess)
             return check_launch("decode_attn: cudaFuncSetAttribute");
         g_attr_done = true;
     }
@@ -698,7 +780,7 @@ int resident_slots() {
         int dev = 0, sms = 148, per = 4;
         if (ensure_attr() == MINIKV_OK && cudaGetDevice(&dev) == cudaSuccess) {
             cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, decode_kernel, kThreads, sizeof(Smem)) !=
+            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, decode_kernel<false>, kThreads, sizeof(Smem)) !=
                     cudaSuccess || per < 1)
                 per = 4;
         }
@@ -760,6 +842,17 @@ size_t decode_workspace_bytes(int B, int Hkv, int max_tokens) {
     return decode_counter_bytes(B, Hkv) + units * (n_rc + per_unit) * 4 * kPartStride * 4;
 }
 
+// Extra workspace of the attention-mass variant: (max, sum) per unit and head,
+// then the log2 scores of up to max_tokens tokens per unit and query head.
+static size_t mass_stats_bytes(int B, int Hkv) { return (((size_t)B * Hkv * 8 * 4 + 255) / 256) * 256; }
+static size_t mass_scores_bytes(int B, int Hkv, int g, int n_tokens) {
+    return (size_t)B * Hkv * g * (size_t)((n_tokens + 3) & ~3) * 4;
+}
+size_t decode_mass_workspace_bytes(int B, int Hq, int Hkv, int max_tokens) {
+    return decode_workspace_bytes(B, Hkv, max_tokens) + mass_stats_bytes(B, Hkv) +
+           mass_scores_bytes(B, Hkv, Hq / Hkv, max_tokens);
+}
+
 // Workspace bytes the next decode call on this cache state will use.
 size_t decode_call_workspace_bytes(const minikv_cache *c) {
     const Plan p = plan(c);
@@ -767,7 +860,7 @@ size_t decode_call_workspace_bytes(const minikv_cache *c) {
 }
 
 int decode_launch(minikv_cache *c, const uint16_t *q, const uint16_t *k_new, const uint16_t *v_new, int Hq,
-                  float sm_scale, uint16_t *out, void *ws, size_t ws_bytes, cudaStream_t stream) {
+                  float sm_scale, uint16_t *out, void *ws, size_t ws_bytes, cudaStream_t stream, float *mass) {
     const int g = Hq / c->Hkv;
     const int ring = c->R + c->G;
     const int r = c->n_res + 1;
@@ -776,7 +869,10 @@ int decode_launch(minikv_cache *c, const uint16_t *q, const uint16_t *k_new, con
         return fail(MINIKV_ERR_CAPACITY, "decode_attn: flushing a key group would exceed cap=%d", c->cap);
     const Plan p = plan(c);
     const size_t cnt_bytes = decode_counter_bytes(c->B, c->Hkv);
-    const size_t need = cnt_bytes + (size_t)p.units * p.S_max * 4 * kPartStride * 4;
+    const size_t part_bytes = (size_t)p.units * p.S_max * 4 * kPartStride * 4;
+    const int n_tok = c->n_packed + r;   // tokens this step attends to
+    size_t need = cnt_bytes + part_bytes;
+    if (mass) need += mass_stats_bytes(c->B, c->Hkv) + mass_scores_bytes(c->B, c->Hkv, g, n_tok);
     if (ws == nullptr || ws_bytes < need)
         return fail(MINIKV_ERR_INVALID_ARG, "decode_attn: workspace of %zu bytes needed, %zu given", need, ws_bytes);
 
@@ -790,6 +886,11 @@ int decode_launch(minikv_cache *c, const uint16_t *q, const uint16_t *k_new, con
     a.counters = reinterpret_cast<unsigned *>(ws);
     a.part = reinterpret_cast<float *>(static_cast<char *>(ws) + cnt_bytes);
     a.err = nullptr;
+    a.stats = mass ? reinterpret_cast<float *>(static_cast<char *>(ws) + cnt_bytes + part_bytes) : nullptr;
+    a.xs = mass ? reinterpret_cast<float *>(static_cast<char *>(ws) + cnt_bytes + part_bytes +
+                                            mass_stats_bytes(c->B, c->Hkv))
+                : nullptr;
+    a.xs_stride = (n_tok + 3) & ~3;
     a.Hkv = c->Hkv; a.g = g; a.G = c->G; a.cap = c->cap; a.ring = ring;
     a.n_q = c->n_packed; a.r = r; a.res_start = c->res_start; a.flush = flush;
     a.groups_cap = c->cap / c->G;
@@ -801,7 +902,33 @@ int decode_launch(minikv_cache *c, const uint16_t *q, const uint16_t *k_new, con
     const int arc = ensure_attr();
     if (arc) return arc;
     const int grid = p.units * p.n_rc + p.P;
-    decode_kernel<<<grid, kThreads, smem, stream>>>(a);
+    if (mass) {
+        decode_kernel<true><<<grid, kThreads, smem, stream>>>(a);
+        int rc = check_launch("decode_attn_mass");
+        if (rc) return rc;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((n_tok + 1023) / 1024, p.units);
+        cfg.blockDim = dim3(256);
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        const float4 *xs = reinterpret_cast<const float4 *>(a.xs);
+        const float *st = a.stats;
+        const int xs_stride4 = a.xs_stride / 4;
+        const long long mass_stride = (long long)c->cap + ring;
+        const bool vec = (mass_stride % 4 == 0) && ((reinterpret_cast<uintptr_t>(mass) & 15u) == 0);
+        switch (g) {
+            case 1: cudaLaunchKernelEx(&cfg, mass_kernel<1>, xs, st, mass, n_tok, xs_stride4, mass_stride, vec); break;
+            case 2: cudaLaunchKernelEx(&cfg, mass_kernel<2>, xs, st, mass, n_tok, xs_stride4, mass_stride, vec); break;
+            case 3: cudaLaunchKernelEx(&cfg, mass_kernel<3>, xs, st, mass, n_tok, xs_stride4, mass_stride, vec); break;
+            default: cudaLaunchKernelEx(&cfg, mass_kernel<4>, xs, st, mass, n_tok, xs_stride4, mass_stride, vec); break;
+        }
+    } else {
+        decode_kernel<false><<<grid, kThreads, smem, stream>>>(a);
+    }
     int rc = check_launch("decode_attn");
     if (rc) return rc;
     // host-side state

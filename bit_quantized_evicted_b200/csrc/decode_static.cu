@@ -25,7 +25,8 @@
 namespace minikv {
 
 int decode_launch(minikv_cache *c, const uint16_t *q, const uint16_t *k_new, const uint16_t *v_new, int Hq,
-                  float sm_scale, uint16_t *out, void *ws, size_t ws_bytes, cudaStream_t stream);
+                  float sm_scale, uint16_t *out, void *ws, size_t ws_bytes, cudaStream_t stream,
+                  float *mass = nullptr);
 int decode_validate(minikv_cache *c, const uint16_t *q, const uint16_t *k_new, const uint16_t *v_new, int Hq,
                     const uint16_t *out);
 size_t decode_counter_bytes(int B, int Hkv);

@@ -32,8 +32,10 @@ size_t prefill_workspace_bytes(int B, int Hq, int W);
 int topk_launch(const float *scores, const uint16_t *k, const uint16_t *v, int B, int Hkv, int T, int W, int keep,
                 int32_t *idx, uint16_t *k_kept, uint16_t *v_kept, cudaStream_t stream);
 int decode_launch(minikv_cache *c, const uint16_t *q, const uint16_t *k_new, const uint16_t *v_new, int Hq,
-                  float sm_scale, uint16_t *out, void *ws, size_t ws_bytes, cudaStream_t stream);
+                  float sm_scale, uint16_t *out, void *ws, size_t ws_bytes, cudaStream_t stream,
+                  float *mass = nullptr);
 size_t decode_workspace_bytes(int B, int Hkv, int max_tokens);
+size_t decode_mass_workspace_bytes(int B, int Hq, int Hkv, int max_tokens);
 
 static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -212,19 +214,23 @@ int minikv_evict_pack(const float *scores, const uint16_t *k, const uint16_t *v,
 
 int minikv_decode_attn(minikv_cache *c, const uint16_t *q, const uint16_t *k_new, const uint16_t *v_new, int Hq,
                        float sm_scale, uint16_t *out, void *ws, size_t ws_bytes, void *stream) {
-    g_err[0] = 0;
-    int rc = check_cache(c);
+    int rc = decode_validate(c, q, k_new, v_new, Hq, out);
     if (rc) return rc;
-    if (!q || !k_new || !v_new || !out || !ws) return fail(MINIKV_ERR_INVALID_ARG, "decode_attn: null pointer");
-    if (!aligned16(q) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(out) || !aligned16(ws))
-        return fail(MINIKV_ERR_INVALID_ARG, "decode_attn: pointers must be 16-byte aligned");
-    if (Hq < 1 || Hq % c->Hkv) return fail(MINIKV_ERR_INVALID_ARG, "decode_attn: Hq=%d, Hkv=%d", Hq, c->Hkv);
-    if (Hq / c->Hkv > 4) return fail(MINIKV_ERR_UNSUPPORTED, "decode_attn: more than 4 query heads per KV head");
-    if (c->Gv != c->D) return fail(MINIKV_ERR_UNSUPPORTED, "decode_attn: value group Gv=%d (needs Gv = D)", c->Gv);
-    if ((size_t)c->B * c->Hkv > 65535) return fail(MINIKV_ERR_UNSUPPORTED, "decode_attn: B*Hkv above 65535");
-    if ((size_t)c->B * c->Hkv * (c->cap / 32) >= (1u << 31))
-        return fail(MINIKV_ERR_UNSUPPORTED, "decode_attn: B*Hkv*cap/32 must stay below 2^31");
+    if (!ws) return fail(MINIKV_ERR_INVALID_ARG, "decode_attn: null workspace");
+    if (!aligned16(ws)) return fail(MINIKV_ERR_INVALID_ARG, "decode_attn: workspace must be 16-byte aligned");
     return decode_launch(c, q, k_new, v_new, Hq, sm_scale, out, ws, ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+int minikv_decode_attn_mass(minikv_cache *c, const uint16_t *q, const uint16_t *k_new, const uint16_t *v_new, int Hq,
+                            float sm_scale, uint16_t *out, float *mass, void *ws, size_t ws_bytes, void *stream) {
+    int rc = decode_validate(c, q, k_new, v_new, Hq, out);
+    if (rc) return rc;
+    if (!ws || !mass) return fail(MINIKV_ERR_INVALID_ARG, "decode_attn_mass: null workspace or mass");
+    if (!aligned16(ws)) return fail(MINIKV_ERR_INVALID_ARG, "decode_attn_mass: workspace must be 16-byte aligned");
+    if (reinterpret_cast<uintptr_t>(mass) & 3u)
+        return fail(MINIKV_ERR_INVALID_ARG, "decode_attn_mass: mass must be 4-byte aligned");
+    return decode_launch(c, q, k_new, v_new, Hq, sm_scale, out, ws, ws_bytes, static_cast<cudaStream_t>(stream),
+                         mass);
 }
 
 size_t minikv_workspace_size(int op, int B, int Hq, int Hkv, int T, int D, int W) {
@@ -233,6 +239,9 @@ size_t minikv_workspace_size(int op, int B, int Hq, int Hkv, int T, int D, int W
         case MINIKV_OP_SELECT_PREFILL: return prefill_workspace_bytes(B, Hq, W);
         case MINIKV_OP_TOPK_EVICT: return 0;
         case MINIKV_OP_DECODE_ATTN: return decode_workspace_bytes(B, Hkv, T);
+        case MINIKV_OP_DECODE_ATTN_MASS:
+            if (B < 1 || Hkv < 1 || Hq < Hkv || Hq % Hkv || T < 0) return 0;
+            return decode_mass_workspace_bytes(B, Hq, Hkv, T);
         default: return 0;
     }
 }

@@ -20,7 +20,7 @@ LIB_PATH = os.environ.get("MINIKV_LIB", os.path.join(_PKG, "libminikv.so"))
 HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "minikv.h")
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CAPACITY, ERR_CUDA = 0, -1, -2, -3, -4
-OP_SELECT_PREFILL, OP_TOPK_EVICT, OP_DECODE_ATTN = 1, 2, 3
+OP_SELECT_PREFILL, OP_TOPK_EVICT, OP_DECODE_ATTN, OP_DECODE_ATTN_MASS = 1, 2, 3, 4
 
 _P = ctypes.c_void_p
 _I = ctypes.c_int
@@ -44,6 +44,7 @@ _SIGS = {
     "minikv_topk_evict": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _Z, _P]),
     "minikv_evict_pack": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, ctypes.POINTER(CacheStruct), _P]),
     "minikv_decode_attn": (_I, [ctypes.POINTER(CacheStruct), _P, _P, _P, _I, _F, _P, _P, _Z, _P]),
+    "minikv_decode_attn_mass": (_I, [ctypes.POINTER(CacheStruct), _P, _P, _P, _I, _F, _P, _P, _P, _Z, _P]),
     "minikv_decode_attn_static": (_I, [ctypes.POINTER(CacheStruct), _P, _P, _P, _I, _F, _P, _P]),
     "minikv_workspace_size": (_Z, [_I, _I, _I, _I, _I, _I, _I]),
     "minikv_last_error_string": (ctypes.c_char_p, []),
@@ -245,6 +246,31 @@ def decode_attn(cache: MiniKVCache, q: torch.Tensor, k_new: torch.Tensor, v_new:
         ctypes.byref(cache.c), _dev(q, torch.float16, "q"), _dev(k_new, torch.float16, "k_new"),
         _dev(v_new, torch.float16, "v_new"), Hq, float(sm_scale), _dev(out, torch.float16, "out"),
         _dev(ws, torch.uint8, "ws"), ws.numel(), _stream(stream, q.device)))
+    return out
+
+
+def decode_attn_mass(cache: MiniKVCache, q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor,
+                     mass: torch.Tensor, sm_scale: float | None = None, out: torch.Tensor | None = None,
+                     ws: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """decode_attn that also adds this step's attention mass of every cached
+    token into mass [B, Hkv, cap + R + G] fp32 (tokens in arrival order).  The
+    default workspace is made once per cache, zero-filled, and kept on it."""
+    B, Hq, D = q.shape
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty_like(q)
+    if tuple(mass.shape) != (cache.B, cache.Hkv, cache.cap + cache.R + cache.G):
+        raise ValueError(f"mass shape {tuple(mass.shape)}: expected {(cache.B, cache.Hkv, cache.cap + cache.R + cache.G)}")
+    if ws is None:
+        need = workspace_size(OP_DECODE_ATTN_MASS, B, Hq, cache.Hkv, cache.cap + cache.R + cache.G, D)
+        if getattr(cache, "ws_mass", None) is None or cache.ws_mass.numel() < need:
+            cache.ws_mass = torch.zeros(need, dtype=torch.uint8, device=cache.device)
+        ws = cache.ws_mass
+    _check(lib().minikv_decode_attn_mass(
+        ctypes.byref(cache.c), _dev(q, torch.float16, "q"), _dev(k_new, torch.float16, "k_new"),
+        _dev(v_new, torch.float16, "v_new"), Hq, float(sm_scale), _dev(out, torch.float16, "out"),
+        _dev(mass, torch.float32, "mass"), _dev(ws, torch.uint8, "ws"), ws.numel(), _stream(stream, q.device)))
     return out
 
 

@@ -15,7 +15,7 @@
  *   - same page, glossary 术语表 "adaptive KV": keep the KV states that matter;
  *   - pre.notesum.ai LongBench table, "MiniKV Pyramid" rows: a keep budget that
  *     differs by layer.
- * The four calls below are this library's reading of those steps.
+ * The calls below are this library's reading of those steps.
  *
  * Conventions for every call
  *   - All tensor pointers are DEVICE pointers, owned by the caller.  The library
@@ -200,6 +200,38 @@ MINIKV_API int minikv_decode_attn(minikv_cache *c, const uint16_t *q, const uint
                        void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * minikv_decode_attn_mass -- minikv_decode_attn that also accumulates, per
+ * cached token, the attention mass the step gave it (H2O-style scores).
+ * Source: summary page, 实验设计 (experiments), which names H2O -- eviction by
+ * accumulated attention -- among the methods MiniKV is compared with; the
+ * per-KV-head sum over the query heads of the group follows the window score
+ * of minikv_select_prefill.
+ *   Arguments, output `out`, cache update and errors as minikv_decode_attn, plus:
+ *   mass [B, Hkv, cap + R + G] fp32, caller-owned, 4-byte aligned, updated in
+ *       place: for every token t the step attends to,
+ *         mass[b, kvh, t] += sum over the Hq/Hkv query heads h of KV head kvh
+ *                            of softmax_t(sm_scale * q_h . kappa_t),
+ *       where t numbers the tokens in the order they entered the cache: the
+ *       n_packed packed tokens first (t = 0 .. n_packed-1), then the residual,
+ *       oldest first, the new token last (t = n_packed + n_res, counted before
+ *       this step's flush).  A flush keeps every token's t.  Entries from
+ *       n_packed + n_res + 1 on are not touched.  Each step adds exactly Hq/Hkv
+ *       to the sum over t (up to fp32 rounding).
+ *   ws: minikv_workspace_size(MINIKV_OP_DECODE_ATTN_MASS, B, Hq, Hkv,
+ *       cap + R + G, D, 0) bytes, zero-filled before first use, reusable like
+ *       the workspace of minikv_decode_attn.
+ * Two kernels are queued: the decode kernel, which also stores each token's
+ * log2 score per query head in ws, and a pass that turns them into
+ * probabilities with the merged softmax state and adds them to `mass`.
+ * Choosing tokens to drop by `mass` is left to the caller.
+ * Errors: those of minikv_decode_attn; INVALID_ARG also for a null or
+ * misaligned `mass`.
+ */
+MINIKV_API int minikv_decode_attn_mass(minikv_cache *c, const uint16_t *q, const uint16_t *k_new,
+                                       const uint16_t *v_new, int Hq, float sm_scale, uint16_t *out,
+                                       float *mass, void *ws, size_t ws_bytes, void *stream);
+
+/*
  * minikv_decode_attn_static -- minikv_decode_attn without a caller workspace.
  * The paper has no counterpart to this call; it exists for callers that may
  * not allocate device memory: hosts whose device memory is entirely planned by
@@ -224,9 +256,11 @@ MINIKV_API int minikv_decode_attn_static(minikv_cache *c, const uint16_t *q, con
 #define MINIKV_OP_SELECT_PREFILL 1
 #define MINIKV_OP_TOPK_EVICT     2
 #define MINIKV_OP_DECODE_ATTN    3
+#define MINIKV_OP_DECODE_ATTN_MASS 4
 
-/* Scratch bytes an op needs.  For MINIKV_OP_DECODE_ATTN pass the cache
- * capacity plus R+G as T (the most tokens a step can attend to). */
+/* Scratch bytes an op needs.  For MINIKV_OP_DECODE_ATTN and
+ * MINIKV_OP_DECODE_ATTN_MASS pass the cache capacity plus R+G as T (the most
+ * tokens a step can attend to). */
 MINIKV_API size_t minikv_workspace_size(int op, int B, int Hq, int Hkv, int T, int D, int W);
 
 /* Why the last failing call on this host thread failed ("" if none). */

@@ -55,6 +55,22 @@ def decode_reference_step(ref, q: torch.Tensor, k_new: torch.Tensor, v_new: torc
     return out
 
 
+def decode_mass_reference_step(ref, q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor, tau: float,
+                               acc: np.ndarray) -> np.ndarray:
+    """O9 + O10 on every (b, KV head): returns out [B, Hq, D] fp64, adds the
+    step's mass into acc [B, Hkv, >= n] and advances ref."""
+    qn, kn, vn = np16(q), np16(k_new), np16(v_new)
+    B, Hq, D = qn.shape
+    H = kn.shape[1]
+    g = Hq // H
+    out = np.zeros((B, Hq, D))
+    for b in range(B):
+        for h in range(H):
+            out[b, h * g:(h + 1) * g] = ref[b][h].step_mass(qn[b, h * g:(h + 1) * g], kn[b, h], vn[b, h], tau,
+                                                            acc[b, h])
+    return out
+
+
 def prefill_reference(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, W: int, tau: float, heads=None):
     """O1 outputs for the listed (b, h) query heads and O2 scores for every (b, KV head)."""
     qn, kn, vn = np16(q), np16(k), np16(v)

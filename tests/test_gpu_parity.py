@@ -2,8 +2,10 @@
 
 Bars: packed codes, scales, zeros, the fp16 residual and kept indices are
 bit-exact; attention outputs (fp16) are within 2e-3 max-abs of the oracle's
-fp64 result; window scores (fp32) within a relative 1e-3 (+1e-6).
+fp64 result; window scores (fp32) within a relative 1e-3 (+1e-6); running
+attention masses within 2e-5 per accumulated step.
 """
+import ctypes
 import math
 
 import numpy as np
@@ -13,7 +15,8 @@ import torch
 from bit_quantized_evicted_b200 import minikv as mk
 from bit_quantized_evicted_b200 import synth
 from oracle import minikv_oracle as O
-from tests.oracle_runs import compare_cache, decode_reference_step, np16, pack_reference, prefill_reference
+from tests.oracle_runs import (compare_cache, decode_mass_reference_step, decode_reference_step, np16,
+                               pack_reference, prefill_reference)
 
 pytestmark = pytest.mark.gpu
 
@@ -192,6 +195,77 @@ def test_decode_vs_oracle(B, Hq, Hkv, N, G, R, steps):
         assert err <= ATOL_OUT, (s, err)
     compare_cache(cache, ref)       # flushes packed bit-exactly
     print(f"decode max-abs error {worst:.2e}")
+
+
+# Attention mass: each step adds g probabilities per KV head; the kernel's
+# log2 scores carry fp32 accumulation and ex2.approx error (relative ~1e-6 on
+# each probability), so the running sums may drift by a few 1e-6 per step.
+ATOL_MASS_PER_STEP = 2e-5
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,N,G,R,steps", [
+    (1, 4, 4, 256, 32, 32, 36),      # g = 1; crosses a flush
+    (2, 8, 2, 1000, 32, 128, 8),     # GQA g = 4, several packed CTAs per KV head
+    (1, 3, 1, 20, 32, 32, 3),        # nothing packed yet; g = 3
+    (1, 2, 2, 96, 32, 0, 40),        # R = 0: the whole residual is packed every 32 steps
+    (2, 4, 2, 700, 64, 64, 70),      # G = 64, two flushes, g = 2
+])
+def test_decode_mass_vs_oracle(B, Hq, Hkv, N, G, R, steps):
+    Gv = 128
+    g = Hq // Hkv
+    k, v = _kv(B, Hkv, N, 500 + N)
+    cap = ((N + steps) // G + 2) * G
+    cache = mk.MiniKVCache(B, Hkv, cap, G=G, Gv=Gv, R=R, Hq=Hq)
+    mk.quant_pack(cache, k, v)
+    ref = pack_reference(k, v, R, G, Gv)
+    L = cap + R + G
+    # running scores start non-zero: the call adds, it does not overwrite
+    mass0 = torch.rand((B, Hkv, L), generator=torch.Generator().manual_seed(N), dtype=torch.float64)
+    acc = mass0.numpy().copy()
+    mass = mass0.float().to(DEV)
+    for s in range(steps):
+        q = synth.normal_fp16((B, Hq, 128), synth.seed_of(11, N, synth.T_QDEC, s), DEV)
+        kn = synth.keys_fp16((B, Hkv, 128), synth.seed_of(11, N, synth.T_KNEW, s), DEV)
+        vn = synth.normal_fp16((B, Hkv, 128), synth.seed_of(11, N, synth.T_VNEW, s), DEV)
+        out = mk.decode_attn_mass(cache, q, kn, vn, mass)
+        torch.cuda.synchronize()
+        oref = decode_mass_reference_step(ref, q, kn, vn, TAU, acc)
+        assert float(np.max(np.abs(out.float().cpu().numpy() - oref))) <= ATOL_OUT, s
+        got = mass.double().cpu().numpy()
+        err = float(np.max(np.abs(got - acc)))
+        assert err <= ATOL_MASS_PER_STEP * (s + 1) + 1e-6, (s, err)
+    n = N + steps
+    got = mass.double().cpu().numpy()
+    np.testing.assert_array_equal(got[:, :, n:], mass0.float().double().numpy()[:, :, n:])   # untouched
+    np.testing.assert_allclose((got - mass0.float().double().numpy())[:, :, :n].sum(-1), g * steps, rtol=1e-5)
+    compare_cache(cache, ref)
+
+
+def test_decode_mass_argument_errors():
+    """Bad arguments are refused before anything is queued: the cache state and
+    the running scores stay as they were."""
+    B, Hq, Hkv = 1, 4, 2
+    cache = mk.MiniKVCache(B, Hkv, 128, R=32, Hq=Hq)
+    k, v = _kv(B, Hkv, 100, 7)
+    mk.quant_pack(cache, k, v)
+    q = torch.zeros((B, Hq, 128), dtype=torch.float16, device=DEV)
+    kn = torch.zeros((B, Hkv, 128), dtype=torch.float16, device=DEV)
+    out = torch.empty_like(q)
+    mass = torch.zeros((B, Hkv, 128 + 32 + 32), dtype=torch.float32, device=DEV)
+    small = torch.zeros(64, dtype=torch.uint8, device=DEV)
+    with pytest.raises(mk.MiniKVError) as e:
+        mk.decode_attn_mass(cache, q, kn, kn, mass, ws=small)
+    assert e.value.code == mk.ERR_INVALID_ARG
+    ws = torch.zeros(mk.workspace_size(mk.OP_DECODE_ATTN_MASS, B, Hq, Hkv, 192), dtype=torch.uint8, device=DEV)
+    L = mk.lib()
+    s = torch.cuda.current_stream().cuda_stream
+    for bad_mass in (None, mass.data_ptr() + 2):
+        rc = L.minikv_decode_attn_mass(ctypes.byref(cache.c), q.data_ptr(), kn.data_ptr(), kn.data_ptr(), Hq,
+                                       TAU, out.data_ptr(), bad_mass, ws.data_ptr(), ws.numel(), s)
+        assert rc == mk.ERR_INVALID_ARG
+    assert (cache.n_packed, cache.n_res) == (64, 36)
+    torch.cuda.synchronize()
+    assert float(mass.abs().sum()) == 0.0
 
 
 def test_decode_workspace_reuse_across_layers():
