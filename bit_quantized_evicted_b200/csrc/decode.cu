@@ -92,7 +92,7 @@ struct Args {
     unsigned *counters;
     int *err;
     float *xs;          // mass variant: absolute log2 scores [unit][g][xs_stride]
-    float *stats;       // mass variant: merged (max, sum) per unit and head [unit][4][2]
+    float *stats;       // mass variant: per unit max[4], sum[4], token count (int bits), pad
     int xs_stride;
     int Hkv, g, G, cap, ring;
     int n_q, r, res_start, flush;
@@ -101,6 +101,50 @@ struct Args {
     int Ns;                           // total slices (< 2^31)
     float scale_log2;
 };
+
+// Ragged batches: each sequence b has its own packed count, residual count (the
+// new token included) and ring origin.  The table travels as a kernel parameter
+// (__grid_constant__, read through the constant cache), so a step needs no
+// host-to-device copy.  sbeg[b] = first flat slice of sequence b's units.
+constexpr int kMaxRaggedSeqs = MINIKV_MAX_RAGGED_SEQS;
+struct SeqTab {
+    int n_q[kMaxRaggedSeqs];
+    int r[kMaxRaggedSeqs];
+    int res_start[kMaxRaggedSeqs];
+    int sbeg[kMaxRaggedSeqs + 1];
+};
+struct ArgsVar : Args {
+    SeqTab tab;
+};
+
+// Per-unit lengths.  Uniform batches read the shared scalars; ragged ones the
+// table.  slice0 = the unit's first slice in the flat list of all units'
+// packed slices; unit_of = the unit holding flat slice x (x < Ns).
+__device__ __forceinline__ int len_nq(const Args &a, int) { return a.n_q; }
+__device__ __forceinline__ int len_r(const Args &a, int) { return a.r; }
+__device__ __forceinline__ int len_rs(const Args &a, int) { return a.res_start; }
+__device__ __forceinline__ int len_spu(const Args &a, int) { return a.spu; }
+__device__ __forceinline__ int slice0(const Args &a, int unit) { return unit * a.spu; }
+__device__ __forceinline__ int unit_of(const Args &a, int x) { return x / a.spu; }
+
+__device__ __forceinline__ int len_nq(const ArgsVar &a, int unit) { return a.tab.n_q[unit / a.Hkv]; }
+__device__ __forceinline__ int len_r(const ArgsVar &a, int unit) { return a.tab.r[unit / a.Hkv]; }
+__device__ __forceinline__ int len_rs(const ArgsVar &a, int unit) { return a.tab.res_start[unit / a.Hkv]; }
+__device__ __forceinline__ int len_spu(const ArgsVar &a, int unit) { return a.tab.n_q[unit / a.Hkv] / kSlice; }
+__device__ __forceinline__ int slice0(const ArgsVar &a, int unit) {
+    const int b = unit / a.Hkv;
+    return a.tab.sbeg[b] + (unit - b * a.Hkv) * (a.tab.n_q[b] / kSlice);
+}
+__device__ __forceinline__ int unit_of(const ArgsVar &a, int x) {
+    // largest b with sbeg[b] <= x; since x < sbeg[B], sequence b has slices
+    int lo = 0, hi = a.units / a.Hkv;
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (a.tab.sbeg[mid] <= x) lo = mid;
+        else hi = mid;
+    }
+    return lo * a.Hkv + (x - a.tab.sbeg[lo]) / (a.tab.n_q[lo] / kSlice);
+}
 
 // element offset of (row, col) in a [rows][128] fp16 tile; 16-byte chunks are
 // XOR-swizzled by row so ldmatrix reads of 8 rows hit distinct banks
@@ -182,8 +226,8 @@ __host__ __device__ constexpr float pair_wo(int i) { return pair_wq(i) * 65536.f
 
 // Write this CTA's partial state for `unit` into slot `slot`, then let the
 // last arriving CTA of the unit (S_u arrivals) merge all slots into `out`.
-template <bool kMass>
-__device__ void finish_unit(const Args &a, Smem &sm, int unit, int slot, int S_u, const float *m_h,
+template <bool kMass, class A>
+__device__ void finish_unit(const A &a, Smem &sm, int unit, int slot, int S_u, const float *m_h,
                             const float *l_h, const float (*y_h)[kD]) {
     const int tid = threadIdx.x;
     float *base = a.part + ((size_t)unit * a.S_max + slot) * 4 * kPartStride;
@@ -216,15 +260,16 @@ __device__ void finish_unit(const Args &a, Smem &sm, int unit, int slot, int S_u
         }
         a.out[((size_t)b * Hq + kvh * a.g + h) * kD + tid] = f2h(__fdividef(Y, L));
         if (kMass && tid == 0) {
-            a.stats[(unit * 4 + h) * 2] = M;
-            a.stats[(unit * 4 + h) * 2 + 1] = L;
+            a.stats[unit * 12 + h] = M;
+            a.stats[unit * 12 + 4 + h] = L;
         }
     }
+    if (kMass && tid == 0) a.stats[unit * 12 + 8] = __int_as_float(len_nq(a, unit) + len_r(a, unit));
 }
 
 // Merge the four warps' states (sm.wm / wl / wy) and hand the CTA partial on.
-template <bool kMass>
-__device__ void merge_warps_and_finish(const Args &a, Smem &sm, int unit, int slot, int S_u) {
+template <bool kMass, class A>
+__device__ void merge_warps_and_finish(const A &a, Smem &sm, int unit, int slot, int S_u) {
     const int tid = threadIdx.x;
     __syncthreads();
     float mh[4], lh[4], yh[4];
@@ -252,14 +297,17 @@ __device__ void merge_warps_and_finish(const Args &a, Smem &sm, int unit, int sl
 __device__ __forceinline__ int cta_of_slice(long long x, int P, int Ns) {
     return (int)(((x + 1) * P - 1) / Ns);
 }
-__device__ __forceinline__ void unit_slots(const Args &a, int unit, int &first, int &S_u) {
-    if (a.spu == 0) {
+template <class A>
+__device__ __forceinline__ void unit_slots(const A &a, int unit, int &first, int &S_u) {
+    const int spu = len_spu(a, unit);
+    if (spu == 0) {
         first = 0;
         S_u = a.n_rc;
         return;
     }
-    first = cta_of_slice((long long)unit * a.spu, a.P, a.Ns);
-    const int last = cta_of_slice((long long)(unit + 1) * a.spu - 1, a.P, a.Ns);
+    const int s0 = slice0(a, unit);
+    first = cta_of_slice(s0, a.P, a.Ns);
+    const int last = cta_of_slice((long long)s0 + spu - 1, a.P, a.Ns);
     S_u = a.n_rc + last - first + 1;
 }
 
@@ -268,8 +316,8 @@ __device__ __forceinline__ void unit_slots(const Args &a, int unit, int &first, 
 // Residual chunk rc of a unit: logical residual tokens [64 rc, 64 rc + 64) in
 // fp16; warp w takes 16 of them as one m-tile.  Scores use q (exact in fp16)
 // as the B operand; outputs the same hi/lo P as the packed path.
-template <bool kMass>
-__device__ void residual_chunk_cta(const Args &a, Smem &sm, int unit, int rc) {
+template <bool kMass, class A>
+__device__ void residual_chunk_cta(const A &a, Smem &sm, int unit, int rc) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g_ = lane >> 2, t_ = lane & 3;
     const int b = unit / a.Hkv, kvh = unit % a.Hkv;
@@ -278,16 +326,16 @@ __device__ void residual_chunk_cta(const Args &a, Smem &sm, int unit, int rc) {
     const uint16_t *vnew = a.v_new + (size_t)unit * kD;
     uint16_t *kres = a.k_res + (size_t)unit * a.ring * kD;
     uint16_t *vres = a.v_res + (size_t)unit * a.ring * kD;
-    const int r = a.r;
+    const int r = len_r(a, unit), res_start = len_rs(a, unit), n_q = len_nq(a, unit);
     const int i0 = rc * kResChunk;
     const int n = min(kResChunk, r - i0);
-    auto slot = [&](int i) { int s = a.res_start + i; return s >= a.ring ? s - a.ring : s; };
+    auto slot = [&](int i) { int s = res_start + i; return s >= a.ring ? s - a.ring : s; };
     auto krow = [&](int i) -> const uint16_t * { return i == r - 1 ? knew : kres + (size_t)slot(i) * kD; };
     auto vrow = [&](int i) -> const uint16_t * { return i == r - 1 ? vnew : vres + (size_t)slot(i) * kD; };
 
     {
         const int ch = tid & 15;
-        int s0 = a.res_start + i0 + (tid >> 4);
+        int s0 = res_start + i0 + (tid >> 4);
         if (s0 >= a.ring) s0 -= a.ring;
 #pragma unroll 2
         for (int row = tid >> 4; row < kResChunk; row += 8) {
@@ -349,7 +397,7 @@ __device__ void residual_chunk_cta(const Args &a, Smem &sm, int unit, int rc) {
             if (kMass) {   // lanes t_ < 2 hold head hA + (i & 1) of token `row`
                 const int h = hA + (i & 1);
                 if (t_ < 2 && h < a.g && row < n)
-                    a.xs[((size_t)unit * a.g + h) * a.xs_stride + a.n_q + i0 + row] = x[i];
+                    a.xs[((size_t)unit * a.g + h) * a.xs_stride + n_q + i0 + row] = x[i];
             }
         }
 #pragma unroll
@@ -396,10 +444,10 @@ __device__ void residual_chunk_cta(const Args &a, Smem &sm, int unit, int rc) {
             sm.wl[warp][hA + 1] = l_w[1];
         }
     }
-    if (a.flush && rc == 0) {
+    if (r == a.ring && rc == 0) {
         // the oldest G residual tokens become key group n_q/G and G value tokens
-        const size_t tok0 = (size_t)unit * a.cap + a.n_q;
-        const size_t grow = (size_t)unit * (a.cap / a.G) + a.n_q / a.G;
+        const size_t tok0 = (size_t)unit * a.cap + n_q;
+        const size_t grow = (size_t)unit * (a.cap / a.G) + n_q / a.G;
         pack_key_group(krow, a.G, a.k_codes_w + tok0 * 8, a.k_scale_w + grow * kD, a.k_zero_w + grow * kD);
         pack_value_tokens(vrow, a.G, kD, a.v_codes_w + tok0 * 8, a.v_scale_w + tok0, a.v_zero_w + tok0);
     }
@@ -412,7 +460,8 @@ __device__ void residual_chunk_cta(const Args &a, Smem &sm, int unit, int rc) {
 
 // Queue the bulk copies of the slice at (unit u, slice j) into this warp's
 // stage.  Called by one lane; no division: G is a power of two.
-__device__ __forceinline__ void issue_slice(const Args &a, Smem &sm, int warp, int stage, int u, int j) {
+template <class A>
+__device__ __forceinline__ void issue_slice(const A &a, Smem &sm, int warp, int stage, int u, int j) {
     SliceBuf &S = sm.st[warp][stage];
     uint64_t *bar = &sm.full[warp][stage];
     const int t0 = j * kSlice;
@@ -431,11 +480,13 @@ __device__ __forceinline__ void issue_slice(const Args &a, Smem &sm, int warp, i
 // that stepping needs no division.
 struct Cursor {
     int u, j;
-    __device__ __forceinline__ void step(int n, int spu) {
+    template <class A>
+    __device__ __forceinline__ void step(const A &a, int n) {
         j += n;
-        while (j >= spu) {
+        int spu = len_spu(a, u);
+        while (j >= spu && u < a.units - 1) {
             j -= spu;
-            ++u;
+            spu = len_spu(a, ++u);
         }
     }
 };
@@ -451,8 +502,8 @@ __device__ __forceinline__ uint32_t qw_pair(const uint16_t *qh, int t_) {
 }
 
 // packed fp32 pairs (two lanes of work per instruction)
-template <bool kMass>
-__device__ void packed_cta(const Args &a, Smem &sm, int c) {
+template <bool kMass, class A>
+__device__ void packed_cta(const A &a, Smem &sm, int c) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g_ = lane >> 2, t_ = lane & 3;
     const int Hq = a.Hkv * a.g;
@@ -465,12 +516,16 @@ __device__ void packed_cta(const Args &a, Smem &sm, int c) {
     }
     __syncthreads();
     // this warp's slices: cs + warp + 4k; `nxt` is the next one to queue
-    Cursor nxt{(cs + warp) / a.spu, (cs + warp) % a.spu};
+    Cursor nxt{0, 0};
     int nxt_x = cs + warp;
+    if (nxt_x < ce) {
+        nxt.u = unit_of(a, nxt_x);
+        nxt.j = nxt_x - slice0(a, nxt.u);
+    }
     if (lane == 0)
         for (int k = 0; k < kWarpStages && nxt_x < ce; ++k) {
             issue_slice(a, sm, warp, k, nxt.u, nxt.j);
-            nxt.step(4, a.spu);
+            nxt.step(a, 4);
             nxt_x += 4;
         }
 
@@ -484,8 +539,9 @@ __device__ void packed_cta(const Args &a, Smem &sm, int c) {
 
     int seg = cs;
     while (seg < ce) {
-        const int unit = seg / a.spu;
-        const int seg_end = min(ce, (unit + 1) * a.spu);
+        const int unit = unit_of(a, seg);
+        const int u_s0 = slice0(a, unit);
+        const int seg_end = min(ce, u_s0 + len_spu(a, unit));
         const int b = unit / a.Hkv, kvh = unit % a.Hkv;
         const uint16_t *qbase = a.q + ((size_t)b * Hq + kvh * a.g) * kD;
         // query rows of this unit for the zero-point mma (rows >= g zero), 16-byte
@@ -582,7 +638,7 @@ __device__ void packed_cta(const Args &a, Smem &sm, int c) {
             if (kMass) {   // lanes t_ < 2: head hA + (i & 1), token 16 mt + 8 (i >> 1) + perm8(g_)
                 const int h = hA;
                 if (t_ < 2) {
-                    float *xrow = a.xs + ((size_t)unit * a.g + h) * a.xs_stride + (size_t)(x - unit * a.spu) * kSlice + pg;
+                    float *xrow = a.xs + ((size_t)unit * a.g + h) * a.xs_stride + (size_t)(x - u_s0) * kSlice + pg;
 #pragma unroll
                     for (int i = 0; i < 4; ++i)
                         if (h + (i & 1) < a.g) {
@@ -659,7 +715,7 @@ __device__ void packed_cta(const Args &a, Smem &sm, int c) {
             __syncwarp();
             if (lane == 0 && nxt_x < ce) {
                 issue_slice(a, sm, warp, stage, nxt.u, nxt.j);
-                nxt.step(4, a.spu);
+                nxt.step(a, 4);
                 nxt_x += 4;
             }
         }
@@ -704,8 +760,8 @@ __device__ void packed_cta(const Args &a, Smem &sm, int c) {
     }
 }
 
-template <bool kMass>
-__global__ void __launch_bounds__(kThreads, 4) decode_kernel(const Args a) {
+template <bool kMass, class A>
+__device__ __forceinline__ void decode_body(const A &a) {
     extern __shared__ __align__(128) unsigned char smem_raw[];
     Smem &sm = *reinterpret_cast<Smem *>(smem_raw);
     // packed CTAs first: they carry most of the work; the short residual CTAs fill in behind them
@@ -716,8 +772,20 @@ __global__ void __launch_bounds__(kThreads, 4) decode_kernel(const Args a) {
     }
 }
 
-// mass[unit][t] += sum_h 2^(xs[unit][h][t] - M_h) / L_h for the n tokens of
-// this step; grid (ceil(n / 1024), units), four consecutive tokens per thread,
+template <bool kMass>
+__global__ void __launch_bounds__(kThreads, 4) decode_kernel(const Args a) {
+    decode_body<kMass>(a);
+}
+
+// ragged batch: per-sequence lengths in the parameter table
+template <bool kMass>
+__global__ void __launch_bounds__(kThreads, 4) decode_ragged_kernel(const __grid_constant__ ArgsVar a) {
+    decode_body<kMass>(a);
+}
+
+// mass[unit][t] += sum_h 2^(xs[unit][h][t] - M_h) / L_h for the n_u tokens
+// the unit attended to this step (n_u, M_h, L_h from the merging CTA's stats);
+// grid (ceil(max n_u / 1024), units), four consecutive tokens per thread,
 // all G_ score loads issued before any use.  Launched as a programmatic
 // dependent of decode_kernel<true>: its launch overlaps the decode kernel's
 // tail and griddepcontrol.wait holds it until that grid has finished and its
@@ -725,10 +793,11 @@ __global__ void __launch_bounds__(kThreads, 4) decode_kernel(const Args a) {
 // entries from n up to the row end hold no score and are never used.
 template <int G_>
 __global__ void __launch_bounds__(256) mass_kernel(const float4 *__restrict__ xs, const float *__restrict__ stats,
-                                                   float *__restrict__ mass, int n, int xs_stride4,
-                                                   long long mass_stride, bool vec) {
+                                                   float *__restrict__ mass, int xs_stride4, long long mass_stride,
+                                                   bool vec) {
     asm volatile("griddepcontrol.wait;\n" ::: "memory");
     const int unit = blockIdx.y;
+    const int n = __float_as_int(__ldg(stats + unit * 12 + 8));
     const int t4 = blockIdx.x * 256 + threadIdx.x;
     if (4 * t4 >= n) return;
     float4 x[G_];
@@ -737,7 +806,7 @@ __global__ void __launch_bounds__(256) mass_kernel(const float4 *__restrict__ xs
     float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll
     for (int h = 0; h < G_; ++h) {
-        const float M = __ldg(stats + (unit * 4 + h) * 2), iL = 1.f / __ldg(stats + (unit * 4 + h) * 2 + 1);
+        const float M = __ldg(stats + unit * 12 + h), iL = 1.f / __ldg(stats + unit * 12 + 4 + h);
         a0 += ex2(x[h].x - M) * iL;
         a1 += ex2(x[h].y - M) * iL;
         a2 += ex2(x[h].z - M) * iL;
@@ -762,13 +831,17 @@ __global__ void __launch_bounds__(256) mass_kernel(const float4 *__restrict__ xs
 int g_slots = 0;   // resident decode CTAs on the device (SMs x CTAs per SM)
 bool g_attr_done = false;
 
+template <class K>
+bool set_smem_attr(K kernel) {
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(Smem)) ==
+           cudaSuccess;
+}
+
 // the kernels' shared memory is above the 48 KB default: opt in once
 int ensure_attr() {
     if (!g_attr_done) {
-        if (cudaFuncSetAttribute(decode_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)sizeof(Smem)) != cudaSuccess ||
-            cudaFuncSetAttribute(decode_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)sizeof(Smem)) != cudaSuccess)
+        if (!set_smem_attr(decode_kernel<false>) || !set_smem_attr(decode_kernel<true>) ||
+            !set_smem_attr(decode_ragged_kernel<false>) || !set_smem_attr(decode_ragged_kernel<true>))
             return check_launch("decode_attn: cudaFuncSetAttribute");
         g_attr_done = true;
     }
@@ -790,16 +863,33 @@ int resident_slots() {
     return g_slots;
 }
 
+// Host state of sequence b: the table of a ragged cache, else the shared scalars.
+int seq_nq(const minikv_cache *c, int b) { return c->seq ? c->seq[3 * b] : c->n_packed; }
+int seq_nres(const minikv_cache *c, int b) { return c->seq ? c->seq[3 * b + 1] : c->n_res; }
+int seq_rs(const minikv_cache *c, int b) { return c->seq ? c->seq[3 * b + 2] : c->res_start; }
+
 struct Plan {
     int units, n_rc, spu, P, S_max, Ns;
+    int max_n;   // most tokens any unit attends to this step
 };
 
 Plan plan(const minikv_cache *c) {
     Plan p;
     p.units = c->B * c->Hkv;
-    p.n_rc = (c->n_res + 1 + kResChunk - 1) / kResChunk;
-    p.spu = c->n_packed / kSlice;
-    p.Ns = p.units * p.spu;   // the caller bounds units * cap below 2^31
+    const int nb = c->seq ? c->B : 1;   // distinct sequence states
+    int max_r = 0;
+    long long Ns = 0;
+    p.max_n = 0;
+    for (int b = 0; b < nb; ++b) {
+        const int r = seq_nres(c, b) + 1;
+        if (r > max_r) max_r = r;
+        if (seq_nq(c, b) + r > p.max_n) p.max_n = seq_nq(c, b) + r;
+        Ns += (long long)c->Hkv * (seq_nq(c, b) / kSlice);
+    }
+    if (!c->seq) Ns *= c->B;
+    p.n_rc = (max_r + kResChunk - 1) / kResChunk;
+    p.spu = c->seq ? 0 : c->n_packed / kSlice;   // slices per unit (uniform batches)
+    p.Ns = (int)Ns;                             // the caller bounds units * cap / 32 below 2^31
     p.P = 0;
     if (p.Ns > 0) {
         // packed CTAs fill every resident slot, all in one wave, so that each SM
@@ -817,10 +907,14 @@ Plan plan(const minikv_cache *c) {
     }
     // partial slots per unit: the residual chunks plus the most packed CTAs any unit meets
     int per_unit = 0;
+    long long lo = 0;
     for (int u = 0; p.Ns > 0 && u < p.units; ++u) {
-        const long long lo = (long long)u * p.spu, hi = lo + p.spu - 1;
+        const int spu = seq_nq(c, c->seq ? u / c->Hkv : 0) / kSlice;
+        if (spu == 0) continue;
+        const long long hi = lo + spu - 1;
         const int first = (int)(((lo + 1) * p.P - 1) / p.Ns), last = (int)(((hi + 1) * p.P - 1) / p.Ns);
         if (last - first + 1 > per_unit) per_unit = last - first + 1;
+        lo = hi + 1;
     }
     p.S_max = p.n_rc + per_unit;
     return p;
@@ -842,9 +936,9 @@ size_t decode_workspace_bytes(int B, int Hkv, int max_tokens) {
     return decode_counter_bytes(B, Hkv) + units * (n_rc + per_unit) * 4 * kPartStride * 4;
 }
 
-// Extra workspace of the attention-mass variant: (max, sum) per unit and head,
-// then the log2 scores of up to max_tokens tokens per unit and query head.
-static size_t mass_stats_bytes(int B, int Hkv) { return (((size_t)B * Hkv * 8 * 4 + 255) / 256) * 256; }
+// Extra workspace of the attention-mass variant: per unit max[4], sum[4] and the
+// token count, then the log2 scores of up to max_tokens tokens per unit and query head.
+static size_t mass_stats_bytes(int B, int Hkv) { return (((size_t)B * Hkv * 12 * 4 + 255) / 256) * 256; }
 static size_t mass_scores_bytes(int B, int Hkv, int g, int n_tokens) {
     return (size_t)B * Hkv * g * (size_t)((n_tokens + 3) & ~3) * 4;
 }
@@ -859,22 +953,70 @@ size_t decode_call_workspace_bytes(const minikv_cache *c) {
     return decode_counter_bytes(c->B, c->Hkv) + (size_t)p.units * p.S_max * 4 * kPartStride * 4;
 }
 
+namespace {
+
+template <class A>
+int launch_decode(const A &a, const Plan &p, bool with_mass, cudaStream_t stream);
+
+template <>
+int launch_decode<Args>(const Args &a, const Plan &p, bool with_mass, cudaStream_t stream) {
+    const int grid = p.units * p.n_rc + p.P;
+    if (with_mass) decode_kernel<true><<<grid, kThreads, sizeof(Smem), stream>>>(a);
+    else decode_kernel<false><<<grid, kThreads, sizeof(Smem), stream>>>(a);
+    return check_launch(with_mass ? "decode_attn_mass" : "decode_attn");
+}
+
+template <>
+int launch_decode<ArgsVar>(const ArgsVar &a, const Plan &p, bool with_mass, cudaStream_t stream) {
+    const int grid = p.units * p.n_rc + p.P;
+    if (with_mass) decode_ragged_kernel<true><<<grid, kThreads, sizeof(Smem), stream>>>(a);
+    else decode_ragged_kernel<false><<<grid, kThreads, sizeof(Smem), stream>>>(a);
+    return check_launch(with_mass ? "decode_attn_mass (ragged)" : "decode_attn (ragged)");
+}
+
+int launch_mass(const Args &a, const Plan &p, float *mass, long long mass_stride, cudaStream_t stream) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((p.max_n + 1023) / 1024, p.units);
+    cfg.blockDim = dim3(256);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const float4 *xs = reinterpret_cast<const float4 *>(a.xs);
+    const float *st = a.stats;
+    const int xs_stride4 = a.xs_stride / 4;
+    const bool vec = (mass_stride % 4 == 0) && ((reinterpret_cast<uintptr_t>(mass) & 15u) == 0);
+    switch (a.g) {
+        case 1: cudaLaunchKernelEx(&cfg, mass_kernel<1>, xs, st, mass, xs_stride4, mass_stride, vec); break;
+        case 2: cudaLaunchKernelEx(&cfg, mass_kernel<2>, xs, st, mass, xs_stride4, mass_stride, vec); break;
+        case 3: cudaLaunchKernelEx(&cfg, mass_kernel<3>, xs, st, mass, xs_stride4, mass_stride, vec); break;
+        default: cudaLaunchKernelEx(&cfg, mass_kernel<4>, xs, st, mass, xs_stride4, mass_stride, vec); break;
+    }
+    return check_launch("decode_attn_mass: mass pass");
+}
+
+}  // namespace
+
 int decode_launch(minikv_cache *c, const uint16_t *q, const uint16_t *k_new, const uint16_t *v_new, int Hq,
                   float sm_scale, uint16_t *out, void *ws, size_t ws_bytes, cudaStream_t stream, float *mass) {
     const int g = Hq / c->Hkv;
     const int ring = c->R + c->G;
-    const int r = c->n_res + 1;
-    const int flush = (r == ring) ? 1 : 0;
-    if (flush && c->n_packed + c->G > c->cap)
-        return fail(MINIKV_ERR_CAPACITY, "decode_attn: flushing a key group would exceed cap=%d", c->cap);
+    const int nb = c->seq ? c->B : 1;
+    for (int b = 0; b < nb; ++b)
+        if (seq_nres(c, b) + 1 == ring && seq_nq(c, b) + c->G > c->cap)
+            return fail(MINIKV_ERR_CAPACITY, "decode_attn: flushing a key group of sequence %d would exceed cap=%d",
+                        b, c->cap);
     const Plan p = plan(c);
     const size_t cnt_bytes = decode_counter_bytes(c->B, c->Hkv);
     const size_t part_bytes = (size_t)p.units * p.S_max * 4 * kPartStride * 4;
-    const int n_tok = c->n_packed + r;   // tokens this step attends to
     size_t need = cnt_bytes + part_bytes;
-    if (mass) need += mass_stats_bytes(c->B, c->Hkv) + mass_scores_bytes(c->B, c->Hkv, g, n_tok);
+    if (mass) need += mass_stats_bytes(c->B, c->Hkv) + mass_scores_bytes(c->B, c->Hkv, g, p.max_n);
     if (ws == nullptr || ws_bytes < need)
         return fail(MINIKV_ERR_INVALID_ARG, "decode_attn: workspace of %zu bytes needed, %zu given", need, ws_bytes);
+    const int arc = ensure_attr();
+    if (arc) return arc;
 
     Args a;
     a.k_codes = c->k_codes; a.v_codes = c->v_codes;
@@ -890,55 +1032,44 @@ int decode_launch(minikv_cache *c, const uint16_t *q, const uint16_t *k_new, con
     a.xs = mass ? reinterpret_cast<float *>(static_cast<char *>(ws) + cnt_bytes + part_bytes +
                                             mass_stats_bytes(c->B, c->Hkv))
                 : nullptr;
-    a.xs_stride = (n_tok + 3) & ~3;
+    a.xs_stride = (p.max_n + 3) & ~3;
     a.Hkv = c->Hkv; a.g = g; a.G = c->G; a.cap = c->cap; a.ring = ring;
-    a.n_q = c->n_packed; a.r = r; a.res_start = c->res_start; a.flush = flush;
+    a.n_q = c->n_packed; a.r = c->n_res + 1; a.res_start = c->res_start; a.flush = (a.r == ring);
     a.groups_cap = c->cap / c->G;
     a.lg2G = 31 - __builtin_clz((unsigned)c->G);
     a.units = p.units; a.n_rc = p.n_rc; a.spu = p.spu; a.P = p.P; a.S_max = p.S_max; a.Ns = p.Ns;
     a.scale_log2 = sm_scale * kLog2e;
 
-    const size_t smem = sizeof(Smem);
-    const int arc = ensure_attr();
-    if (arc) return arc;
-    const int grid = p.units * p.n_rc + p.P;
-    if (mass) {
-        decode_kernel<true><<<grid, kThreads, smem, stream>>>(a);
-        int rc = check_launch("decode_attn_mass");
-        if (rc) return rc;
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3((n_tok + 1023) / 1024, p.units);
-        cfg.blockDim = dim3(256);
-        cfg.stream = stream;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attr[0].val.programmaticStreamSerializationAllowed = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        const float4 *xs = reinterpret_cast<const float4 *>(a.xs);
-        const float *st = a.stats;
-        const int xs_stride4 = a.xs_stride / 4;
-        const long long mass_stride = (long long)c->cap + ring;
-        const bool vec = (mass_stride % 4 == 0) && ((reinterpret_cast<uintptr_t>(mass) & 15u) == 0);
-        switch (g) {
-            case 1: cudaLaunchKernelEx(&cfg, mass_kernel<1>, xs, st, mass, n_tok, xs_stride4, mass_stride, vec); break;
-            case 2: cudaLaunchKernelEx(&cfg, mass_kernel<2>, xs, st, mass, n_tok, xs_stride4, mass_stride, vec); break;
-            case 3: cudaLaunchKernelEx(&cfg, mass_kernel<3>, xs, st, mass, n_tok, xs_stride4, mass_stride, vec); break;
-            default: cudaLaunchKernelEx(&cfg, mass_kernel<4>, xs, st, mass, n_tok, xs_stride4, mass_stride, vec); break;
+    int rc;
+    if (c->seq) {
+        ArgsVar av;
+        static_cast<Args &>(av) = a;
+        av.tab.sbeg[0] = 0;
+        for (int b = 0; b < c->B; ++b) {
+            av.tab.n_q[b] = seq_nq(c, b);
+            av.tab.r[b] = seq_nres(c, b) + 1;
+            av.tab.res_start[b] = seq_rs(c, b);
+            av.tab.sbeg[b + 1] = av.tab.sbeg[b] + c->Hkv * (av.tab.n_q[b] / kSlice);
         }
+        rc = launch_decode(av, p, mass != nullptr, stream);
     } else {
-        decode_kernel<false><<<grid, kThreads, smem, stream>>>(a);
+        rc = launch_decode(a, p, mass != nullptr, stream);
     }
-    int rc = check_launch("decode_attn");
     if (rc) return rc;
-    // host-side state
-    c->n_res = r;
-    if (flush) {
-        c->n_packed += c->G;
-        c->n_res -= c->G;
-        c->res_start = (c->res_start + c->G) % ring;
-    }
-    return MINIKV_OK;
+    // host-side state: append, then flush G tokens where the ring is full
+    auto advance = [&](int &n_packed, int &n_res, int &res_start) {
+        n_res += 1;
+        if (n_res == ring) {
+            n_packed += c->G;
+            n_res -= c->G;
+            res_start = (res_start + c->G) % ring;
+        }
+    };
+    if (c->seq)
+        for (int b = 0; b < c->B; ++b) advance(c->seq[3 * b], c->seq[3 * b + 1], c->seq[3 * b + 2]);
+    else
+        advance(c->n_packed, c->n_res, c->res_start);
+    return mass ? launch_mass(a, p, mass, (long long)c->cap + ring, stream) : MINIKV_OK;
 }
 
 }  // namespace minikv

@@ -24,7 +24,7 @@ int check_launch(const char *what) {
 }
 
 int pack_launch(minikv_cache *c, const uint16_t *k, const uint16_t *v, int N, cudaStream_t stream,
-                const int32_t *idx = nullptr, int T = 0);
+                const int32_t *idx = nullptr, int T = 0, int seq = -1);
 int select_launch(const float *scores, int B, int Hkv, int T, int W, int keep, int32_t *idx, cudaStream_t stream);
 int prefill_launch(const uint16_t *q, const uint16_t *k, const uint16_t *v, int B, int Hq, int Hkv, int T, int W,
                    float sm_scale, uint16_t *o, float *scores, void *ws, cudaStream_t stream);
@@ -61,10 +61,21 @@ static int check_cache(const minikv_cache *c) {
     const void *ptrs[8] = {c->k_codes, c->v_codes, c->k_scale, c->k_zero, c->v_scale, c->v_zero, c->k_res, c->v_res};
     for (const void *p : ptrs)
         if (!p || !aligned16(p)) return fail(MINIKV_ERR_INVALID_ARG, "cache array null or not 16-byte aligned");
-    if (c->n_packed < 0 || c->n_packed % c->G || c->n_packed > c->cap || c->n_res < 0 ||
-        c->n_res >= c->R + c->G || c->res_start < 0 || c->res_start >= c->R + c->G)
+    auto bad_state = [&](int n_packed, int n_res, int res_start) {
+        return n_packed < 0 || n_packed % c->G || n_packed > c->cap || n_res < 0 || n_res >= c->R + c->G ||
+               res_start < 0 || res_start >= c->R + c->G;
+    };
+    if (c->seq) {
+        if (c->B > MINIKV_MAX_RAGGED_SEQS)
+            return fail(MINIKV_ERR_UNSUPPORTED, "ragged cache with B=%d above %d", c->B, MINIKV_MAX_RAGGED_SEQS);
+        for (int b = 0; b < c->B; ++b)
+            if (bad_state(c->seq[3 * b], c->seq[3 * b + 1], c->seq[3 * b + 2]))
+                return fail(MINIKV_ERR_INVALID_ARG, "state of sequence %d: n_packed=%d n_res=%d res_start=%d", b,
+                            c->seq[3 * b], c->seq[3 * b + 1], c->seq[3 * b + 2]);
+    } else if (bad_state(c->n_packed, c->n_res, c->res_start)) {
         return fail(MINIKV_ERR_INVALID_ARG, "cache state n_packed=%d n_res=%d res_start=%d", c->n_packed, c->n_res,
                     c->res_start);
+    }
     return MINIKV_OK;
 }
 
@@ -84,8 +95,13 @@ int decode_validate(minikv_cache *c, const uint16_t *q, const uint16_t *k_new, c
     if ((size_t)c->B * c->Hkv > 65535) return fail(MINIKV_ERR_UNSUPPORTED, "decode_attn: B*Hkv above 65535");
     if ((size_t)c->B * c->Hkv * (c->cap / 32) >= (1u << 31))
         return fail(MINIKV_ERR_UNSUPPORTED, "decode_attn: B*Hkv*cap/32 must stay below 2^31");
-    if (c->n_res + 1 == c->R + c->G && c->n_packed + c->G > c->cap)
-        return fail(MINIKV_ERR_CAPACITY, "decode_attn: flushing a key group would exceed cap=%d", c->cap);
+    const int nb = c->seq ? c->B : 1;
+    for (int b = 0; b < nb; ++b) {
+        const int n_packed = c->seq ? c->seq[3 * b] : c->n_packed, n_res = c->seq ? c->seq[3 * b + 1] : c->n_res;
+        if (n_res + 1 == c->R + c->G && n_packed + c->G > c->cap)
+            return fail(MINIKV_ERR_CAPACITY, "decode_attn: flushing a key group of sequence %d would exceed cap=%d",
+                        b, c->cap);
+    }
     return MINIKV_OK;
 }
 
@@ -130,6 +146,19 @@ int minikv_cache_bind(minikv_cache *c, void *base, size_t bytes, int B, int Hkv,
     c->k_res = reinterpret_cast<uint16_t *>(take(u * (R + G) * D * 2));
     c->v_res = reinterpret_cast<uint16_t *>(take(u * (R + G) * D * 2));
     c->n_packed = 0; c->n_res = 0; c->res_start = 0;
+    c->seq = nullptr;
+    return MINIKV_OK;
+}
+
+int minikv_cache_set_ragged(minikv_cache *c, int *seq) {
+    g_err[0] = 0;
+    if (!c) return fail(MINIKV_ERR_INVALID_ARG, "cache_set_ragged: null cache");
+    if (seq && (c->B < 1 || c->B > MINIKV_MAX_RAGGED_SEQS))
+        return fail(MINIKV_ERR_UNSUPPORTED, "cache_set_ragged: B=%d (1..%d)", c->B, MINIKV_MAX_RAGGED_SEQS);
+    c->seq = seq;
+    c->n_packed = 0; c->n_res = 0; c->res_start = 0;
+    if (seq)
+        for (int i = 0; i < 3 * c->B; ++i) seq[i] = 0;
     return MINIKV_OK;
 }
 
@@ -141,6 +170,19 @@ int minikv_quant_pack(minikv_cache *c, const uint16_t *k, const uint16_t *v, int
     if (n_tokens > 0 && (!k || !v || !aligned16(k) || !aligned16(v)))
         return fail(MINIKV_ERR_INVALID_ARG, "quant_pack: k/v null or not 16-byte aligned");
     return pack_launch(c, k, v, n_tokens, static_cast<cudaStream_t>(stream));
+}
+
+int minikv_quant_pack_seq(minikv_cache *c, int b, const uint16_t *k, const uint16_t *v, int n_tokens,
+                          void *stream) {
+    g_err[0] = 0;
+    int rc = check_cache(c);
+    if (rc) return rc;
+    if (!c->seq) return fail(MINIKV_ERR_INVALID_ARG, "quant_pack_seq: the cache is not ragged");
+    if (b < 0 || b >= c->B) return fail(MINIKV_ERR_INVALID_ARG, "quant_pack_seq: sequence %d of %d", b, c->B);
+    if (n_tokens < 0) return fail(MINIKV_ERR_INVALID_ARG, "quant_pack_seq: n_tokens=%d", n_tokens);
+    if (n_tokens > 0 && (!k || !v || !aligned16(k) || !aligned16(v)))
+        return fail(MINIKV_ERR_INVALID_ARG, "quant_pack_seq: k/v null or not 16-byte aligned");
+    return pack_launch(c, k, v, n_tokens, static_cast<cudaStream_t>(stream), nullptr, 0, b);
 }
 
 int minikv_select_prefill(const uint16_t *q, const uint16_t *k, const uint16_t *v, int B, int Hq, int Hkv, int T,
@@ -185,8 +227,10 @@ int minikv_topk_evict(const float *scores, const uint16_t *k, const uint16_t *v,
     return topk_launch(scores, k, v, B, Hkv, T, W, keep, idx, k_kept, v_kept, static_cast<cudaStream_t>(stream));
 }
 
-int minikv_evict_pack(const float *scores, const uint16_t *k, const uint16_t *v, int B, int Hkv, int T, int D, int W,
-                      int keep, int32_t *idx, minikv_cache *c, void *stream) {
+// shared by minikv_evict_pack (seq < 0: B prompts into every sequence) and
+// minikv_evict_pack_seq (one prompt into sequence seq)
+static int evict_pack_impl(const float *scores, const uint16_t *k, const uint16_t *v, int B, int Hkv, int T, int D,
+                           int W, int keep, int32_t *idx, minikv_cache *c, int seq, void *stream) {
     g_err[0] = 0;
     int rc = check_cache(c);
     if (rc) return rc;
@@ -196,9 +240,15 @@ int minikv_evict_pack(const float *scores, const uint16_t *k, const uint16_t *v,
     if (B < 1 || Hkv < 1 || T < 1 || W < 0 || keep < 1)
         return fail(MINIKV_ERR_INVALID_ARG, "evict_pack: B=%d Hkv=%d T=%d W=%d keep=%d", B, Hkv, T, W, keep);
     if (D != kD) return fail(MINIKV_ERR_UNSUPPORTED, "evict_pack: D=%d (only 128)", D);
-    if (B != c->B || Hkv != c->Hkv)
+    if (seq >= 0) {
+        if (!c->seq) return fail(MINIKV_ERR_INVALID_ARG, "evict_pack_seq: the cache is not ragged");
+        if (seq >= c->B) return fail(MINIKV_ERR_INVALID_ARG, "evict_pack_seq: sequence %d of %d", seq, c->B);
+        if (Hkv != c->Hkv)
+            return fail(MINIKV_ERR_INVALID_ARG, "evict_pack_seq: Hkv=%d but the cache has Hkv=%d", Hkv, c->Hkv);
+    } else if (B != c->B || Hkv != c->Hkv) {
         return fail(MINIKV_ERR_INVALID_ARG, "evict_pack: B=%d Hkv=%d but the cache has B=%d Hkv=%d", B, Hkv, c->B,
                     c->Hkv);
+    }
     if (keep < T && W > keep)
         return fail(MINIKV_ERR_INVALID_ARG, "evict_pack: window W=%d above the budget keep=%d", W, keep);
     if ((size_t)B * Hkv > 65535) return fail(MINIKV_ERR_UNSUPPORTED, "evict_pack: B*Hkv above 65535");
@@ -209,7 +259,21 @@ int minikv_evict_pack(const float *scores, const uint16_t *k, const uint16_t *v,
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     rc = select_launch(scores, B, Hkv, T, W, keep, idx, s);
     if (rc) return rc;
-    return pack_launch(c, k, v, n, s, idx, T);
+    return pack_launch(c, k, v, n, s, idx, T, seq);
+}
+
+int minikv_evict_pack(const float *scores, const uint16_t *k, const uint16_t *v, int B, int Hkv, int T, int D, int W,
+                      int keep, int32_t *idx, minikv_cache *c, void *stream) {
+    return evict_pack_impl(scores, k, v, B, Hkv, T, D, W, keep, idx, c, -1, stream);
+}
+
+int minikv_evict_pack_seq(const float *scores, const uint16_t *k, const uint16_t *v, int Hkv, int T, int D, int W,
+                          int keep, int32_t *idx, minikv_cache *c, int b, void *stream) {
+    if (b < 0) {
+        g_err[0] = 0;
+        return fail(MINIKV_ERR_INVALID_ARG, "evict_pack_seq: sequence %d", b);
+    }
+    return evict_pack_impl(scores, k, v, 1, Hkv, T, D, W, keep, idx, c, b, stream);
 }
 
 int minikv_decode_attn(minikv_cache *c, const uint16_t *q, const uint16_t *k_new, const uint16_t *v_new, int Hq,

@@ -27,16 +27,18 @@ struct PackArgs {
     uint16_t *k_scale, *k_zero, *v_scale, *v_zero;
     uint16_t *k_res, *v_res;
     int N, n_q, r, G, Gv, cap, ring, n_groups;
+    int unit0;   // cache unit of grid row 0 (b * Hkv when one sequence of a ragged batch is loaded)
 };
 
 constexpr int kResPerBlock = 32;   // residual tokens copied per block
 
 __global__ void __launch_bounds__(128) pack_kernel(const PackArgs a) {
-    const int unit = blockIdx.y;
+    const int src_unit = blockIdx.y;           // unit of the source tensors
+    const int unit = a.unit0 + blockIdx.y;     // unit of the cache
     const size_t rows = a.idx ? (size_t)a.T : (size_t)a.N;
-    const uint16_t *ku = a.k + (size_t)unit * rows * kD;
-    const uint16_t *vu = a.v + (size_t)unit * rows * kD;
-    const int32_t *iu = a.idx ? a.idx + (size_t)unit * a.N : nullptr;
+    const uint16_t *ku = a.k + (size_t)src_unit * rows * kD;
+    const uint16_t *vu = a.v + (size_t)src_unit * rows * kD;
+    const int32_t *iu = a.idx ? a.idx + (size_t)src_unit * a.N : nullptr;
     auto src_row = [&](int t) -> size_t { return iu ? (size_t)iu[t] : (size_t)t; };   // compacted -> source row
     if ((int)blockIdx.x < a.n_groups) {
         const int grp = blockIdx.x;
@@ -65,9 +67,10 @@ __global__ void __launch_bounds__(128) pack_kernel(const PackArgs a) {
 }  // namespace
 
 // idx == nullptr: k, v are [B,Hkv,N,D]; else k, v are [B,Hkv,T,D] and row t of
-// unit u is idx[u][t] (idx [B,Hkv,N], ascending positions < T).
+// unit u is idx[u][t] (idx [B,Hkv,N], ascending positions < T).  seq >= 0 loads
+// sequence `seq` of a ragged cache only (k, v, idx then without the B axis).
 int pack_launch(minikv_cache *c, const uint16_t *k, const uint16_t *v, int N, cudaStream_t stream,
-                const int32_t *idx, int T) {
+                const int32_t *idx, int T, int seq) {
     int n_q, r;
     if (N >= c->R) {
         r = c->R + (N - c->R) % c->G;
@@ -86,17 +89,30 @@ int pack_launch(minikv_cache *c, const uint16_t *k, const uint16_t *v, int N, cu
     a.k_res = c->k_res; a.v_res = c->v_res;
     a.N = N; a.n_q = n_q; a.r = r; a.G = c->G; a.Gv = c->Gv; a.cap = c->cap; a.ring = c->R + c->G;
     a.n_groups = n_q / c->G;
+    a.unit0 = seq >= 0 ? seq * c->Hkv : 0;
     const int n_res_blocks = (r + kResPerBlock - 1) / kResPerBlock;
     const int gx = a.n_groups + n_res_blocks;
-    const int units = c->B * c->Hkv;
+    const int units = seq >= 0 ? c->Hkv : c->B * c->Hkv;
     if (gx > 0 && units > 0) {
         pack_kernel<<<dim3(gx, units), 128, 0, stream>>>(a);
         int rc = check_launch("quant_pack");
         if (rc) return rc;
     }
+    if (seq >= 0) {
+        c->seq[3 * seq] = n_q;
+        c->seq[3 * seq + 1] = r;
+        c->seq[3 * seq + 2] = 0;
+        return MINIKV_OK;
+    }
     c->n_packed = n_q;
     c->n_res = r;
     c->res_start = 0;
+    if (c->seq)
+        for (int b = 0; b < c->B; ++b) {
+            c->seq[3 * b] = n_q;
+            c->seq[3 * b + 1] = r;
+            c->seq[3 * b + 2] = 0;
+        }
     return MINIKV_OK;
 }
 

@@ -33,13 +33,18 @@ class CacheStruct(ctypes.Structure):
     _fields_ = [("B", _I), ("Hkv", _I), ("D", _I), ("G", _I), ("Gv", _I), ("R", _I), ("cap", _I),
                 ("k_codes", _P), ("v_codes", _P), ("k_scale", _P), ("k_zero", _P),
                 ("v_scale", _P), ("v_zero", _P), ("k_res", _P), ("v_res", _P),
-                ("n_packed", _I), ("n_res", _I), ("res_start", _I)]
+                ("n_packed", _I), ("n_res", _I), ("res_start", _I), ("seq", _P)]
+
+MAX_RAGGED_SEQS = 256
 
 
 _SIGS = {
     "minikv_cache_bytes": (_Z, [_I, _I, _I, _I, _I, _I, _I]),
     "minikv_cache_bind": (_I, [ctypes.POINTER(CacheStruct), _P, _Z, _I, _I, _I, _I, _I, _I, _I]),
+    "minikv_cache_set_ragged": (_I, [ctypes.POINTER(CacheStruct), _P]),
     "minikv_quant_pack": (_I, [ctypes.POINTER(CacheStruct), _P, _P, _I, _P]),
+    "minikv_quant_pack_seq": (_I, [ctypes.POINTER(CacheStruct), _I, _P, _P, _I, _P]),
+    "minikv_evict_pack_seq": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, ctypes.POINTER(CacheStruct), _I, _P]),
     "minikv_select_prefill": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P, _Z, _P]),
     "minikv_topk_evict": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _Z, _P]),
     "minikv_evict_pack": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, ctypes.POINTER(CacheStruct), _P]),
@@ -117,6 +122,23 @@ class MiniKVCache:
             ws = torch.zeros(workspace_size(OP_DECODE_ATTN, B, Hq or Hkv, Hkv, cap + R + G, D),
                              dtype=torch.uint8, device=device)
         self.ws = ws
+        self._seq = None
+
+    def set_ragged(self) -> "MiniKVCache":
+        """Give every sequence its own length (per-sequence host state, all empty)."""
+        self._seq = (ctypes.c_int * (3 * self.B))()
+        _check(lib().minikv_cache_set_ragged(ctypes.byref(self.c), ctypes.cast(self._seq, _P)))
+        return self
+
+    @property
+    def ragged(self) -> bool:
+        return self._seq is not None
+
+    def seq_state(self, b: int) -> tuple[int, int, int]:
+        """(n_packed, n_res, res_start) of sequence b (either kind of batch)."""
+        if self._seq is None:
+            return self.n_packed, self.n_res, self.res_start
+        return self._seq[3 * b], self._seq[3 * b + 1], self._seq[3 * b + 2]
 
     # shape / state
     B = property(lambda s: s.c.B)
@@ -150,19 +172,33 @@ class MiniKVCache:
             v_res=self._view(self.c.v_res, torch.float16, (B, H, ring, D)))
 
     def residual(self) -> tuple[torch.Tensor, torch.Tensor]:
-        """Residual tokens in logical order (oldest first): [B, Hkv, n_res, D]."""
+        """Residual tokens in logical order (oldest first): [B, Hkv, n_res, D] (uniform batch)."""
         a = self.arrays()
         ring = self.R + self.G
         idx = torch.tensor([(self.res_start + i) % ring for i in range(self.n_res)], device=self.device,
                            dtype=torch.long)
         return a["k_res"][:, :, idx], a["v_res"][:, :, idx]
 
+    def residual_seq(self, b: int) -> tuple[torch.Tensor, torch.Tensor]:
+        """Residual tokens of sequence b in logical order: [Hkv, n_res_b, D]."""
+        a = self.arrays()
+        ring = self.R + self.G
+        _, n_res, rs = self.seq_state(b)
+        idx = torch.tensor([(rs + i) % ring for i in range(n_res)], device=self.device, dtype=torch.long)
+        return a["k_res"][b][:, idx], a["v_res"][b][:, idx]
+
     def byte_counts(self) -> dict:
-        """Algorithmic bytes a decode step reads for this state, per (b, KV head)."""
+        """Algorithmic bytes the next decode step reads, per (b, KV head) of a
+        uniform batch; on a ragged batch, summed over all units ('total')."""
         D, G, Gv = self.D, self.G, self.Gv
-        nq, r = self.n_packed, self.n_res + 1
-        packed = nq * (D // 4) * 2 + (nq // G) * D * 4 + nq * (D // Gv) * 4
-        return dict(packed=packed, residual=r * D * 4, per_unit=packed + r * D * 4)
+
+        def unit(nq, r):
+            return nq * (D // 4) * 2 + (nq // G) * D * 4 + nq * (D // Gv) * 4, r * D * 4
+        if self._seq is None:
+            packed, res = unit(self.n_packed, self.n_res + 1)
+            return dict(packed=packed, residual=res, per_unit=packed + res, total=(packed + res) * self.B * self.Hkv)
+        tot = sum(sum(unit(self._seq[3 * b], self._seq[3 * b + 1] + 1)) for b in range(self.B)) * self.Hkv
+        return dict(total=tot)
 
 
 def quant_pack(cache: MiniKVCache, k: torch.Tensor, v: torch.Tensor, stream=None) -> None:
@@ -173,6 +209,30 @@ def quant_pack(cache: MiniKVCache, k: torch.Tensor, v: torch.Tensor, stream=None
     kp = _dev(k, torch.float16, "k") if N else None
     vp = _dev(v, torch.float16, "v") if N else None
     _check(lib().minikv_quant_pack(ctypes.byref(cache.c), kp, vp, N, _stream(stream, cache.device)))
+
+
+def quant_pack_seq(cache: MiniKVCache, b: int, k: torch.Tensor, v: torch.Tensor, stream=None) -> None:
+    """Load sequence b of a ragged cache: k, v [Hkv, N, D] fp16 (N of its own)."""
+    N = k.shape[1] if k.dim() == 3 else 0
+    if k.shape != v.shape or k.shape[0] != cache.Hkv or k.shape[2] != cache.D:
+        raise ValueError(f"k/v shape {tuple(k.shape)} does not match the cache")
+    kp = _dev(k, torch.float16, "k") if N else None
+    vp = _dev(v, torch.float16, "v") if N else None
+    _check(lib().minikv_quant_pack_seq(ctypes.byref(cache.c), b, kp, vp, N, _stream(stream, cache.device)))
+
+
+def evict_pack_seq(cache: MiniKVCache, b: int, scores: torch.Tensor, k: torch.Tensor, v: torch.Tensor, W: int,
+                   keep: int, idx: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """One prompt (scores [Hkv, T], k, v [Hkv, T, D]) kept and packed into
+    sequence b of a ragged cache; returns idx [Hkv, min(keep, T)]."""
+    Hkv, T, D = k.shape
+    n = min(keep, T)
+    if idx is None:
+        idx = torch.empty((Hkv, n), dtype=torch.int32, device=k.device)
+    _check(lib().minikv_evict_pack_seq(
+        _dev(scores, torch.float32, "scores"), _dev(k, torch.float16, "k"), _dev(v, torch.float16, "v"),
+        Hkv, T, D, W, keep, _dev(idx, torch.int32, "idx"), ctypes.byref(cache.c), b, _stream(stream, k.device)))
+    return idx
 
 
 def select_prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, W: int, sm_scale: float | None = None,

@@ -65,9 +65,15 @@ extern "C" {
  *   k_res, v_res     [B, Hkv, R+G, D] fp16: ring of the newest tokens, kept in
  *       fp16; logical residual token i (0 = oldest) is in slot
  *       (res_start + i) mod (R+G).
- * Host-side state (same for every sequence and head of the layer): n_packed
- * packed tokens (a multiple of G), n_res residual tokens, ring origin
- * res_start.  Calls update it synchronously when they queue their work.
+ * Host-side state: n_packed packed tokens (a multiple of G), n_res residual
+ * tokens, ring origin res_start.  Calls update it synchronously when they
+ * queue their work.
+ *   - Uniform batch (seq == NULL): one state for every sequence and head.
+ *   - Ragged batch (seq != NULL, see minikv_cache_set_ragged): seq is a HOST
+ *     array [B][3] = (n_packed, n_res, res_start) per sequence, owned by the
+ *     caller and kept alive while the cache is used; the three scalars are then
+ *     not read.  Sequences of one batch may hold different numbers of packed
+ *     and residual tokens (unequal prompts, unequal budgets).
  * Dequantized value of a code c: c * scale + zero.
  */
 typedef struct minikv_cache {
@@ -77,7 +83,11 @@ typedef struct minikv_cache {
     uint16_t *v_scale, *v_zero;
     uint16_t *k_res, *v_res;
     int n_packed, n_res, res_start;
+    int *seq;
 } minikv_cache;
+
+/* Most sequences a ragged batch may hold. */
+#define MINIKV_MAX_RAGGED_SEQS 256
 
 /* Bytes of device memory one layer's cache needs (each array 256-byte aligned),
  * or 0 if the shape is invalid. */
@@ -85,9 +95,24 @@ MINIKV_API size_t minikv_cache_bytes(int B, int Hkv, int D, int G, int Gv, int R
 
 /* Fill *c with the shape, point its arrays into `base` (a device buffer of at
  * least minikv_cache_bytes(...) bytes, 256-byte aligned) and reset the state to
- * empty.  Touches no device memory. */
+ * empty (uniform batch, seq = NULL).  Touches no device memory. */
 MINIKV_API int minikv_cache_bind(minikv_cache *c, void *base, size_t bytes,
                       int B, int Hkv, int D, int G, int Gv, int R, int cap);
+
+/*
+ * minikv_cache_set_ragged -- give each sequence of the batch its own length.
+ * Source: none on the pages (they state no batching rule); serving batches
+ * prompts of unequal length, so each sequence keeps its own packed and
+ * residual counts.
+ *   seq: HOST array of 3*B ints, caller-owned, alive while the cache is used;
+ *   every sequence is reset to empty (0, 0, 0).  seq = NULL turns the cache
+ *   back into a uniform batch, also empty.  Touches no device memory.
+ * Afterwards minikv_quant_pack / minikv_evict_pack set every sequence (same
+ * length for all), minikv_quant_pack_seq / minikv_evict_pack_seq set one, and
+ * the decode calls step every sequence from its own state.
+ * Errors: INVALID_ARG (null cache), UNSUPPORTED (B > MINIKV_MAX_RAGGED_SEQS).
+ */
+MINIKV_API int minikv_cache_set_ragged(minikv_cache *c, int *seq);
 
 /*
  * minikv_quant_pack -- load a fresh compacted sequence into the cache.
@@ -108,6 +133,17 @@ MINIKV_API int minikv_cache_bind(minikv_cache *c, void *base, size_t bytes,
  */
 MINIKV_API int minikv_quant_pack(minikv_cache *c, const uint16_t *k, const uint16_t *v,
                       int n_tokens, void *stream);
+
+/*
+ * minikv_quant_pack_seq -- minikv_quant_pack for sequence b of a ragged cache
+ * only: k, v [Hkv, n_tokens, D] fp16 become sequence b's kept tokens (same
+ * split and quantizer); seq[b] = (n_tokens - r, r, 0).  Other sequences are
+ * untouched.
+ * Errors: as minikv_quant_pack; INVALID_ARG also if the cache is not ragged or
+ * b is outside [0, B).
+ */
+MINIKV_API int minikv_quant_pack_seq(minikv_cache *c, int b, const uint16_t *k, const uint16_t *v,
+                                     int n_tokens, void *stream);
 
 /*
  * minikv_select_prefill -- "selective flash attention" over the prompt.
@@ -174,6 +210,17 @@ MINIKV_API int minikv_evict_pack(const float *scores, const uint16_t *k, const u
                       int32_t *idx, minikv_cache *c, void *stream);
 
 /*
+ * minikv_evict_pack_seq -- minikv_evict_pack of ONE prompt (scores [Hkv, T],
+ * k, v [Hkv, T, D], idx [Hkv, min(keep, T)]) into sequence b of a ragged
+ * cache; T and keep are this prompt's own.  Other sequences are untouched.
+ * Errors: as minikv_evict_pack; INVALID_ARG also if the cache is not ragged or
+ * b is outside [0, B).
+ */
+MINIKV_API int minikv_evict_pack_seq(const float *scores, const uint16_t *k, const uint16_t *v,
+                                     int Hkv, int T, int D, int W, int keep, int32_t *idx,
+                                     minikv_cache *c, int b, void *stream);
+
+/*
  * minikv_decode_attn -- one decoding step of one layer over the 2-bit cache.
  * Source: abstract ("specialized CUDA kernels ... compatible with
  * FlashAttention"); summary page, 方法论 (the compact 2-bit layout it reads).
@@ -187,6 +234,9 @@ MINIKV_API int minikv_evict_pack(const float *scores, const uint16_t *k, const u
  * 3. If the residual now holds R+G tokens, its oldest G are quantized (same
  *    rules as minikv_quant_pack) into key group n_packed/G: n_packed += G,
  *    n_res -= G.
+ * On a ragged cache every step runs per sequence, from and into its own state
+ * (one launch for the whole batch; the split of packed tokens over CTAs
+ * follows the actual per-sequence lengths).
  *   ws: minikv_workspace_size(MINIKV_OP_DECODE_ATTN, B, Hq, Hkv, cap, D, 0)
  *       bytes, ZERO-FILLED before its first use; every call leaves it ready for
  *       the next (its arrival counters return to zero).  Calls that share one

@@ -140,3 +140,48 @@ def test_evict_pack_argument_errors():
     # misaligned K
     assert L.minikv_evict_pack(p, p + 2, p, 1, 2, 512, 128, 32, 96, p, ctypes.byref(c), None) == mk.ERR_INVALID_ARG
     assert (c.n_packed, c.n_res, c.res_start) == (0, 0, 0)   # the cache state is untouched on error
+
+
+def test_ragged_cache_state_and_argument_errors():
+    """Per-sequence host state: set_ragged resets it, the loaders reject a
+    non-ragged cache or a bad row, and a bad per-sequence state is refused
+    before any launch."""
+    L = mk.lib()
+    p = 1 << 24
+    c = _bound_cache(B=3, Hkv=2, cap=256)
+    assert c.seq is None
+    # loaders of one sequence need a ragged cache
+    assert L.minikv_quant_pack_seq(ctypes.byref(c), 0, p, p, 10, None) == mk.ERR_INVALID_ARG
+    assert L.minikv_evict_pack_seq(p, p, p, 2, 512, 128, 32, 96, p, ctypes.byref(c), 0, None) == mk.ERR_INVALID_ARG
+    seq = (ctypes.c_int * 9)(*range(1, 10))
+    assert L.minikv_cache_set_ragged(ctypes.byref(c), ctypes.cast(seq, ctypes.c_void_p)) == 0
+    assert list(seq) == [0] * 9
+    assert c.seq is not None
+    # row outside [0, B); capacity of one row; Hkv mismatch; negative row
+    assert L.minikv_quant_pack_seq(ctypes.byref(c), 3, p, p, 10, None) == mk.ERR_INVALID_ARG
+    assert L.minikv_quant_pack_seq(ctypes.byref(c), -1, p, p, 10, None) == mk.ERR_INVALID_ARG
+    assert L.minikv_quant_pack_seq(ctypes.byref(c), 1, p, p, 400, None) == mk.ERR_CAPACITY
+    assert L.minikv_evict_pack_seq(p, p, p, 3, 512, 128, 32, 96, p, ctypes.byref(c), 0, None) == mk.ERR_INVALID_ARG
+    assert L.minikv_evict_pack_seq(p, p, p, 2, 512, 128, 32, 96, p, ctypes.byref(c), -2, None) == mk.ERR_INVALID_ARG
+    assert L.minikv_evict_pack_seq(p, p, p, 2, 512, 128, 32, 330, p, ctypes.byref(c), 2, None) == mk.ERR_CAPACITY
+    assert list(seq) == [0] * 9
+    # an inconsistent state of one sequence, and a flush past capacity in one sequence
+    seq[3 * 1] = 17
+    assert L.minikv_decode_attn(ctypes.byref(c), p, p, p, 2, 0.1, p, p, 1 << 20, None) == mk.ERR_INVALID_ARG
+    assert b"sequence 1" in L.minikv_last_error_string()
+    seq[3 * 1] = 0
+    seq[3 * 2], seq[3 * 2 + 1] = 256, 32 + 32 - 1
+    assert L.minikv_decode_attn(ctypes.byref(c), p, p, p, 2, 0.1, p, p, 1 << 20, None) == mk.ERR_CAPACITY
+    assert b"sequence 2" in L.minikv_last_error_string()
+    assert (seq[6], seq[7]) == (256, 63)
+    # back to a uniform batch
+    assert L.minikv_cache_set_ragged(ctypes.byref(c), None) == 0
+    assert c.seq is None and (c.n_packed, c.n_res, c.res_start) == (0, 0, 0)
+
+
+def test_ragged_batch_limit():
+    L = mk.lib()
+    c = _bound_cache(B=mk.MAX_RAGGED_SEQS + 1, Hkv=1, cap=64)
+    seq = (ctypes.c_int * (3 * (mk.MAX_RAGGED_SEQS + 1)))()
+    assert L.minikv_cache_set_ragged(ctypes.byref(c), ctypes.cast(seq, ctypes.c_void_p)) == mk.ERR_UNSUPPORTED
+    assert c.seq is None
