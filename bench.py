@@ -10,6 +10,10 @@ kept and packed 2-bit (key group G=32, value group 128, fp16 residual R=128).
 A step is one generated token for the whole batch through all 32 layers: per
 layer one minikv_decode_attn call (append the new token, attend over the
 packed + residual cache, flush a key group to 2 bits every G steps).  The
+calls are made one per layer from Python (host-side state), or, with
+`--launch graph` (the default for the ragged workload), the caches keep their
+per-sequence state on the GPU and the 32 calls of a step are captured once in a
+CUDA graph and replayed every step.  The
 per-layer caches (2.5 GB per step) are walked in order, so the working set is
 far larger than the 126 MB L2.  The same run also times the prompt rows of
 the path on a LLaMA2-7B-shaped prefill (32 layers x 32 heads, 4096 tokens,
@@ -52,6 +56,11 @@ DECODE_PRESETS = {
     # every token kept, only quantized (the KIVI-like point of the method): 32K context
     "quant_only_32k_decode": dict(workload="quant_only_32k_decode", layers=32, batch=16, q_heads=32, kv_heads=8,
                                   head_dim=128, context=32768, keep_pct=100, G=32, Gv=128, R=128),
+    # ragged batch: the 16 prompts' contexts rise evenly from 4K to 32K tokens, 20 % kept of each
+    "mistral7b_gqa_ragged_decode": dict(workload="mistral7b_gqa_ragged_decode", layers=32, batch=16, q_heads=32,
+                                        kv_heads=8, head_dim=128, context="4096..32768 (even ramp over the batch)",
+                                        contexts=[4096 + (32768 - 4096) * b // 15 for b in range(16)],
+                                        keep_pct=20, G=32, Gv=128, R=128),
 }
 PREFILL_PRESETS = {
     "llama2_7b_prefill_select": dict(workload="llama2_7b_prefill_select", layers=32, batch=1, q_heads=32,
@@ -202,7 +211,17 @@ def cpu_tokens_per_s(rate):
     return rate * DECODE["batch"] / units_per_step
 
 
+def seq_keeps():
+    """Kept tokens per sequence of a ragged workload (None for uniform batches)."""
+    if "contexts" not in DECODE:
+        return None
+    return [keep_of(t, DECODE["keep_pct"]) for t in DECODE["contexts"]]
+
+
 def decode_keeps():
+    """Kept tokens per layer (the longest sequence's, for a ragged batch)."""
+    if "contexts" in DECODE:
+        return [max(seq_keeps())] * DECODE["layers"]
     return [keep_of(DECODE["context"], DECODE["keep_pct"], l, DECODE["layers"]) for l in range(DECODE["layers"])]
 
 
@@ -210,6 +229,10 @@ def decode_config(extra=None, step_bytes=None):
     c = {k: v for k, v in DECODE.items()}
     keeps = decode_keeps()
     c["keep"] = keeps[0] if len(set(keeps)) == 1 else f"{keeps[0]}..{keeps[-1]} (per layer)"
+    if "contexts" in DECODE:
+        sk = seq_keeps()
+        c.pop("contexts")
+        c["keep"] = f"{min(sk)}..{max(sk)} (per sequence, mean {sum(sk) / len(sk):.0f})"
     gb = (step_bytes or 0) / 1e9
     c["l2"] = (f"inputs larger than L2: {DECODE['layers']} distinct layer caches, {gb:.2f} GB read per step"
                if step_bytes else f"inputs larger than L2: {DECODE['layers']} distinct layer caches")
@@ -257,16 +280,29 @@ def make_decode_state(torch, mk, synth, device, warmup, steps):
     ws = torch.zeros(mk.workspace_size(op, B, Hq, Hkv, cap_max + R + G), dtype=torch.uint8, device=device)
     wid = 4 if DECODE["workload"] == "mistral7b_gqa_decode" else 40 + list(DECODE_PRESETS).index(DECODE["workload"])
     caches = []
+    sk = seq_keeps()
     for l in range(L):
         N = keeps[l]
         cap = ((N + total_steps) // G + 2) * G
-        k = torch.empty((B, Hkv, N, 128), dtype=torch.float16, device=device)
-        v = torch.empty_like(k)
-        for b in range(B):
-            k[b] = synth.keys_fp16((Hkv, N, 128), synth.seed_of(wid, l, synth.T_K, 0, b), device)
-            v[b] = synth.normal_fp16((Hkv, N, 128), synth.seed_of(wid, l, synth.T_V, 0, b), device)
         c = mk.MiniKVCache(B, Hkv, cap, G=G, Gv=Gv, R=R, Hq=Hq, device=device, ws=ws)
-        mk.quant_pack(c, k, v)
+        if not DECODE.get("eager"):
+            c.set_device_state()   # per-sequence state on the GPU: steps replay from CUDA graphs
+        elif sk is not None:
+            c.set_ragged()
+        if sk is not None:   # ragged: each sequence loaded into its own row with its own length
+            for b in range(B):
+                kb = synth.keys_fp16((Hkv, sk[b], 128), synth.seed_of(wid, l, synth.T_K, 0, b), device)
+                vb = synth.normal_fp16((Hkv, sk[b], 128), synth.seed_of(wid, l, synth.T_V, 0, b), device)
+                mk.quant_pack_seq(c, b, kb, vb)
+                del kb, vb
+            k = v = None
+        else:
+            k = torch.empty((B, Hkv, N, 128), dtype=torch.float16, device=device)
+            v = torch.empty_like(k)
+            for b in range(B):
+                k[b] = synth.keys_fp16((Hkv, N, 128), synth.seed_of(wid, l, synth.T_K, 0, b), device)
+                v[b] = synth.normal_fp16((Hkv, N, 128), synth.seed_of(wid, l, synth.T_V, 0, b), device)
+            mk.quant_pack(c, k, v)
         # H2O-style running attention mass per token (--mass)
         c.mass = torch.zeros((B, Hkv, cap + R + G), dtype=torch.float32, device=device) if DECODE.get("mass") else None
         caches.append(c)
@@ -286,11 +322,41 @@ def make_decode_state(torch, mk, synth, device, warmup, steps):
     return caches, ws, qin, knin, vnin, out
 
 
-def unit_bytes(c):
-    n = BYTES_PER_PACKED * c.n_packed + BYTES_PER_RESIDUAL * (c.n_res + 1)
-    if c.mass is not None:   # read and write of one fp32 running score per token
-        n += 8 * (c.n_packed + c.n_res + 1)
-    return n
+class LengthMirror:
+    """Host copy of every layer's per-sequence (n_packed, n_res), advanced the
+    way a decode step advances the cache (append; flush G tokens when the ring
+    of R+G is full), so that the algorithmic bytes of each step are known
+    without reading the GPU's state."""
+
+    def __init__(self, layer_lengths, G, R):
+        self.G, self.ring = G, R + G
+
+        def split(N):
+            if N < R:
+                return [0, N]
+            r = R + (N - R) % G
+            return [N - r, r]
+        self.st = [[split(N) for N in lens] for lens in layer_lengths]
+
+    def layer_bytes(self, l, Hkv, mass):
+        """Bytes one layer-step reads: per (sequence, KV head) unit its packed and
+        residual tokens (and one fp32 running score read and written per token
+        with --mass)."""
+        total = 0
+        for nq, nr in self.st[l]:
+            n = BYTES_PER_PACKED * nq + BYTES_PER_RESIDUAL * (nr + 1)
+            if mass:
+                n += 8 * (nq + nr + 1)
+            total += n * Hkv
+        return total
+
+    def advance(self):
+        for layer in self.st:
+            for s in layer:
+                s[1] += 1
+                if s[1] == self.ring:
+                    s[0] += self.G
+                    s[1] -= self.G
 
 
 def decode_call(mk, c, q, kn, vn, out, ws):
@@ -387,28 +453,49 @@ def run_gpu(args):
 
     mk.lib()
     pk = peaks()
-    L, B = DECODE["layers"], DECODE["batch"]
+    L, B, Hkv = DECODE["layers"], DECODE["batch"], DECODE["kv_heads"]
     caches, ws, qin, knin, vnin, out = make_decode_state(torch, mk, synth, device, args.warmup, args.steps)
+    sk = seq_keeps()
+    mirror = LengthMirror([sk if sk is not None else [n] * B for n in decode_keeps()], DECODE["G"], DECODE["R"])
+    with_mass = bool(DECODE.get("mass"))
+    eager = bool(DECODE.get("eager"))
     P = qin.shape[0]
-    stream = torch.cuda.current_stream(device)
 
-    def step(s, q_src, kn_src, vn_src, ev=None, nbytes=None):
-        p = s % P
+    def layer_calls(q_src, kn_src, vn_src, p, ev=None, o=None):
+        """One decode step: the L layer calls, on the current stream."""
+        o = out if o is None else o
         for l in range(L):
-            if nbytes is not None:
-                nbytes.append(unit_bytes(caches[l]) * B * DECODE["kv_heads"])
             if ev is not None:
-                ev[l][0].record(stream)
-            decode_call(mk, caches[l], q_src[p, l], kn_src[p, l], vn_src[p, l], out[l], ws)
+                ev[l][0].record()
+            decode_call(mk, caches[l], q_src[p, l], kn_src[p, l], vn_src[p, l], o[l], ws)
             if ev is not None:
-                ev[l][1].record(stream)
+                ev[l][1].record()
+
+    def step_bytes():
+        return [mirror.layer_bytes(l, Hkv, with_mass) for l in range(L)]
 
     for s in range(args.warmup):
-        step(s, qin, knin, vnin)
+        layer_calls(qin, knin, vnin, s % P)
+        mirror.advance()
     torch.cuda.synchronize()
 
+    # Graph mode (default): the caches keep their state on the GPU, so one
+    # captured step per input-pool slot replays correctly at every later step.
+    # Timing events are recorded between replays, not inside the graphs (event
+    # nodes inside a graph would sit between the kernels and slow the step).
+    graphs = []
+    if not eager:
+        for p in range(P):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                layer_calls(qin, knin, vnin, p)
+            graphs.append(g)
+        torch.cuda.synchronize()
+
     # ---- device-timed region
+    stream = torch.cuda.current_stream(device)
     evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(L)] for _ in range(args.steps)]
+    sev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
     nbytes = []
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
@@ -416,52 +503,95 @@ def run_gpu(args):
     with ClockSampler(local) as clk:
         t0.record(stream)
         for s in range(args.steps):
-            step(args.warmup + s, qin, knin, vnin, ev=evs[s], nbytes=nbytes)
+            p = (args.warmup + s) % P
+            nbytes.append(step_bytes())
+            if eager:
+                layer_calls(qin, knin, vnin, p, evs[s])
+            else:
+                sev[s][0].record(stream)
+                graphs[p].replay()
+                sev[s][1].record(stream)
+            mirror.advance()
         t1.record(stream)
         torch.cuda.synchronize()
     barrier()
     ms = t0.elapsed_time(t1)
-    kern_ms = [evs[s][l][0].elapsed_time(evs[s][l][1]) for s in range(args.steps) for l in range(L)]
+    launch_bytes = [b for sb in nbytes for b in sb]
+    if eager:
+        kern_ms = [evs[s][l][0].elapsed_time(evs[s][l][1]) for s in range(args.steps) for l in range(L)]
+    else:   # a replay runs the L layer launches back to back: its time / L per launch (gaps included)
+        kern_ms = [sev[s][0].elapsed_time(sev[s][1]) / L for s in range(args.steps)]
     if world > 1:
         t = torch.tensor([ms], device=device)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms = float(t.item())
     tok_s = B * args.steps * world / (ms * 1e-3)
-    alg_bytes = sum(nbytes)
-    mean_launch_bytes = alg_bytes / len(nbytes)
+    alg_bytes = sum(sum(sb) for sb in nbytes)
+    mean_launch_bytes = sum(launch_bytes) / len(launch_bytes)
     mean_launch_s = statistics.mean(kern_ms) * 1e-3
     achieved = mean_launch_bytes / mean_launch_s / 1e9
     step_gbs = alg_bytes / (ms * 1e-3) / 1e9
+    del graphs
 
-    # ---- end to end: inputs from pinned host memory, outputs back, each step
+    # ---- end to end: inputs from pinned host memory, outputs back, each step.
+    # Two buffer sets: while step s computes, a copy stream brings step s+1's
+    # inputs in and takes step s-1's outputs out (stream order and events keep
+    # each buffer's copies and its compute apart).
     hq = qin.cpu().pin_memory()
     hk = knin.cpu().pin_memory()
     hv = vnin.cpu().pin_memory()
-    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    dq, dk, dv = torch.empty_like(qin[:1]), torch.empty_like(knin[:1]), torch.empty_like(vnin[:1])
-    h2d = (dq.numel() + dk.numel() + dv.numel()) * 2
+    dq = [torch.empty_like(qin[:1]) for _ in range(2)]
+    dk = [torch.empty_like(knin[:1]) for _ in range(2)]
+    dv = [torch.empty_like(vnin[:1]) for _ in range(2)]
+    dout = [torch.empty_like(out) for _ in range(2)]
+    hout = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
+    h2d = (dq[0].numel() + dk[0].numel() + dv[0].numel()) * 2
     d2h = out.numel() * 2
+    g_e2e = []
+    if not eager:
+        for i in range(2):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                layer_calls(dq[i], dk[i], dv[i], 0, o=dout[i])
+            g_e2e.append(g)
+    copy = torch.cuda.Stream(device)
+    in_ready = [torch.cuda.Event() for _ in range(2)]
+    done = [torch.cuda.Event() for _ in range(2)]
     torch.cuda.synchronize()
     barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
+    copy.wait_stream(stream)
     for s in range(args.steps):
-        p = s % P
-        dq.copy_(hq[p:p + 1], non_blocking=True)
-        dk.copy_(hk[p:p + 1], non_blocking=True)
-        dv.copy_(hv[p:p + 1], non_blocking=True)
-        for l in range(L):
-            decode_call(mk, caches[l], dq[0, l], dk[0, l], dv[0, l], out[l], ws)
-        hout.copy_(out, non_blocking=True)
+        i, p = s % 2, s % P
+        with torch.cuda.stream(copy):
+            dq[i].copy_(hq[p:p + 1], non_blocking=True)
+            dk[i].copy_(hk[p:p + 1], non_blocking=True)
+            dv[i].copy_(hv[p:p + 1], non_blocking=True)
+            in_ready[i].record(copy)
+        stream.wait_event(in_ready[i])
+        if eager:
+            layer_calls(dq[i], dk[i], dv[i], 0, o=dout[i])
+        else:
+            g_e2e[i].replay()
+        done[i].record(stream)
+        with torch.cuda.stream(copy):
+            copy.wait_event(done[i])
+            hout[i].copy_(dout[i], non_blocking=True)
+    stream.wait_stream(copy)
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
+    del g_e2e
     e2e_ms = e0.elapsed_time(e1)
     if world > 1:
         t = torch.tensor([e2e_ms], device=device)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         e2e_ms = float(t.item())
     e2e_tok_s = B * args.steps * world / (e2e_ms * 1e-3)
+    status_bad = sum(sum(c.status()) for c in caches)
+    if status_bad:
+        raise RuntimeError(f"{status_bad} sequences hit the cache capacity")
 
     prefill = run_prefill(torch, mk, synth, device) if not args.no_prefill else None
     if prefill:
@@ -487,7 +617,10 @@ def run_gpu(args):
             "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "u2+f16 (2-bit codes, fp16 scales/residual, fp32 accumulate)",
             "data": "synthetic",
-            "config": decode_config({"parallelism": f"replicas x{world}"}, step_bytes=alg_bytes / args.steps),
+            "config": decode_config({"parallelism": f"replicas x{world}",
+                                     "launch": "eager: one Python call per layer" if eager else
+                                     "one CUDA graph replay per step (32 captured layer calls, state on the GPU)"},
+                                    step_bytes=alg_bytes / args.steps),
             "hbm_gbs": step_gbs, "hbm_frac_of_peak": step_gbs / pk["hbm"],
             "roofline": {"bound": "hbm", "kernel": "decode_kernel", "achieved": achieved, "peak": pk["hbm"],
                          "unit": "GB/s", "frac": achieved / pk["hbm"], "traffic": traffic,
@@ -516,6 +649,10 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--workload", default="mistral7b_gqa_decode", choices=list(DECODE_PRESETS),
                     help="decode workload (the default one carries the bench line's target)")
+    ap.add_argument("--launch", default="auto", choices=["auto", "graph", "eager"],
+                    help="graph: state on the GPU, one captured CUDA graph replayed per step; eager: one Python "
+                         "call per layer, host-side state; auto: graph for ragged batches (eager is host-bound "
+                         "there), eager otherwise (its kernel is a little faster)")
     ap.add_argument("--mass", action="store_true",
                     help="decode with minikv_decode_attn_mass (H2O-style running attention mass per token)")
     ap.add_argument("--prefill-workload", default="llama2_7b_prefill_select", choices=list(PREFILL_PRESETS))
@@ -532,6 +669,8 @@ def main():
         DECODE["layers"] = args.layers
     if args.mass:
         DECODE["mass"] = True
+    if args.launch == "eager" or (args.launch == "auto" and "contexts" not in DECODE):
+        DECODE["eager"] = True
     if args.prefill_layers is not None:
         PREFILL["layers"] = args.prefill_layers
     if args.warmup < 3:

@@ -148,14 +148,15 @@ __device__ __forceinline__ float canon_zero(float x) { return __fadd_rn(x, 0.0f)
 
 // Pack one key group: G tokens x 128 channels -> codes (token-major words),
 // one (scale, zero) per channel.  Called by all 128 threads of a CTA
-// (thread c = channel c).  row(t) returns a pointer to token t's 128 fp16.
-template <class RowFn>
-__device__ __forceinline__ void pack_key_group(RowFn row, int G, uint32_t *codes /* [G][8] */,
+// (thread c = channel c).  at(t, c) points to channel c of token t (global or
+// shared memory; channels 4k..4k+3 must be contiguous).
+template <class AtFn>
+__device__ __forceinline__ void pack_key_group(AtFn at, int G, uint32_t *codes /* [G][8] */,
                                                uint16_t *scale_out /* [128] */, uint16_t *zero_out) {
     const int c = threadIdx.x;
     float mn = INFINITY, mx = -INFINITY;
     for (int t = 0; t < G; ++t) {
-        float x = h2f(row(t)[c]);
+        float x = h2f(*at(t, c));
         mn = fminf(mn, x);
         mx = fmaxf(mx, x);
     }
@@ -167,7 +168,7 @@ __device__ __forceinline__ void pack_key_group(RowFn row, int G, uint32_t *codes
     zero_out[c] = f2h(mn);
     const int lane = c & 31;
     for (int t = 0; t < G; ++t) {
-        uint32_t w = quant_code(h2f(row(t)[c]), mn, s) << (2 * (lane & 15));
+        uint32_t w = quant_code(h2f(*at(t, c)), mn, s) << (2 * (lane & 15));
         w |= __shfl_xor_sync(0xffffffffu, w, 1);
         w |= __shfl_xor_sync(0xffffffffu, w, 2);
         w |= __shfl_xor_sync(0xffffffffu, w, 4);
@@ -179,13 +180,13 @@ __device__ __forceinline__ void pack_key_group(RowFn row, int G, uint32_t *codes
 // Pack value tokens: each of n tokens is quantized per block of Gv channels.
 // Called by all 128 threads (4 warps, one token per warp at a time; lane l
 // owns channels 4l..4l+3).  Gv in {16, 32, 64, 128}.
-template <class RowFn>
-__device__ __forceinline__ void pack_value_tokens(RowFn row, int n, int Gv, uint32_t *codes /* [n][8] */,
+template <class AtFn>
+__device__ __forceinline__ void pack_value_tokens(AtFn at, int n, int Gv, uint32_t *codes /* [n][8] */,
                                                   uint16_t *scale_out /* [n][128/Gv] */, uint16_t *zero_out) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int lanes_per_block = Gv >> 2;
     for (int t = warp; t < n; t += 4) {
-        const uint16_t *p = row(t) + 4 * lane;
+        const uint16_t *p = at(t, 4 * lane);
         uint2 raw = *reinterpret_cast<const uint2 *>(p);
         float x[4] = {h2f(raw.x & 0xffff), h2f(raw.x >> 16), h2f(raw.y & 0xffff), h2f(raw.y >> 16)};
         float mn = fminf(fminf(x[0], x[1]), fminf(x[2], x[3]));

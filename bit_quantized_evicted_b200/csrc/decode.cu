@@ -91,6 +91,8 @@ struct Args {
     float *part;
     unsigned *counters;
     int *err;
+    unsigned *grid_counter;   // device-state mode: CTAs of this launch that have finished (self-resetting)
+    int *dseq;                // device-state mode: per-sequence state [B][4] in device memory
     float *xs;          // mass variant: absolute log2 scores [unit][g][xs_stride]
     float *stats;       // mass variant: per unit max[4], sum[4], token count (int bits), pad
     int xs_stride;
@@ -124,6 +126,7 @@ __device__ __forceinline__ int len_nq(const Args &a, int) { return a.n_q; }
 __device__ __forceinline__ int len_r(const Args &a, int) { return a.r; }
 __device__ __forceinline__ int len_rs(const Args &a, int) { return a.res_start; }
 __device__ __forceinline__ int len_spu(const Args &a, int) { return a.spu; }
+__device__ __forceinline__ int seq_spu(const Args &a, int) { return a.spu; }
 __device__ __forceinline__ int slice0(const Args &a, int unit) { return unit * a.spu; }
 __device__ __forceinline__ int unit_of(const Args &a, int x) { return x / a.spu; }
 
@@ -131,6 +134,7 @@ __device__ __forceinline__ int len_nq(const ArgsVar &a, int unit) { return a.tab
 __device__ __forceinline__ int len_r(const ArgsVar &a, int unit) { return a.tab.r[unit / a.Hkv]; }
 __device__ __forceinline__ int len_rs(const ArgsVar &a, int unit) { return a.tab.res_start[unit / a.Hkv]; }
 __device__ __forceinline__ int len_spu(const ArgsVar &a, int unit) { return a.tab.n_q[unit / a.Hkv] / kSlice; }
+__device__ __forceinline__ int seq_spu(const ArgsVar &a, int b) { return a.tab.n_q[b] / kSlice; }
 __device__ __forceinline__ int slice0(const ArgsVar &a, int unit) {
     const int b = unit / a.Hkv;
     return a.tab.sbeg[b] + (unit - b * a.Hkv) * (a.tab.n_q[b] / kSlice);
@@ -145,6 +149,49 @@ __device__ __forceinline__ int unit_of(const ArgsVar &a, int x) {
     }
     return lo * a.Hkv + (x - a.tab.sbeg[lo]) / (a.tab.n_q[lo] / kSlice);
 }
+
+// Device-state mode: the per-sequence state lives in device memory (dseq), so
+// one launch configuration serves every step and the calls can be captured in
+// a CUDA graph.  Each CTA copies the state into shared memory behind Smem
+// (DevTab) before it starts; the partition of the packed slices over the
+// packed CTAs is then computed from it, on the device.
+struct ArgsDev : Args {};
+struct DevTab {   // followed by n_q[B], r[B], res_start[B], sbeg[B + 1]
+    int Ns, P;    // packed slices this step, packed CTAs that take a share
+};
+__device__ __forceinline__ unsigned char *dyn_smem() {
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    return smem_raw;
+}
+__device__ __forceinline__ DevTab &dev_tab() { return *reinterpret_cast<DevTab *>(dyn_smem() + sizeof(Smem)); }
+__device__ __forceinline__ int *dev_arr(const ArgsDev &a, int k) {   // k = 0 n_q, 1 r, 2 res_start, 3 sbeg
+    return reinterpret_cast<int *>(dyn_smem() + sizeof(Smem) + sizeof(DevTab)) + k * (a.units / a.Hkv);
+}
+__device__ __forceinline__ int len_nq(const ArgsDev &a, int unit) { return dev_arr(a, 0)[unit / a.Hkv]; }
+__device__ __forceinline__ int len_r(const ArgsDev &a, int unit) { return dev_arr(a, 1)[unit / a.Hkv]; }
+__device__ __forceinline__ int len_rs(const ArgsDev &a, int unit) { return dev_arr(a, 2)[unit / a.Hkv]; }
+__device__ __forceinline__ int len_spu(const ArgsDev &a, int unit) { return dev_arr(a, 0)[unit / a.Hkv] / kSlice; }
+__device__ __forceinline__ int seq_spu(const ArgsDev &a, int b) { return dev_arr(a, 0)[b] / kSlice; }
+__device__ __forceinline__ int slice0(const ArgsDev &a, int unit) {
+    const int b = unit / a.Hkv;
+    return dev_arr(a, 3)[b] + (unit - b * a.Hkv) * (dev_arr(a, 0)[b] / kSlice);
+}
+__device__ __forceinline__ int unit_of(const ArgsDev &a, int x) {
+    const int *sbeg = dev_arr(a, 3);
+    int lo = 0, hi = a.units / a.Hkv;
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (sbeg[mid] <= x) lo = mid;
+        else hi = mid;
+    }
+    return lo * a.Hkv + (x - sbeg[lo]) / (dev_arr(a, 0)[lo] / kSlice);
+}
+
+// the partition of packed slices over packed CTAs (host-planned, or this step's on the device)
+__device__ __forceinline__ int part_Ns(const Args &a) { return a.Ns; }
+__device__ __forceinline__ int part_P(const Args &a) { return a.P; }
+__device__ __forceinline__ int part_Ns(const ArgsDev &) { return dev_tab().Ns; }
+__device__ __forceinline__ int part_P(const ArgsDev &) { return dev_tab().P; }
 
 // element offset of (row, col) in a [rows][128] fp16 tile; 16-byte chunks are
 // XOR-swizzled by row so ldmatrix reads of 8 rows hit distinct banks
@@ -306,8 +353,8 @@ __device__ __forceinline__ void unit_slots(const A &a, int unit, int &first, int
         return;
     }
     const int s0 = slice0(a, unit);
-    first = cta_of_slice(s0, a.P, a.Ns);
-    const int last = cta_of_slice((long long)s0 + spu - 1, a.P, a.Ns);
+    first = cta_of_slice(s0, part_P(a), part_Ns(a));
+    const int last = cta_of_slice((long long)s0 + spu - 1, part_P(a), part_Ns(a));
     S_u = a.n_rc + last - first + 1;
 }
 
@@ -330,8 +377,8 @@ __device__ void residual_chunk_cta(const A &a, Smem &sm, int unit, int rc) {
     const int i0 = rc * kResChunk;
     const int n = min(kResChunk, r - i0);
     auto slot = [&](int i) { int s = res_start + i; return s >= a.ring ? s - a.ring : s; };
-    auto krow = [&](int i) -> const uint16_t * { return i == r - 1 ? knew : kres + (size_t)slot(i) * kD; };
-    auto vrow = [&](int i) -> const uint16_t * { return i == r - 1 ? vnew : vres + (size_t)slot(i) * kD; };
+    auto krow = [&](int i, int c) -> const uint16_t * { return (i == r - 1 ? knew : kres + (size_t)slot(i) * kD) + c; };
+    auto vrow = [&](int i, int c) -> const uint16_t * { return (i == r - 1 ? vnew : vres + (size_t)slot(i) * kD) + c; };
 
     {
         const int ch = tid & 15;
@@ -444,12 +491,20 @@ __device__ void residual_chunk_cta(const A &a, Smem &sm, int unit, int rc) {
             sm.wl[warp][hA + 1] = l_w[1];
         }
     }
-    if (r == a.ring && rc == 0) {
+    if (r == a.ring && n_q + a.G <= a.cap && rc == 0) {
         // the oldest G residual tokens become key group n_q/G and G value tokens
         const size_t tok0 = (size_t)unit * a.cap + n_q;
         const size_t grow = (size_t)unit * (a.cap / a.G) + n_q / a.G;
-        pack_key_group(krow, a.G, a.k_codes_w + tok0 * 8, a.k_scale_w + grow * kD, a.k_zero_w + grow * kD);
-        pack_value_tokens(vrow, a.G, kD, a.v_codes_w + tok0 * 8, a.v_scale_w + tok0, a.v_zero_w + tok0);
+        if (a.G <= kResChunk) {   // the group is in this CTA's shared tile (logical rows 0..63)
+            __syncthreads();
+            auto kat = [&](int i, int c) -> const uint16_t * { return sm.res.k + swz(i, c); };
+            auto vat = [&](int i, int c) -> const uint16_t * { return sm.res.v + swz(i, c); };
+            pack_key_group(kat, a.G, a.k_codes_w + tok0 * 8, a.k_scale_w + grow * kD, a.k_zero_w + grow * kD);
+            pack_value_tokens(vat, a.G, kD, a.v_codes_w + tok0 * 8, a.v_scale_w + tok0, a.v_zero_w + tok0);
+        } else {
+            pack_key_group(krow, a.G, a.k_codes_w + tok0 * 8, a.k_scale_w + grow * kD, a.k_zero_w + grow * kD);
+            pack_value_tokens(vrow, a.G, kD, a.v_codes_w + tok0 * 8, a.v_scale_w + tok0, a.v_zero_w + tok0);
+        }
     }
     int first, S_u;
     unit_slots(a, unit, first, S_u);
@@ -476,17 +531,21 @@ __device__ __forceinline__ void issue_slice(const A &a, Smem &sm, int warp, int 
     bulk_g2s(S.vz, a.v_zero + tok, kSlice * 2, bar);
 }
 
-// A warp's position in the flat slice list, kept as (unit, slice in unit) so
-// that stepping needs no division.
+// A warp's position in the flat slice list, kept as (unit, its sequence b, its
+// KV head kh, slice in unit j) so that stepping needs no division.
 struct Cursor {
-    int u, j;
+    int u, b, kh, j;
     template <class A>
     __device__ __forceinline__ void step(const A &a, int n) {
         j += n;
-        int spu = len_spu(a, u);
+        int spu = seq_spu(a, b);
         while (j >= spu && u < a.units - 1) {
             j -= spu;
-            spu = len_spu(a, ++u);
+            ++u;
+            if (++kh == a.Hkv) {
+                kh = 0;
+                spu = seq_spu(a, ++b);
+            }
         }
     }
 };
@@ -507,7 +566,9 @@ __device__ void packed_cta(const A &a, Smem &sm, int c) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g_ = lane >> 2, t_ = lane & 3;
     const int Hq = a.Hkv * a.g;
-    const int cs = (int)((long long)c * a.Ns / a.P), ce = (int)((long long)(c + 1) * a.Ns / a.P);
+    const int Ns = part_Ns(a), P = part_P(a);
+    if (c >= P) return;   // no share this step (device-state mode plans for the largest step)
+    const int cs = (int)((long long)c * Ns / P), ce = (int)((long long)(c + 1) * Ns / P);
 
     if (tid == 0) {
         for (int w = 0; w < 4; ++w)
@@ -516,10 +577,12 @@ __device__ void packed_cta(const A &a, Smem &sm, int c) {
     }
     __syncthreads();
     // this warp's slices: cs + warp + 4k; `nxt` is the next one to queue
-    Cursor nxt{0, 0};
+    Cursor nxt{0, 0, 0, 0};
     int nxt_x = cs + warp;
     if (nxt_x < ce) {
         nxt.u = unit_of(a, nxt_x);
+        nxt.b = nxt.u / a.Hkv;
+        nxt.kh = nxt.u - nxt.b * a.Hkv;
         nxt.j = nxt_x - slice0(a, nxt.u);
     }
     if (lane == 0)
@@ -777,6 +840,71 @@ __global__ void __launch_bounds__(kThreads, 4) decode_kernel(const Args a) {
     decode_body<kMass>(a);
 }
 
+// Device-state mode: copy the state in, run the CTA's work, and let the last CTA
+// of the launch advance the state of every sequence (append; flush G tokens
+// where the ring is full).  A flush that would pass `cap` is not done: the
+// sequence keeps its state and its status word is set to 1.
+template <bool kMass>
+__global__ void __launch_bounds__(kThreads, 4) decode_dev_kernel(const ArgsDev a) {
+    const int tid = threadIdx.x;
+    const int B = a.units / a.Hkv;
+    int *nq = dev_arr(a, 0), *rr = dev_arr(a, 1), *rs = dev_arr(a, 2), *sbeg = dev_arr(a, 3);
+    for (int b = tid; b < B; b += kThreads) {
+        const int4 st = __ldcg(reinterpret_cast<const int4 *>(a.dseq) + b);
+        nq[b] = st.x;
+        rr[b] = st.y + 1;
+        rs[b] = st.z;
+    }
+    __syncthreads();
+    if (tid < 32) {   // sbeg = exclusive prefix of Hkv * slices, one warp, 32 sequences per pass
+        int carry = 0;
+        for (int b0 = 0; b0 < B; b0 += 32) {
+            const int b = b0 + tid;
+            const int v = b < B ? a.Hkv * (nq[b] / kSlice) : 0;
+            int x = v;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, x, o);
+                if (tid >= o) x += y;
+            }
+            if (b < B) sbeg[b] = carry + x - v;
+            carry += __shfl_sync(0xffffffffu, x, 31);
+        }
+        if (tid == 0) {
+            sbeg[B] = carry;
+            DevTab &t = dev_tab();
+            t.Ns = carry;
+            long long P = a.P;   // packed CTAs of the grid; at least 4 slices each
+            if (P > (carry + 3) / 4) P = (carry + 3) / 4;
+            t.P = (int)P;
+        }
+    }
+    __syncthreads();
+    decode_body<kMass>(a);
+    __syncthreads();
+    if (tid == 0) {
+        __threadfence();
+        const unsigned n = gridDim.x;
+        if (atomicInc(a.grid_counter, n - 1) == n - 1) {
+            __threadfence();
+            for (int b = 0; b < B; ++b) {
+                int4 st = make_int4(nq[b], rr[b], rs[b], __ldcg(a.dseq + 4 * b + 3));   // status stays set
+                if (rr[b] == a.ring) {
+                    if (nq[b] + a.G <= a.cap) {
+                        st.x += a.G;
+                        st.y -= a.G;
+                        st.z = (st.z + a.G) % a.ring;
+                    } else {
+                        st.y -= 1;   // state unchanged
+                        st.w = 1;
+                    }
+                }
+                reinterpret_cast<int4 *>(a.dseq)[b] = st;
+            }
+        }
+    }
+}
+
 // ragged batch: per-sequence lengths in the parameter table
 template <bool kMass>
 __global__ void __launch_bounds__(kThreads, 4) decode_ragged_kernel(const __grid_constant__ ArgsVar a) {
@@ -840,8 +968,13 @@ bool set_smem_attr(K kernel) {
 // the kernels' shared memory is above the 48 KB default: opt in once
 int ensure_attr() {
     if (!g_attr_done) {
+        const int dev_max = (int)(sizeof(Smem) + sizeof(DevTab) + (4 * kMaxRaggedSeqs + 1) * sizeof(int));
         if (!set_smem_attr(decode_kernel<false>) || !set_smem_attr(decode_kernel<true>) ||
-            !set_smem_attr(decode_ragged_kernel<false>) || !set_smem_attr(decode_ragged_kernel<true>))
+            !set_smem_attr(decode_ragged_kernel<false>) || !set_smem_attr(decode_ragged_kernel<true>) ||
+            cudaFuncSetAttribute(decode_dev_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, dev_max) !=
+                cudaSuccess ||
+            cudaFuncSetAttribute(decode_dev_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, dev_max) !=
+                cudaSuccess)
             return check_launch("decode_attn: cudaFuncSetAttribute");
         g_attr_done = true;
     }
@@ -873,9 +1006,52 @@ struct Plan {
     int max_n;   // most tokens any unit attends to this step
 };
 
+// shared memory of decode_dev_kernel for a batch of B sequences
+size_t dev_smem_bytes(int B) { return sizeof(Smem) + sizeof(DevTab) + (4 * (size_t)B + 1) * sizeof(int); }
+
+// resident decode_dev_kernel CTAs for this shared-memory size (looked up once
+// per size, so that calls under stream capture make no occupancy query)
+int dev_slots(size_t smem) {
+    static size_t last_smem = 0;
+    static int last_slots = 0;
+    if (smem == last_smem && last_slots > 0) return last_slots;
+    int dev = 0, sms = 148, per = 4;
+    if (ensure_attr() == MINIKV_OK && cudaGetDevice(&dev) == cudaSuccess) {
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, decode_dev_kernel<false>, kThreads, smem) !=
+                cudaSuccess || per < 1)
+            per = 1;
+    }
+    cudaGetLastError();
+    last_smem = smem;
+    last_slots = (sms > 0 ? sms : 148) * per;
+    return last_slots;
+}
+
 Plan plan(const minikv_cache *c) {
     Plan p;
     p.units = c->B * c->Hkv;
+    if (c->dseq) {
+        // device-state mode: one configuration for every state the cache can hold;
+        // the kernel partitions this step's slices itself
+        const int ring = c->R + c->G;
+        const int spu_cap = c->cap / kSlice;
+        p.n_rc = (ring + kResChunk - 1) / kResChunk;
+        p.spu = 0;
+        p.Ns = p.units * spu_cap;
+        p.P = 0;
+        if (p.Ns > 0) {
+            long long P = dev_slots(dev_smem_bytes(c->B));
+            if (P > (p.Ns + 3) / 4) P = (p.Ns + 3) / 4;
+            if (P > kMaxPackedCtas) P = kMaxPackedCtas;
+            p.P = (int)(P < 1 ? 1 : P);
+        }
+        int per_unit = p.Ns > 0 ? spu_cap / 3 + 2 : 0;
+        if (per_unit > p.P) per_unit = p.P;
+        p.S_max = p.n_rc + per_unit;
+        p.max_n = c->cap + ring;
+        return p;
+    }
     const int nb = c->seq ? c->B : 1;   // distinct sequence states
     int max_r = 0;
     long long Ns = 0;
@@ -922,8 +1098,9 @@ Plan plan(const minikv_cache *c) {
 
 }  // namespace
 
-// Bytes of the workspace prefix that holds the per-unit arrival counters.
-size_t decode_counter_bytes(int B, int Hkv) { return (((size_t)B * Hkv * 4 + 255) / 256) * 256; }
+// Bytes of the workspace prefix that holds the per-unit arrival counters and
+// the launch-wide counter of the device-state mode.
+size_t decode_counter_bytes(int B, int Hkv) { return (((size_t)B * Hkv * 4 + 4 + 255) / 256) * 256; }
 
 size_t decode_workspace_bytes(int B, int Hkv, int max_tokens) {
     const size_t units = (size_t)B * Hkv;
@@ -974,6 +1151,15 @@ int launch_decode<ArgsVar>(const ArgsVar &a, const Plan &p, bool with_mass, cuda
     return check_launch(with_mass ? "decode_attn_mass (ragged)" : "decode_attn (ragged)");
 }
 
+template <>
+int launch_decode<ArgsDev>(const ArgsDev &a, const Plan &p, bool with_mass, cudaStream_t stream) {
+    const int grid = p.units * p.n_rc + p.P;
+    const size_t smem = dev_smem_bytes(a.units / a.Hkv);
+    if (with_mass) decode_dev_kernel<true><<<grid, kThreads, smem, stream>>>(a);
+    else decode_dev_kernel<false><<<grid, kThreads, smem, stream>>>(a);
+    return check_launch(with_mass ? "decode_attn_mass (device state)" : "decode_attn (device state)");
+}
+
 int launch_mass(const Args &a, const Plan &p, float *mass, long long mass_stride, cudaStream_t stream) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((p.max_n + 1023) / 1024, p.units);
@@ -1003,7 +1189,7 @@ int decode_launch(minikv_cache *c, const uint16_t *q, const uint16_t *k_new, con
                   float sm_scale, uint16_t *out, void *ws, size_t ws_bytes, cudaStream_t stream, float *mass) {
     const int g = Hq / c->Hkv;
     const int ring = c->R + c->G;
-    const int nb = c->seq ? c->B : 1;
+    const int nb = c->dseq ? 0 : (c->seq ? c->B : 1);   // device state: checked on the device
     for (int b = 0; b < nb; ++b)
         if (seq_nres(c, b) + 1 == ring && seq_nq(c, b) + c->G > c->cap)
             return fail(MINIKV_ERR_CAPACITY, "decode_attn: flushing a key group of sequence %d would exceed cap=%d",
@@ -1026,6 +1212,8 @@ int decode_launch(minikv_cache *c, const uint16_t *q, const uint16_t *k_new, con
     a.k_res = c->k_res; a.v_res = c->v_res;
     a.q = q; a.k_new = k_new; a.v_new = v_new; a.out = out;
     a.counters = reinterpret_cast<unsigned *>(ws);
+    a.grid_counter = a.counters + p.units;
+    a.dseq = c->dseq;
     a.part = reinterpret_cast<float *>(static_cast<char *>(ws) + cnt_bytes);
     a.err = nullptr;
     a.stats = mass ? reinterpret_cast<float *>(static_cast<char *>(ws) + cnt_bytes + part_bytes) : nullptr;
@@ -1041,7 +1229,13 @@ int decode_launch(minikv_cache *c, const uint16_t *q, const uint16_t *k_new, con
     a.scale_log2 = sm_scale * kLog2e;
 
     int rc;
-    if (c->seq) {
+    if (c->dseq) {
+        ArgsDev ad;
+        static_cast<Args &>(ad) = a;
+        rc = launch_decode(ad, p, mass != nullptr, stream);
+        if (rc) return rc;
+        return mass ? launch_mass(a, p, mass, (long long)c->cap + ring, stream) : MINIKV_OK;
+    } else if (c->seq) {
         ArgsVar av;
         static_cast<Args &>(av) = a;
         av.tab.sbeg[0] = 0;

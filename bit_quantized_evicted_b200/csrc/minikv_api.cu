@@ -65,7 +65,10 @@ static int check_cache(const minikv_cache *c) {
         return n_packed < 0 || n_packed % c->G || n_packed > c->cap || n_res < 0 || n_res >= c->R + c->G ||
                res_start < 0 || res_start >= c->R + c->G;
     };
-    if (c->seq) {
+    if (c->dseq) {
+        if (c->B > MINIKV_MAX_RAGGED_SEQS)
+            return fail(MINIKV_ERR_UNSUPPORTED, "device-state cache with B=%d above %d", c->B, MINIKV_MAX_RAGGED_SEQS);
+    } else if (c->seq) {
         if (c->B > MINIKV_MAX_RAGGED_SEQS)
             return fail(MINIKV_ERR_UNSUPPORTED, "ragged cache with B=%d above %d", c->B, MINIKV_MAX_RAGGED_SEQS);
         for (int b = 0; b < c->B; ++b)
@@ -95,7 +98,7 @@ int decode_validate(minikv_cache *c, const uint16_t *q, const uint16_t *k_new, c
     if ((size_t)c->B * c->Hkv > 65535) return fail(MINIKV_ERR_UNSUPPORTED, "decode_attn: B*Hkv above 65535");
     if ((size_t)c->B * c->Hkv * (c->cap / 32) >= (1u << 31))
         return fail(MINIKV_ERR_UNSUPPORTED, "decode_attn: B*Hkv*cap/32 must stay below 2^31");
-    const int nb = c->seq ? c->B : 1;
+    const int nb = c->dseq ? 0 : (c->seq ? c->B : 1);   // a device-resident state is checked on the device
     for (int b = 0; b < nb; ++b) {
         const int n_packed = c->seq ? c->seq[3 * b] : c->n_packed, n_res = c->seq ? c->seq[3 * b + 1] : c->n_res;
         if (n_res + 1 == c->R + c->G && n_packed + c->G > c->cap)
@@ -147,6 +150,25 @@ int minikv_cache_bind(minikv_cache *c, void *base, size_t bytes, int B, int Hkv,
     c->v_res = reinterpret_cast<uint16_t *>(take(u * (R + G) * D * 2));
     c->n_packed = 0; c->n_res = 0; c->res_start = 0;
     c->seq = nullptr;
+    c->dseq = nullptr;
+    return MINIKV_OK;
+}
+
+int minikv_cache_set_device_state(minikv_cache *c, int *dseq, void *stream) {
+    g_err[0] = 0;
+    if (!c) return fail(MINIKV_ERR_INVALID_ARG, "cache_set_device_state: null cache");
+    if (dseq) {
+        if (c->B < 1 || c->B > MINIKV_MAX_RAGGED_SEQS)
+            return fail(MINIKV_ERR_UNSUPPORTED, "cache_set_device_state: B=%d (1..%d)", c->B, MINIKV_MAX_RAGGED_SEQS);
+        if (!aligned16(dseq)) return fail(MINIKV_ERR_INVALID_ARG, "cache_set_device_state: dseq not 16-byte aligned");
+        cudaError_t e = cudaMemsetAsync(dseq, 0, (size_t)c->B * 4 * sizeof(int), static_cast<cudaStream_t>(stream));
+        if (e != cudaSuccess)
+            return fail(MINIKV_ERR_CUDA, "cache_set_device_state: clearing the state: %s", cudaGetErrorString(e));
+    }
+    c->dseq = dseq;
+    c->n_packed = 0; c->n_res = 0; c->res_start = 0;
+    if (c->seq)
+        for (int i = 0; i < 3 * c->B; ++i) c->seq[i] = 0;
     return MINIKV_OK;
 }
 
@@ -177,7 +199,7 @@ int minikv_quant_pack_seq(minikv_cache *c, int b, const uint16_t *k, const uint1
     g_err[0] = 0;
     int rc = check_cache(c);
     if (rc) return rc;
-    if (!c->seq) return fail(MINIKV_ERR_INVALID_ARG, "quant_pack_seq: the cache is not ragged");
+    if (!c->seq && !c->dseq) return fail(MINIKV_ERR_INVALID_ARG, "quant_pack_seq: the cache is not ragged");
     if (b < 0 || b >= c->B) return fail(MINIKV_ERR_INVALID_ARG, "quant_pack_seq: sequence %d of %d", b, c->B);
     if (n_tokens < 0) return fail(MINIKV_ERR_INVALID_ARG, "quant_pack_seq: n_tokens=%d", n_tokens);
     if (n_tokens > 0 && (!k || !v || !aligned16(k) || !aligned16(v)))
@@ -241,7 +263,7 @@ static int evict_pack_impl(const float *scores, const uint16_t *k, const uint16_
         return fail(MINIKV_ERR_INVALID_ARG, "evict_pack: B=%d Hkv=%d T=%d W=%d keep=%d", B, Hkv, T, W, keep);
     if (D != kD) return fail(MINIKV_ERR_UNSUPPORTED, "evict_pack: D=%d (only 128)", D);
     if (seq >= 0) {
-        if (!c->seq) return fail(MINIKV_ERR_INVALID_ARG, "evict_pack_seq: the cache is not ragged");
+        if (!c->seq && !c->dseq) return fail(MINIKV_ERR_INVALID_ARG, "evict_pack_seq: the cache is not ragged");
         if (seq >= c->B) return fail(MINIKV_ERR_INVALID_ARG, "evict_pack_seq: sequence %d of %d", seq, c->B);
         if (Hkv != c->Hkv)
             return fail(MINIKV_ERR_INVALID_ARG, "evict_pack_seq: Hkv=%d but the cache has Hkv=%d", Hkv, c->Hkv);

@@ -28,6 +28,8 @@ struct PackArgs {
     uint16_t *k_res, *v_res;
     int N, n_q, r, G, Gv, cap, ring, n_groups;
     int unit0;   // cache unit of grid row 0 (b * Hkv when one sequence of a ragged batch is loaded)
+    int *dseq;   // device-state mode: [B][4] state words to set (rows seq0 .. seq0 + n_seq - 1), else null
+    int seq0, n_seq;
 };
 
 constexpr int kResPerBlock = 32;   // residual tokens copied per block
@@ -40,11 +42,14 @@ __global__ void __launch_bounds__(128) pack_kernel(const PackArgs a) {
     const uint16_t *vu = a.v + (size_t)src_unit * rows * kD;
     const int32_t *iu = a.idx ? a.idx + (size_t)src_unit * a.N : nullptr;
     auto src_row = [&](int t) -> size_t { return iu ? (size_t)iu[t] : (size_t)t; };   // compacted -> source row
+    if (a.dseq && blockIdx.x == 0 && blockIdx.y == 0)
+        for (int b = threadIdx.x; b < a.n_seq; b += 128)
+            reinterpret_cast<int4 *>(a.dseq)[a.seq0 + b] = make_int4(a.n_q, a.r, 0, 0);
     if ((int)blockIdx.x < a.n_groups) {
         const int grp = blockIdx.x;
         const int t0 = grp * a.G;
-        auto krow = [&](int t) { return ku + src_row(t0 + t) * kD; };
-        auto vrow = [&](int t) { return vu + src_row(t0 + t) * kD; };
+        auto krow = [&](int t, int c) { return ku + src_row(t0 + t) * kD + c; };
+        auto vrow = [&](int t, int c) { return vu + src_row(t0 + t) * kD + c; };
         const size_t tok = (size_t)unit * a.cap + t0;
         const size_t grow = (size_t)unit * (a.cap / a.G) + grp;
         pack_key_group(krow, a.G, a.k_codes + tok * 8, a.k_scale + grow * kD, a.k_zero + grow * kD);
@@ -69,6 +74,7 @@ __global__ void __launch_bounds__(128) pack_kernel(const PackArgs a) {
 // idx == nullptr: k, v are [B,Hkv,N,D]; else k, v are [B,Hkv,T,D] and row t of
 // unit u is idx[u][t] (idx [B,Hkv,N], ascending positions < T).  seq >= 0 loads
 // sequence `seq` of a ragged cache only (k, v, idx then without the B axis).
+// With a device-state cache, block (0, 0) also writes the loaded rows' state.
 int pack_launch(minikv_cache *c, const uint16_t *k, const uint16_t *v, int N, cudaStream_t stream,
                 const int32_t *idx, int T, int seq) {
     int n_q, r;
@@ -90,8 +96,12 @@ int pack_launch(minikv_cache *c, const uint16_t *k, const uint16_t *v, int N, cu
     a.N = N; a.n_q = n_q; a.r = r; a.G = c->G; a.Gv = c->Gv; a.cap = c->cap; a.ring = c->R + c->G;
     a.n_groups = n_q / c->G;
     a.unit0 = seq >= 0 ? seq * c->Hkv : 0;
+    a.dseq = c->dseq;
+    a.seq0 = seq >= 0 ? seq : 0;
+    a.n_seq = seq >= 0 ? 1 : c->B;
     const int n_res_blocks = (r + kResPerBlock - 1) / kResPerBlock;
-    const int gx = a.n_groups + n_res_blocks;
+    int gx = a.n_groups + n_res_blocks;
+    if (c->dseq && gx == 0) gx = 1;   // an empty load still sets the device state
     const int units = seq >= 0 ? c->Hkv : c->B * c->Hkv;
     if (gx > 0 && units > 0) {
         pack_kernel<<<dim3(gx, units), 128, 0, stream>>>(a);
@@ -99,9 +109,11 @@ int pack_launch(minikv_cache *c, const uint16_t *k, const uint16_t *v, int N, cu
         if (rc) return rc;
     }
     if (seq >= 0) {
-        c->seq[3 * seq] = n_q;
-        c->seq[3 * seq + 1] = r;
-        c->seq[3 * seq + 2] = 0;
+        if (c->seq) {
+            c->seq[3 * seq] = n_q;
+            c->seq[3 * seq + 1] = r;
+            c->seq[3 * seq + 2] = 0;
+        }
         return MINIKV_OK;
     }
     c->n_packed = n_q;

@@ -33,7 +33,7 @@ class CacheStruct(ctypes.Structure):
     _fields_ = [("B", _I), ("Hkv", _I), ("D", _I), ("G", _I), ("Gv", _I), ("R", _I), ("cap", _I),
                 ("k_codes", _P), ("v_codes", _P), ("k_scale", _P), ("k_zero", _P),
                 ("v_scale", _P), ("v_zero", _P), ("k_res", _P), ("v_res", _P),
-                ("n_packed", _I), ("n_res", _I), ("res_start", _I), ("seq", _P)]
+                ("n_packed", _I), ("n_res", _I), ("res_start", _I), ("seq", _P), ("dseq", _P)]
 
 MAX_RAGGED_SEQS = 256
 
@@ -42,6 +42,7 @@ _SIGS = {
     "minikv_cache_bytes": (_Z, [_I, _I, _I, _I, _I, _I, _I]),
     "minikv_cache_bind": (_I, [ctypes.POINTER(CacheStruct), _P, _Z, _I, _I, _I, _I, _I, _I, _I]),
     "minikv_cache_set_ragged": (_I, [ctypes.POINTER(CacheStruct), _P]),
+    "minikv_cache_set_device_state": (_I, [ctypes.POINTER(CacheStruct), _P, _P]),
     "minikv_quant_pack": (_I, [ctypes.POINTER(CacheStruct), _P, _P, _I, _P]),
     "minikv_quant_pack_seq": (_I, [ctypes.POINTER(CacheStruct), _I, _P, _P, _I, _P]),
     "minikv_evict_pack_seq": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, ctypes.POINTER(CacheStruct), _I, _P]),
@@ -123,6 +124,7 @@ class MiniKVCache:
                              dtype=torch.uint8, device=device)
         self.ws = ws
         self._seq = None
+        self.dseq = None
 
     def set_ragged(self) -> "MiniKVCache":
         """Give every sequence its own length (per-sequence host state, all empty)."""
@@ -130,15 +132,31 @@ class MiniKVCache:
         _check(lib().minikv_cache_set_ragged(ctypes.byref(self.c), ctypes.cast(self._seq, _P)))
         return self
 
+    def set_device_state(self, stream=None) -> "MiniKVCache":
+        """Keep the per-sequence state in device memory (dseq [B, 4] int32:
+        n_packed, n_res, res_start, status): decode steps then queue the same
+        launches every step and can be captured in a CUDA graph."""
+        self.dseq = torch.zeros((self.B, 4), dtype=torch.int32, device=self.device)
+        _check(lib().minikv_cache_set_device_state(ctypes.byref(self.c), self.dseq.data_ptr(),
+                                                   _stream(stream, self.device)))
+        return self
+
     @property
     def ragged(self) -> bool:
-        return self._seq is not None
+        return self._seq is not None or self.dseq is not None
 
     def seq_state(self, b: int) -> tuple[int, int, int]:
-        """(n_packed, n_res, res_start) of sequence b (either kind of batch)."""
+        """(n_packed, n_res, res_start) of sequence b (any kind of batch; a
+        device-resident state is read back, which synchronizes)."""
+        if self.dseq is not None:
+            return tuple(int(x) for x in self.dseq[b, :3].cpu())
         if self._seq is None:
             return self.n_packed, self.n_res, self.res_start
         return self._seq[3 * b], self._seq[3 * b + 1], self._seq[3 * b + 2]
+
+    def status(self) -> list[int]:
+        """Device-state mode: per-sequence status words (1 = a flush was refused at cap)."""
+        return [int(x) for x in self.dseq[:, 3].cpu()] if self.dseq is not None else [0] * self.B
 
     # shape / state
     B = property(lambda s: s.c.B)
@@ -194,10 +212,11 @@ class MiniKVCache:
 
         def unit(nq, r):
             return nq * (D // 4) * 2 + (nq // G) * D * 4 + nq * (D // Gv) * 4, r * D * 4
-        if self._seq is None:
+        if not self.ragged:
             packed, res = unit(self.n_packed, self.n_res + 1)
             return dict(packed=packed, residual=res, per_unit=packed + res, total=(packed + res) * self.B * self.Hkv)
-        tot = sum(sum(unit(self._seq[3 * b], self._seq[3 * b + 1] + 1)) for b in range(self.B)) * self.Hkv
+        st = [self.seq_state(b) for b in range(self.B)]
+        tot = sum(sum(unit(nq, nr + 1)) for nq, nr, _ in st) * self.Hkv
         return dict(total=tot)
 
 

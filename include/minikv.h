@@ -74,6 +74,11 @@ extern "C" {
  *     caller and kept alive while the cache is used; the three scalars are then
  *     not read.  Sequences of one batch may hold different numbers of packed
  *     and residual tokens (unequal prompts, unequal budgets).
+ *   - Device-resident state (dseq != NULL, see minikv_cache_set_device_state):
+ *     the per-sequence state lives in a DEVICE array [B][4] = (n_packed,
+ *     n_res, res_start, status); kernels read and advance it, the host fields
+ *     are not read, and a decode step queues the same launches whatever the
+ *     lengths, so a caller can capture steps in a CUDA graph and replay them.
  * Dequantized value of a code c: c * scale + zero.
  */
 typedef struct minikv_cache {
@@ -84,6 +89,7 @@ typedef struct minikv_cache {
     uint16_t *k_res, *v_res;
     int n_packed, n_res, res_start;
     int *seq;
+    int *dseq;
 } minikv_cache;
 
 /* Most sequences a ragged batch may hold. */
@@ -115,6 +121,29 @@ MINIKV_API int minikv_cache_bind(minikv_cache *c, void *base, size_t bytes,
 MINIKV_API int minikv_cache_set_ragged(minikv_cache *c, int *seq);
 
 /*
+ * minikv_cache_set_device_state -- keep the per-sequence state on the GPU.
+ * Source: none on the pages; decode steps whose launches do not depend on the
+ * host's view of the lengths can be captured once in a CUDA graph and
+ * replayed every step, which removes the per-call host cost.
+ *   dseq: DEVICE array of 4*B int32, 16-byte aligned, caller-owned, alive while
+ *   the cache is used: (n_packed, n_res, res_start, status) per sequence.  It
+ *   is zero-filled on `stream` (every sequence empty).  dseq = NULL returns to
+ *   host-side state (also empty).
+ * In this mode the loaders (minikv_quant_pack, minikv_evict_pack and their
+ * _seq forms) write the loaded rows' state into dseq from their kernel, and
+ * each decode call (minikv_decode_attn, _mass, _static) runs one launch
+ * configuration fixed by the cache's shape: the kernel reads the state,
+ * splits this step's packed tokens over its CTAs, and its last CTA advances
+ * every sequence's state.  A step whose flush would pass `cap` leaves that
+ * sequence's state unchanged (its new token is not kept) and sets its status
+ * word to 1; the host learns it by reading dseq.  Capacity is therefore not
+ * checked on the host in this mode.
+ * Errors: INVALID_ARG (null cache, misaligned dseq), UNSUPPORTED
+ * (B > MINIKV_MAX_RAGGED_SEQS), CUDA (the fill could not be queued).
+ */
+MINIKV_API int minikv_cache_set_device_state(minikv_cache *c, int *dseq, void *stream);
+
+/*
  * minikv_quant_pack -- load a fresh compacted sequence into the cache.
  * Source: summary page, 方法论 (sub-channel key quantization, per-token value
  * quantization, compact layout); the fp16 residual of the newest tokens.
@@ -139,8 +168,8 @@ MINIKV_API int minikv_quant_pack(minikv_cache *c, const uint16_t *k, const uint1
  * only: k, v [Hkv, n_tokens, D] fp16 become sequence b's kept tokens (same
  * split and quantizer); seq[b] = (n_tokens - r, r, 0).  Other sequences are
  * untouched.
- * Errors: as minikv_quant_pack; INVALID_ARG also if the cache is not ragged or
- * b is outside [0, B).
+ * Errors: as minikv_quant_pack; INVALID_ARG also if the cache is neither
+ * ragged nor device-state, or b is outside [0, B).
  */
 MINIKV_API int minikv_quant_pack_seq(minikv_cache *c, int b, const uint16_t *k, const uint16_t *v,
                                      int n_tokens, void *stream);
@@ -213,8 +242,8 @@ MINIKV_API int minikv_evict_pack(const float *scores, const uint16_t *k, const u
  * minikv_evict_pack_seq -- minikv_evict_pack of ONE prompt (scores [Hkv, T],
  * k, v [Hkv, T, D], idx [Hkv, min(keep, T)]) into sequence b of a ragged
  * cache; T and keep are this prompt's own.  Other sequences are untouched.
- * Errors: as minikv_evict_pack; INVALID_ARG also if the cache is not ragged or
- * b is outside [0, B).
+ * Errors: as minikv_evict_pack; INVALID_ARG also if the cache is neither
+ * ragged nor device-state, or b is outside [0, B).
  */
 MINIKV_API int minikv_evict_pack_seq(const float *scores, const uint16_t *k, const uint16_t *v,
                                      int Hkv, int T, int D, int W, int keep, int32_t *idx,

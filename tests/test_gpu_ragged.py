@@ -38,11 +38,14 @@ def _seq_kv(Hkv, N, seed):
     return k, v
 
 
-def _load(lengths, Hq, Hkv, G, R, steps, seed):
-    """A ragged cache loaded sequence by sequence, and the oracle's slices."""
+def _load(lengths, Hq, Hkv, G, R, steps, seed, device_state=False, cap=None):
+    """A ragged cache (host-side or device-resident per-sequence state) loaded
+    sequence by sequence, and the oracle's slices."""
     B = len(lengths)
-    cap = ((max(lengths) + steps) // G + 2) * G
-    cache = mk.MiniKVCache(B, Hkv, cap, G=G, Gv=128, R=R, Hq=Hq).set_ragged()
+    if cap is None:
+        cap = ((max(lengths) + steps) // G + 2) * G
+    cache = mk.MiniKVCache(B, Hkv, cap, G=G, Gv=128, R=R, Hq=Hq)
+    cache.set_device_state() if device_state else cache.set_ragged()
     ref = []
     for b, N in enumerate(lengths):
         k, v = _seq_kv(Hkv, N, seed + b)
@@ -77,15 +80,16 @@ def _compare_seq(cache, b, slices):
         np.testing.assert_array_equal(vr[h].view(np.uint16), np.array(s.res_v, np.uint16).reshape(s.r, 128))
 
 
+@pytest.mark.parametrize("device_state", [False, True])
 @pytest.mark.parametrize("lengths,Hq,Hkv,G,R,steps", [
     ((300, 20, 1000, 0, 161), 8, 2, 32, 32, 40),        # g = 4; an empty and an all-residual sequence
     ((700, 64, 2100), 4, 4, 64, 64, 70),                # g = 1, G = 64, flushes at different steps
     ((96, 33, 129, 500, 1, 64), 3, 1, 32, 0, 35),       # g = 3, R = 0
 ])
-def test_ragged_decode_vs_oracle(lengths, Hq, Hkv, G, R, steps):
+def test_ragged_decode_vs_oracle(lengths, Hq, Hkv, G, R, steps, device_state):
     B = len(lengths)
     g = Hq // Hkv
-    cache, ref = _load(lengths, Hq, Hkv, G, R, steps, 700)
+    cache, ref = _load(lengths, Hq, Hkv, G, R, steps, 700, device_state)
     for b in range(B):
         _compare_seq(cache, b, ref[b])
     worst = 0.0
@@ -187,3 +191,83 @@ def test_evict_pack_seq_prompts_of_different_lengths():
     # loading one row leaves the others as they were
     for b in range(len(prompts)):
         assert cache.seq_state(b)[0] + cache.seq_state(b)[1] == min(prompts[b][0], prompts[b][1])
+
+
+# ------------------------------------------------- device state + CUDA graphs
+
+@pytest.mark.parametrize("with_mass", [False, True])
+def test_device_state_steps_replayed_from_one_cuda_graph(with_mass):
+    """With the state on the device, one captured decode step replays correctly
+    for every later step: lengths grow, flushes happen, sequences differ."""
+    lengths, Hq, Hkv, G, R, steps = (300, 20, 1000, 0, 161), 8, 2, 32, 32, 40
+    B, g = len(lengths), Hq // Hkv
+    cache, ref = _load(lengths, Hq, Hkv, G, R, steps + 1, 900, device_state=True)
+    L = cache.cap + R + G
+    mass = torch.zeros((B, Hkv, L), dtype=torch.float32, device=DEV)
+    acc = np.zeros((B, Hkv, L))
+    q_s = torch.zeros((B, Hq, 128), dtype=torch.float16, device=DEV)
+    kn_s = torch.zeros((B, Hkv, 128), dtype=torch.float16, device=DEV)
+    vn_s = torch.zeros_like(kn_s)
+    out_s = torch.zeros_like(q_s)
+
+    def call():
+        if with_mass:
+            mk.decode_attn_mass(cache, q_s, kn_s, vn_s, mass, out=out_s)
+        else:
+            mk.decode_attn(cache, q_s, kn_s, vn_s, out=out_s)
+
+    graph = None
+    for s in range(steps):
+        q, kn, vn = _step_inputs(B, Hq, Hkv, 91, s)
+        q_s.copy_(q)
+        kn_s.copy_(kn)
+        vn_s.copy_(vn)
+        if s == 0:
+            call()                       # eager first step (also sets up the library)
+            torch.cuda.synchronize()
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                call()                   # captured, not run
+        else:
+            graph.replay()
+        torch.cuda.synchronize()
+        qn, knn, vnn = np16(q), np16(kn), np16(vn)
+        got = out_s.float().cpu().numpy()
+        for b in range(B):
+            for h in range(Hkv):
+                sl = ref[b][h]
+                args = (qn[b, h * g:(h + 1) * g], knn[b, h], vnn[b, h], TAU)
+                o = sl.step_mass(*args, acc[b, h]) if with_mass else sl.step(*args)
+                assert float(np.max(np.abs(got[b, h * g:(h + 1) * g] - o))) <= ATOL_OUT, (s, b, h)
+        if with_mass:
+            err = float(np.max(np.abs(mass.double().cpu().numpy() - acc)))
+            assert err <= ATOL_MASS_PER_STEP * (s + 1) + 1e-6, (s, err)
+    for b in range(B):
+        _compare_seq(cache, b, ref[b])
+    assert cache.status() == [0] * B
+    del graph
+
+
+def test_device_state_refuses_a_flush_past_capacity():
+    """cap leaves no room for another key group: the step that would flush
+    still attends correctly, then keeps the sequence's state and sets its
+    status word; the other sequence, with room, flushes normally."""
+    G, R, Hq, Hkv = 32, 32, 2, 2
+    lengths = (64 + 62, 62)          # r = 62 each: the second step fills the ring
+    cache, ref = _load(lengths, Hq, Hkv, G, R, 0, 950, device_state=True, cap=64)
+    assert [cache.seq_state(b) for b in range(2)] == [(64, 62, 0), (0, 62, 0)]
+    for s in range(2):
+        q, kn, vn = _step_inputs(2, Hq, Hkv, 96, s)
+        out = mk.decode_attn(cache, q, kn, vn)
+        torch.cuda.synchronize()
+        qn, knn, vnn = np16(q), np16(kn), np16(vn)
+        for b in range(2):
+            for h in range(Hkv):
+                o = ref[b][h].step(qn[b, h:h + 1], knn[b, h], vnn[b, h], TAU)
+                assert float(np.max(np.abs(out.float().cpu().numpy()[b, h:h + 1] - o))) <= ATOL_OUT, (s, b, h)
+    assert cache.seq_state(0) == (64, 63, 0) and cache.status()[0] == 1     # refused, unchanged
+    assert cache.seq_state(1) == (32, 32, 32) and cache.status()[1] == 0    # flushed
+    _compare_seq(cache, 1, ref[1])
+    a = cache.arrays()
+    for h in range(Hkv):                                                    # the full sequence's packed part intact
+        np.testing.assert_array_equal(a["k_codes"][0, h, :64].cpu().numpy().view(np.uint32), ref[0][h].k_codes[:64])
