@@ -146,71 +146,137 @@ __device__ __forceinline__ uint32_t quant_code(float x, float zero, float scale)
 // -0 and +0 are the same extreme; store +0.
 __device__ __forceinline__ float canon_zero(float x) { return __fadd_rn(x, 0.0f); }
 
+// element offset of (row, col) in a [rows][128] fp16 tile; 16-byte chunks are
+// XOR-swizzled by row so ldmatrix reads of 8 rows, and column reads of one
+// row by a warp, hit distinct banks
+__device__ __forceinline__ int swz(int row, int col) {
+    return row * kD + ((((col >> 3) ^ (row & 7))) << 3) + (col & 7);
+}
+
+// fp16 bits -> float, 8 at a time (one 16-byte chunk)
+__device__ __forceinline__ void h8_to_f(uint4 v, float *x) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        x[2 * i] = h2f((uint16_t)(w[i] & 0xffffu));
+        x[2 * i + 1] = h2f((uint16_t)(w[i] >> 16));
+    }
+}
+
 // Pack one key group: G tokens x 128 channels -> codes (token-major words),
-// one (scale, zero) per channel.  Called by all 128 threads of a CTA
-// (thread c = channel c).  at(t, c) points to channel c of token t (global or
-// shared memory; channels 4k..4k+3 must be contiguous).
+// one (scale, zero) per channel.  Called by all 128 threads of a CTA.
+// at(t, c) points to channel c of token t (global or shared memory); the 8
+// channels of each aligned 8-channel chunk are contiguous and 16-byte aligned.
+// scr: 256 floats of shared scratch.
+//   1. thread c: min / max of channel c over the G tokens -> (zero, scale);
+//   2. thread i: code words i, i + 128, ... (token w / 8, channels 16 (w % 8)
+//      .. +15), each from two 16-byte loads and 16 independent quantizations.
 template <class AtFn>
 __device__ __forceinline__ void pack_key_group(AtFn at, int G, uint32_t *codes /* [G][8] */,
-                                               uint16_t *scale_out /* [128] */, uint16_t *zero_out) {
+                                               uint16_t *scale_out /* [128] */, uint16_t *zero_out,
+                                               float *scr /* [256] shared */) {
     const int c = threadIdx.x;
     float mn = INFINITY, mx = -INFINITY;
+#pragma unroll 8
     for (int t = 0; t < G; ++t) {
-        float x = h2f(*at(t, c));
+        const float x = h2f(*at(t, c));
         mn = fminf(mn, x);
         mx = fmaxf(mx, x);
     }
     mn = canon_zero(mn);
     mx = canon_zero(mx);
-    uint16_t sb = quant_scale(mn, mx);
-    float s = h2f(sb);
+    const uint16_t sb = quant_scale(mn, mx);
     scale_out[c] = sb;
     zero_out[c] = f2h(mn);
-    const int lane = c & 31;
-    for (int t = 0; t < G; ++t) {
-        uint32_t w = quant_code(h2f(*at(t, c)), mn, s) << (2 * (lane & 15));
-        w |= __shfl_xor_sync(0xffffffffu, w, 1);
-        w |= __shfl_xor_sync(0xffffffffu, w, 2);
-        w |= __shfl_xor_sync(0xffffffffu, w, 4);
-        w |= __shfl_xor_sync(0xffffffffu, w, 8);
-        if ((lane & 15) == 0) codes[t * 8 + (c >> 4)] = w;
+    scr[c] = mn;
+    scr[128 + c] = h2f(sb);
+    __syncthreads();
+    for (int wi = c; wi < G * 8; wi += 128) {
+        const int t = wi >> 3, c0 = 16 * (wi & 7);
+        float x[16];
+        h8_to_f(*reinterpret_cast<const uint4 *>(at(t, c0)), x);
+        h8_to_f(*reinterpret_cast<const uint4 *>(at(t, c0 + 8)), x + 8);
+        uint32_t w = 0;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) w |= quant_code(x[i], scr[c0 + i], scr[128 + c0 + i]) << (2 * i);
+        codes[wi] = w;
     }
+    __syncthreads();   // scr is free again
 }
 
 // Pack value tokens: each of n tokens is quantized per block of Gv channels.
-// Called by all 128 threads (4 warps, one token per warp at a time; lane l
-// owns channels 4l..4l+3).  Gv in {16, 32, 64, 128}.
+// Called by all 128 threads: thread 4j + k of a pass takes token (pass * 32 + j)
+// and its channels 32k .. 32k+31 (two code words); min / max of a block wider
+// than 32 channels are combined over the Gv/32 threads that share it.
+// Gv in {16, 32, 64, 128}.  at() as for pack_key_group.
 template <class AtFn>
 __device__ __forceinline__ void pack_value_tokens(AtFn at, int n, int Gv, uint32_t *codes /* [n][8] */,
                                                   uint16_t *scale_out /* [n][128/Gv] */, uint16_t *zero_out) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int lanes_per_block = Gv >> 2;
-    for (int t = warp; t < n; t += 4) {
-        const uint16_t *p = at(t, 4 * lane);
-        uint2 raw = *reinterpret_cast<const uint2 *>(p);
-        float x[4] = {h2f(raw.x & 0xffff), h2f(raw.x >> 16), h2f(raw.y & 0xffff), h2f(raw.y >> 16)};
-        float mn = fminf(fminf(x[0], x[1]), fminf(x[2], x[3]));
-        float mx = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
-        for (int o = 1; o < lanes_per_block; o <<= 1) {
-            mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-        }
-        mn = canon_zero(mn);
-        mx = canon_zero(mx);
-        uint16_t sb = quant_scale(mn, mx);
-        float s = h2f(sb);
-        if ((lane & (lanes_per_block - 1)) == 0) {
-            int blk = lane / lanes_per_block;
-            scale_out[t * (kD / Gv) + blk] = sb;
-            zero_out[t * (kD / Gv) + blk] = f2h(mn);
-        }
-        // lane l holds channels 4l..4l+3 -> bits 8*(l%4) .. of word l/4
-        uint32_t w = 0;
+    const int k = threadIdx.x & 3;
+    const int nb = kD / Gv;   // blocks per token
+    for (int t0 = 0; t0 < n; t0 += 32) {
+        const int t = t0 + (threadIdx.x >> 2);
+        const bool live = t < n;
+        float x[32];
+        if (live) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) w |= quant_code(x[i], mn, s) << (2 * (4 * (lane & 3) + i));
-        w |= __shfl_xor_sync(0xffffffffu, w, 1);
-        w |= __shfl_xor_sync(0xffffffffu, w, 2);
-        if ((lane & 3) == 0) codes[t * 8 + (lane >> 2)] = w;
+            for (int q = 0; q < 4; ++q) h8_to_f(*reinterpret_cast<const uint4 *>(at(t, 32 * k + 8 * q)), x + 8 * q);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) x[i] = 0.f;
+        }
+        // (mn, s) of the block(s) these 32 channels fall in: halves h = 0, 1 (16 channels each)
+        float mnh[2], sh[2];
+        if (Gv == 16) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                float mn = x[16 * h], mx = x[16 * h];
+#pragma unroll
+                for (int i = 1; i < 16; ++i) {
+                    mn = fminf(mn, x[16 * h + i]);
+                    mx = fmaxf(mx, x[16 * h + i]);
+                }
+                mn = canon_zero(mn);
+                mx = canon_zero(mx);
+                const uint16_t sb = quant_scale(mn, mx);
+                if (live) {
+                    scale_out[t * nb + 2 * k + h] = sb;
+                    zero_out[t * nb + 2 * k + h] = f2h(mn);
+                }
+                mnh[h] = mn;
+                sh[h] = h2f(sb);
+            }
+        } else {
+            float mn = x[0], mx = x[0];
+#pragma unroll
+            for (int i = 1; i < 32; ++i) {
+                mn = fminf(mn, x[i]);
+                mx = fmaxf(mx, x[i]);
+            }
+            for (int o = 1; o < Gv / 32; o <<= 1) {   // the threads of one token are adjacent lanes
+                mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            }
+            mn = canon_zero(mn);
+            mx = canon_zero(mx);
+            const uint16_t sb = quant_scale(mn, mx);
+            const int per = Gv / 32;   // threads per block
+            if (live && (k % per) == 0) {
+                scale_out[t * nb + k / per] = sb;
+                zero_out[t * nb + k / per] = f2h(mn);
+            }
+            mnh[0] = mnh[1] = mn;
+            sh[0] = sh[1] = h2f(sb);
+        }
+        if (live) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                uint32_t w = 0;
+#pragma unroll
+                for (int i = 0; i < 16; ++i) w |= quant_code(x[16 * h + i], mnh[h], sh[h]) << (2 * i);
+                codes[t * 8 + 2 * k + h] = w;
+            }
+        }
     }
 }
 

@@ -193,12 +193,6 @@ __device__ __forceinline__ int part_P(const Args &a) { return a.P; }
 __device__ __forceinline__ int part_Ns(const ArgsDev &) { return dev_tab().Ns; }
 __device__ __forceinline__ int part_P(const ArgsDev &) { return dev_tab().P; }
 
-// element offset of (row, col) in a [rows][128] fp16 tile; 16-byte chunks are
-// XOR-swizzled by row so ldmatrix reads of 8 rows hit distinct banks
-__device__ __forceinline__ int swz(int row, int col) {
-    return row * kD + ((((col >> 3) ^ (row & 7))) << 3) + (col & 7);
-}
-
 // column of element `col` of query row h in the swizzled sm.qn rows
 __device__ __forceinline__ int qn_col(int h, int col) { return (((col >> 3) ^ h) << 3) | (col & 7); }
 
@@ -495,14 +489,15 @@ __device__ void residual_chunk_cta(const A &a, Smem &sm, int unit, int rc) {
         // the oldest G residual tokens become key group n_q/G and G value tokens
         const size_t tok0 = (size_t)unit * a.cap + n_q;
         const size_t grow = (size_t)unit * (a.cap / a.G) + n_q / a.G;
+        float *scr = reinterpret_cast<float *>(&sm.qn[0][0]);   // unused by residual CTAs otherwise
         if (a.G <= kResChunk) {   // the group is in this CTA's shared tile (logical rows 0..63)
             __syncthreads();
             auto kat = [&](int i, int c) -> const uint16_t * { return sm.res.k + swz(i, c); };
             auto vat = [&](int i, int c) -> const uint16_t * { return sm.res.v + swz(i, c); };
-            pack_key_group(kat, a.G, a.k_codes_w + tok0 * 8, a.k_scale_w + grow * kD, a.k_zero_w + grow * kD);
+            pack_key_group(kat, a.G, a.k_codes_w + tok0 * 8, a.k_scale_w + grow * kD, a.k_zero_w + grow * kD, scr);
             pack_value_tokens(vat, a.G, kD, a.v_codes_w + tok0 * 8, a.v_scale_w + tok0, a.v_zero_w + tok0);
         } else {
-            pack_key_group(krow, a.G, a.k_codes_w + tok0 * 8, a.k_scale_w + grow * kD, a.k_zero_w + grow * kD);
+            pack_key_group(krow, a.G, a.k_codes_w + tok0 * 8, a.k_scale_w + grow * kD, a.k_zero_w + grow * kD, scr);
             pack_value_tokens(vrow, a.G, kD, a.v_codes_w + tok0 * 8, a.v_scale_w + tok0, a.v_zero_w + tok0);
         }
     }

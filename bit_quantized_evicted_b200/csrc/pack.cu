@@ -5,8 +5,9 @@
 // into a compact layout.  The newest r tokens stay fp16 in the residual ring.
 //
 // Grid (n_groups + n_res_blocks, B*Hkv), 128 threads.  Block x < n_groups packs
-// key group x (G tokens, thread = channel) and the same G value tokens (warp =
-// token); the remaining blocks copy residual tokens into ring slots 0..r-1.
+// key group x and the same G value tokens: it first stages the G key and value
+// rows in shared memory (cp.async, all in flight), then quantizes from there;
+// the remaining blocks copy residual tokens into ring slots 0..r-1.
 // Memory-bound: 512 B read and 84 B written per packed token and KV head.
 //
 // minikv_evict_pack runs the same kernel with an index list: compacted token
@@ -33,6 +34,7 @@ struct PackArgs {
 };
 
 constexpr int kResPerBlock = 32;   // residual tokens copied per block
+constexpr int kStageG = 64;        // key groups up to this size are staged in shared memory (32 KB)
 
 __global__ void __launch_bounds__(128) pack_kernel(const PackArgs a) {
     const int src_unit = blockIdx.y;           // unit of the source tensors
@@ -48,13 +50,35 @@ __global__ void __launch_bounds__(128) pack_kernel(const PackArgs a) {
     if ((int)blockIdx.x < a.n_groups) {
         const int grp = blockIdx.x;
         const int t0 = grp * a.G;
-        auto krow = [&](int t, int c) { return ku + src_row(t0 + t) * kD + c; };
-        auto vrow = [&](int t, int c) { return vu + src_row(t0 + t) * kD + c; };
         const size_t tok = (size_t)unit * a.cap + t0;
         const size_t grow = (size_t)unit * (a.cap / a.G) + grp;
-        pack_key_group(krow, a.G, a.k_codes + tok * 8, a.k_scale + grow * kD, a.k_zero + grow * kD);
-        pack_value_tokens(vrow, a.G, a.Gv, a.v_codes + tok * 8, a.v_scale + tok * (kD / a.Gv),
-                          a.v_zero + tok * (kD / a.Gv));
+        __shared__ float scr[256];
+        if (a.G <= kStageG) {
+            // stage the group's G key rows and G value rows in shared memory
+            // (swizzled), every 16-byte copy in flight at once, then pack from there
+            extern __shared__ __align__(16) uint16_t tile[];   // [2][G][128]
+            uint16_t *kt = tile, *vt = tile + a.G * kD;
+            for (int e = threadIdx.x; e < a.G * 16; e += 128) {
+                const int t = e >> 4, ch = e & 15;
+                const size_t src = src_row(t0 + t) * kD + ch * 8;
+                cp_async16(smem_addr(kt + swz(t, ch * 8)), ku + src, true);
+                cp_async16(smem_addr(vt + swz(t, ch * 8)), vu + src, true);
+            }
+            cp_async_commit();
+            cp_async_wait<0>();
+            __syncthreads();
+            auto kat = [&](int t, int c) -> const uint16_t * { return kt + swz(t, c); };
+            auto vat = [&](int t, int c) -> const uint16_t * { return vt + swz(t, c); };
+            pack_key_group(kat, a.G, a.k_codes + tok * 8, a.k_scale + grow * kD, a.k_zero + grow * kD, scr);
+            pack_value_tokens(vat, a.G, a.Gv, a.v_codes + tok * 8, a.v_scale + tok * (kD / a.Gv),
+                              a.v_zero + tok * (kD / a.Gv));
+        } else {
+            auto krow = [&](int t, int c) { return ku + src_row(t0 + t) * kD + c; };
+            auto vrow = [&](int t, int c) { return vu + src_row(t0 + t) * kD + c; };
+            pack_key_group(krow, a.G, a.k_codes + tok * 8, a.k_scale + grow * kD, a.k_zero + grow * kD, scr);
+            pack_value_tokens(vrow, a.G, a.Gv, a.v_codes + tok * 8, a.v_scale + tok * (kD / a.Gv),
+                              a.v_zero + tok * (kD / a.Gv));
+        }
     } else {
         const int i0 = ((int)blockIdx.x - a.n_groups) * kResPerBlock;
         // 16 x 16-byte chunks per token row; 128 threads copy 8 rows per pass
@@ -104,7 +128,8 @@ int pack_launch(minikv_cache *c, const uint16_t *k, const uint16_t *v, int N, cu
     if (c->dseq && gx == 0) gx = 1;   // an empty load still sets the device state
     const int units = seq >= 0 ? c->Hkv : c->B * c->Hkv;
     if (gx > 0 && units > 0) {
-        pack_kernel<<<dim3(gx, units), 128, 0, stream>>>(a);
+        const size_t smem = c->G <= kStageG ? (size_t)2 * c->G * kD * sizeof(uint16_t) : 0;
+        pack_kernel<<<dim3(gx, units), 128, smem, stream>>>(a);
         int rc = check_launch("quant_pack");
         if (rc) return rc;
     }
