@@ -95,12 +95,15 @@ def peaks():
         return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
 
 
-def recorded_traffic(kernel: str, source: str):
+def recorded_traffic(kernel: str, sources):
     """dram bytes per launch from the committed ncu summary, if it was taken on
-    the current source of the kernel (else None)."""
+    the current sources of the kernel (else None)."""
     path = os.path.join(ROOT, "profiles", "traffic.txt")
     try:
-        sha = hashlib.sha256(open(source, "rb").read()).hexdigest()[:16]
+        h = hashlib.sha256()
+        for src in sources:
+            h.update(open(src, "rb").read())
+        sha = h.hexdigest()[:16]
         for line in open(path):
             f = line.split()
             if len(f) >= 4 and f[0] == kernel and f[1] == sha:
@@ -607,8 +610,9 @@ def run_gpu(args):
                          f"heads, fp64) in {dt:.1f} s on {threads} threads, scaled to 32 layers x 16 x 8 units "
                          f"per step"}
 
+    csrc = os.path.join(ROOT, "bit_quantized_evicted_b200", "csrc")
     traffic, traffic_note = recorded_traffic(
-        "decode_kernel", os.path.join(ROOT, "bit_quantized_evicted_b200", "csrc", "decode.cu"))
+        "decode_kernel", [os.path.join(csrc, "decode.cu"), os.path.join(csrc, "common.cuh")])
     if DECODE.get("mass"):
         traffic, traffic_note = None, "no capture of the attention-mass variant (decode_kernel<true> + mass_kernel)"
     if rank == 0:

@@ -136,12 +136,35 @@ __device__ __forceinline__ void bulk_g2s(void *sdst, const void *gsrc, uint32_t 
 __device__ __forceinline__ uint16_t quant_scale(float mn, float mx) {
     return f2h(__fdiv_rn(__fsub_rn(mx, mn), 3.0f));
 }
-// code = clamp(rint((x - zero) / scale), 0, 3), 0 when scale == 0.
+// code = clamp(rint((x - zero) / scale), 0, 3), 0 when scale == 0: the
+// definition; the pack helpers compute it as quant_code_thr below.
 __device__ __forceinline__ uint32_t quant_code(float x, float zero, float scale) {
     if (scale == 0.0f) return 0u;
     float q = rintf(__fdiv_rn(__fsub_rn(x, zero), scale));
     q = fminf(fmaxf(q, 0.0f), 3.0f);
     return static_cast<uint32_t>(q);
+}
+// The same code without a division.  With d = fp32(x - zero) >= 0 and s > 0,
+// rint(RN(d / s)) is decided by where the exact quotient d/s lies against the
+// rounding boundaries of RN at 0.5, 1.5 and 2.5 (ties to even):
+//   code >= 1  <=>  RN(d/s) >  0.5  <=>  d/s >  0.5 + 2^-25
+//   code >= 2  <=>  RN(d/s) >= 1.5  <=>  d/s >= 1.5 - 2^-24
+//   code >= 3  <=>  RN(d/s) >  2.5  <=>  d/s >  2.5 + 2^-23
+// Each boundary times s is exact in fp64 (at most 25 x 24 significant bits);
+// rounding it down (for >) or up (for >=) to fp32 gives a threshold that an
+// fp32 d can be compared with exactly.  s == 0 gives code 0 everywhere.
+struct QThr {
+    float t1, t2, t3;
+};
+__device__ __forceinline__ QThr quant_thresholds(float s) {
+    if (s == 0.0f) return {INFINITY, INFINITY, INFINITY};
+    const double sd = (double)s;
+    return {__double2float_rd(sd * (0.5 + 0x1p-25)), __double2float_ru(sd * (1.5 - 0x1p-24)),
+            __double2float_rd(sd * (2.5 + 0x1p-23))};
+}
+__device__ __forceinline__ uint32_t quant_code_thr(float x, float zero, const QThr &t) {
+    const float d = __fsub_rn(x, zero);
+    return (uint32_t)(d > t.t1) + (uint32_t)(d >= t.t2) + (uint32_t)(d > t.t3);
 }
 // -0 and +0 are the same extreme; store +0.
 __device__ __forceinline__ float canon_zero(float x) { return __fadd_rn(x, 0.0f); }
@@ -167,14 +190,14 @@ __device__ __forceinline__ void h8_to_f(uint4 v, float *x) {
 // one (scale, zero) per channel.  Called by all 128 threads of a CTA.
 // at(t, c) points to channel c of token t (global or shared memory); the 8
 // channels of each aligned 8-channel chunk are contiguous and 16-byte aligned.
-// scr: 256 floats of shared scratch.
+// scr: 512 floats of shared scratch.
 //   1. thread c: min / max of channel c over the G tokens -> (zero, scale);
 //   2. thread i: code words i, i + 128, ... (token w / 8, channels 16 (w % 8)
 //      .. +15), each from two 16-byte loads and 16 independent quantizations.
 template <class AtFn>
 __device__ __forceinline__ void pack_key_group(AtFn at, int G, uint32_t *codes /* [G][8] */,
                                                uint16_t *scale_out /* [128] */, uint16_t *zero_out,
-                                               float *scr /* [256] shared */) {
+                                               float *scr /* [512] shared */) {
     const int c = threadIdx.x;
     float mn = INFINITY, mx = -INFINITY;
 #pragma unroll 8
@@ -188,8 +211,11 @@ __device__ __forceinline__ void pack_key_group(AtFn at, int G, uint32_t *codes /
     const uint16_t sb = quant_scale(mn, mx);
     scale_out[c] = sb;
     zero_out[c] = f2h(mn);
+    const QThr th = quant_thresholds(h2f(sb));
     scr[c] = mn;
-    scr[128 + c] = h2f(sb);
+    scr[128 + c] = th.t1;
+    scr[256 + c] = th.t2;
+    scr[384 + c] = th.t3;
     __syncthreads();
     for (int wi = c; wi < G * 8; wi += 128) {
         const int t = wi >> 3, c0 = 16 * (wi & 7);
@@ -198,7 +224,10 @@ __device__ __forceinline__ void pack_key_group(AtFn at, int G, uint32_t *codes /
         h8_to_f(*reinterpret_cast<const uint4 *>(at(t, c0 + 8)), x + 8);
         uint32_t w = 0;
 #pragma unroll
-        for (int i = 0; i < 16; ++i) w |= quant_code(x[i], scr[c0 + i], scr[128 + c0 + i]) << (2 * i);
+        for (int i = 0; i < 16; ++i) {
+            const QThr t = {scr[128 + c0 + i], scr[256 + c0 + i], scr[384 + c0 + i]};
+            w |= quant_code_thr(x[i], scr[c0 + i], t) << (2 * i);
+        }
         codes[wi] = w;
     }
     __syncthreads();   // scr is free again
@@ -226,7 +255,8 @@ __device__ __forceinline__ void pack_value_tokens(AtFn at, int n, int Gv, uint32
             for (int i = 0; i < 32; ++i) x[i] = 0.f;
         }
         // (mn, s) of the block(s) these 32 channels fall in: halves h = 0, 1 (16 channels each)
-        float mnh[2], sh[2];
+        float mnh[2];
+        QThr th[2];
         if (Gv == 16) {
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
@@ -244,7 +274,7 @@ __device__ __forceinline__ void pack_value_tokens(AtFn at, int n, int Gv, uint32
                     zero_out[t * nb + 2 * k + h] = f2h(mn);
                 }
                 mnh[h] = mn;
-                sh[h] = h2f(sb);
+                th[h] = quant_thresholds(h2f(sb));
             }
         } else {
             float mn = x[0], mx = x[0];
@@ -266,14 +296,14 @@ __device__ __forceinline__ void pack_value_tokens(AtFn at, int n, int Gv, uint32
                 zero_out[t * nb + k / per] = f2h(mn);
             }
             mnh[0] = mnh[1] = mn;
-            sh[0] = sh[1] = h2f(sb);
+            th[0] = th[1] = quant_thresholds(h2f(sb));
         }
         if (live) {
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 uint32_t w = 0;
 #pragma unroll
-                for (int i = 0; i < 16; ++i) w |= quant_code(x[16 * h + i], mnh[h], sh[h]) << (2 * i);
+                for (int i = 0; i < 16; ++i) w |= quant_code_thr(x[16 * h + i], mnh[h], th[h]) << (2 * i);
                 codes[t * 8 + 2 * k + h] = w;
             }
         }

@@ -52,7 +52,7 @@ __global__ void __launch_bounds__(128) pack_kernel(const PackArgs a) {
         const int t0 = grp * a.G;
         const size_t tok = (size_t)unit * a.cap + t0;
         const size_t grow = (size_t)unit * (a.cap / a.G) + grp;
-        __shared__ float scr[256];
+        __shared__ float scr[512];
         if (a.G <= kStageG) {
             // stage the group's G key rows and G value rows in shared memory
             // (swizzled), every 16-byte copy in flight at once, then pack from there
