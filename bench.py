@@ -113,6 +113,27 @@ def recorded_traffic(kernel: str, sources):
     return None, None
 
 
+# ------------------------------------------------------------ multi-rank
+
+def max_over_ranks(x: float, device) -> float:
+    """The largest of every rank's x (the job is as slow as its slowest rank);
+    x itself when the job has one rank.  `device` is where the all-reduce
+    tensor lives (the rank's GPU under NCCL, the CPU under gloo)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(batch: int, steps: int, world: int, ms: float) -> float:
+    """Whole-job throughput: every rank generates `batch` tokens per step, and
+    the job took `ms` (the slowest rank's time)."""
+    return batch * steps * world / (ms * 1e-3)
+
+
 # ----------------------------------------------------------------- clocks
 
 class ClockSampler:
@@ -524,11 +545,8 @@ def run_gpu(args):
         kern_ms = [evs[s][l][0].elapsed_time(evs[s][l][1]) for s in range(args.steps) for l in range(L)]
     else:   # a replay runs the L layer launches back to back: its time / L per launch (gaps included)
         kern_ms = [sev[s][0].elapsed_time(sev[s][1]) / L for s in range(args.steps)]
-    if world > 1:
-        t = torch.tensor([ms], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-    tok_s = B * args.steps * world / (ms * 1e-3)
+    ms = max_over_ranks(ms, device)
+    tok_s = job_tokens_per_s(B, args.steps, world, ms)
     alg_bytes = sum(sum(sb) for sb in nbytes)
     mean_launch_bytes = sum(launch_bytes) / len(launch_bytes)
     mean_launch_s = statistics.mean(kern_ms) * 1e-3
@@ -587,11 +605,8 @@ def run_gpu(args):
     barrier()
     del g_e2e
     e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_tok_s = B * args.steps * world / (e2e_ms * 1e-3)
+    e2e_ms = max_over_ranks(e2e_ms, device)
+    e2e_tok_s = job_tokens_per_s(B, args.steps, world, e2e_ms)
     status_bad = sum(sum(c.status()) for c in caches)
     if status_bad:
         raise RuntimeError(f"{status_bad} sequences hit the cache capacity")
