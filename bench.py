@@ -383,11 +383,11 @@ class LengthMirror:
                     s[1] -= self.G
 
 
-def decode_call(mk, c, q, kn, vn, out, ws):
+def decode_call(mk, c, q, kn, vn, out, ws, stream):
     if c.mass is not None:
-        mk.decode_attn_mass(c, q, kn, vn, c.mass, out=out, ws=ws)
+        mk.decode_attn_mass(c, q, kn, vn, c.mass, out=out, ws=ws, stream=stream)
     else:
-        mk.decode_attn(c, q, kn, vn, out=out, ws=ws)
+        mk.decode_attn(c, q, kn, vn, out=out, ws=ws, stream=stream)
 
 
 def run_prefill(torch, mk, synth, device):
@@ -486,14 +486,16 @@ def run_gpu(args):
     P = qin.shape[0]
 
     def layer_calls(q_src, kn_src, vn_src, p, ev=None, o=None):
-        """One decode step: the L layer calls, on the current stream."""
+        """One decode step: the L layer calls, on the current stream (looked up
+        once per step, not once per call: it is host time on every call)."""
         o = out if o is None else o
+        cur = torch.cuda.current_stream()
         for l in range(L):
             if ev is not None:
-                ev[l][0].record()
-            decode_call(mk, caches[l], q_src[p, l], kn_src[p, l], vn_src[p, l], o[l], ws)
+                ev[l][0].record(cur)
+            decode_call(mk, caches[l], q_src[p, l], kn_src[p, l], vn_src[p, l], o[l], ws, cur)
             if ev is not None:
-                ev[l][1].record()
+                ev[l][1].record(cur)
 
     def step_bytes():
         return [mirror.layer_bytes(l, Hkv, with_mass) for l in range(L)]

@@ -288,23 +288,49 @@ __device__ void finish_unit(const A &a, Smem &sm, int unit, int slot, int S_u, c
     const float *ub = a.part + (size_t)unit * a.S_max * 4 * kPartStride;
     const int b = unit / a.Hkv, kvh = unit % a.Hkv;
     const int Hq = a.Hkv * a.g;
-    for (int h = 0; h < a.g; ++h) {
-        float M = -INFINITY;
-        for (int s = 0; s < S_u; ++s) M = fmaxf(M, __ldcg(ub + (s * 4 + h) * kPartStride + 128));
-        float L = 0.f, Y = 0.f;
-        for (int s = 0; s < S_u; ++s) {
-            const float *p = ub + (s * 4 + h) * kPartStride;
-            const float ms = __ldcg(p + 128);
-            const float f = (ms == -INFINITY) ? 0.f : ex2(ms - M);
-            L += f * __ldcg(p + 129);
-            Y += f * __ldcg(p + tid);
-        }
-        a.out[((size_t)b * Hq + kvh * a.g + h) * kD + tid] = f2h(__fdividef(Y, L));
-        if (kMass && tid == 0) {
-            a.stats[unit * 12 + h] = M;
-            a.stats[unit * 12 + 4 + h] = L;
-        }
+    // one pass over the unit's partials, all heads together, four slots per
+    // round with every load of the round issued before any is used (online
+    // rescaling: the running max moves to the larger of the two)
+    float M[4], L[4], Y[4];
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+        M[h] = -INFINITY;
+        L[h] = 0.f;
+        Y[h] = 0.f;
     }
+    for (int s0 = 0; s0 < S_u; s0 += 4) {
+        float ms[4][4], ls[4][4], ys[4][4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+                const bool ok = (s0 + j < S_u) && (h < a.g);
+                const float *p = ub + ((s0 + j) * 4 + h) * kPartStride;
+                ms[j][h] = ok ? __ldcg(p + 128) : -INFINITY;
+                ls[j][h] = ok ? __ldcg(p + 129) : 0.f;
+                ys[j][h] = ok ? __ldcg(p + tid) : 0.f;
+            }
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+                const float m = ms[j][h], Mn = fmaxf(M[h], m);
+                const float fo = (M[h] == -INFINITY) ? 0.f : ex2(M[h] - Mn);
+                const float fs = (m == -INFINITY) ? 0.f : ex2(m - Mn);
+                L[h] = fmaf(L[h], fo, ls[j][h] * fs);
+                Y[h] = fmaf(Y[h], fo, ys[j][h] * fs);
+                M[h] = Mn;
+            }
+    }
+#pragma unroll
+    for (int h = 0; h < 4; ++h)
+        if (h < a.g) {
+            a.out[((size_t)b * Hq + kvh * a.g + h) * kD + tid] = f2h(__fdividef(Y[h], L[h]));
+            if (kMass && tid == 0) {
+                a.stats[unit * 12 + h] = M[h];
+                a.stats[unit * 12 + 4 + h] = L[h];
+            }
+        }
     if (kMass && tid == 0) a.stats[unit * 12 + 8] = __int_as_float(len_nq(a, unit) + len_r(a, unit));
 }
 
