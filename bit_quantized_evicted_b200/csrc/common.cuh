@@ -13,6 +13,15 @@ int fail(int code, const char *fmt, ...);
 int check_launch(const char *what);
 
 constexpr int kD = 128;                  // the one supported head size
+constexpr int kMaxDevices = 64;          // device ordinals of the per-device set-up caches
+
+// The current device's ordinal, or -1 if it cannot be read or is not below
+// kMaxDevices (host code; per-device caches are indexed by it).
+inline int current_device() {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+    return (dev >= 0 && dev < kMaxDevices) ? dev : -1;
+}
 constexpr float kLog2e = 1.4426950408889634f;
 
 __device__ __forceinline__ float h2f(uint16_t b) { return __half2float(__ushort_as_half(b)); }

@@ -35,7 +35,6 @@ size_t decode_call_workspace_bytes(const minikv_cache *c);
 namespace {
 
 constexpr size_t kStaticScratchBytes = size_t(8) << 20;
-constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) unsigned char g_decode_scratch[kStaticScratchBytes];
 
@@ -43,11 +42,20 @@ std::mutex g_mu;
 void *g_scratch_addr[kMaxDevices] = {};
 
 // Device address of g_decode_scratch on the current device (looked up once).
-int scratch_address(void **out) {
+// The work is queued on `stream`, so the stream must belong to that device:
+// otherwise the kernel would clear and use another GPU's copy of the array.
+int scratch_address(cudaStream_t stream, void **out) {
     int dev = -1;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return fail(MINIKV_ERR_CUDA, "decode_attn_static: cudaGetDevice: %s", cudaGetErrorString(e));
     if (dev < 0 || dev >= kMaxDevices) return fail(MINIKV_ERR_UNSUPPORTED, "decode_attn_static: device %d", dev);
+    int sdev = -1;
+    e = cudaStreamGetDevice(stream, &sdev);
+    if (e != cudaSuccess)
+        return fail(MINIKV_ERR_INVALID_ARG, "decode_attn_static: cudaStreamGetDevice: %s", cudaGetErrorString(e));
+    if (sdev != dev)
+        return fail(MINIKV_ERR_INVALID_ARG, "decode_attn_static: the stream belongs to device %d, the current device is %d",
+                    sdev, dev);
     std::lock_guard<std::mutex> lock(g_mu);
     if (!g_scratch_addr[dev]) {
         void *p = nullptr;
@@ -76,10 +84,10 @@ extern "C" int minikv_decode_attn_static(minikv_cache *c, const uint16_t *q, con
                     "decode_attn_static: this step needs %zu bytes of scratch but the static buffer holds %zu; "
                     "use minikv_decode_attn with a caller workspace",
                     need, kStaticScratchBytes);
-    void *scratch = nullptr;
-    rc = scratch_address(&scratch);
-    if (rc) return rc;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    void *scratch = nullptr;
+    rc = scratch_address(s, &scratch);
+    if (rc) return rc;
     cudaError_t e = cudaMemsetAsync(scratch, 0, decode_counter_bytes(c->B, c->Hkv), s);
     if (e != cudaSuccess)
         return fail(MINIKV_ERR_CUDA, "decode_attn_static: clearing counters: %s", cudaGetErrorString(e));

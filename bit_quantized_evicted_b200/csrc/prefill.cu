@@ -9,10 +9,13 @@
 // probabilities P[i, j] = exp(s_ij - lse_i) and sums them per key over the rows
 // and over the query heads of each KV head.
 //
-// Kernel 1 (fa_fwd_kernel): 64 query rows x 64 keys per step, 4 warps of 16
-// rows, fp16 mma.sync with fp32 accumulation, K/V double-buffered by cp.async
-// in XOR-swizzled shared memory.  Kernel 2 (window_score_kernel): one CTA per
-// 64 keys of one KV head; S^T = K Q_w^T on the tensor cores, then column sums.
+// Kernel 1 (fa_tc_kernel): one CTA per 128-row query tile of one (sequence,
+// query head); S = Q K^T and O += P V on the tcgen05 tensor cores with fp32
+// accumulators in tensor memory, Q/K/V brought in by TMA (128-byte swizzle),
+// warp-specialised K and V producers, a single MMA-issuing thread and four
+// softmax warps (one thread per query row).  Kernel 2 (window_score_kernel):
+// one CTA per 64 keys of one KV head; S^T = K Q_w^T with mma.sync, then the
+// column sums of exp(S - lse) over the window rows.
 #include <cudaTypedefs.h>
 #include <math.h>
 
@@ -455,8 +458,11 @@ __global__ void __launch_bounds__(128) window_score_kernel(const ScoreArgs a) {
     }
 }
 
-bool g_attr_fa = false;
-size_t g_attr_score = 0;
+// Shared-memory opt-ins, per device (a function attribute applies to the device
+// current when it is set), guarded for calls from several host threads.
+std::mutex g_attr_mu;
+bool g_attr_fa[kMaxDevices] = {};
+size_t g_attr_score[kMaxDevices] = {};
 
 std::mutex g_encode_mu;
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
@@ -501,11 +507,16 @@ int prefill_launch(const uint16_t *q, const uint16_t *k, const uint16_t *v, int 
     fa.nqt = (T + kTileM - 1) / kTileM;
     fa.scale_log2 = sm_scale * kLog2e;
     const size_t fa_smem = sizeof(FaSmem) + 1024;
-    if (!g_attr_fa) {
-        if (cudaFuncSetAttribute(fa_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fa_smem) !=
-            cudaSuccess)
-            return check_launch("select_prefill: attribute");
-        g_attr_fa = true;
+    const int dev = current_device();
+    if (dev < 0) return check_launch("select_prefill: cudaGetDevice");
+    {
+        std::lock_guard<std::mutex> lk(g_attr_mu);
+        if (!g_attr_fa[dev]) {
+            if (cudaFuncSetAttribute(fa_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fa_smem) !=
+                cudaSuccess)
+                return check_launch("select_prefill: attribute");
+            g_attr_fa[dev] = true;
+        }
     }
     fa_tc_kernel<<<(unsigned)(fa.nqt * B * Hq), kFaThreads, fa_smem, stream>>>(mq, mk, mv, mo, fa);
     rc = check_launch("select_prefill: flash attention");
@@ -517,11 +528,14 @@ int prefill_launch(const uint16_t *q, const uint16_t *k, const uint16_t *v, int 
     sa.scale_log2 = fa.scale_log2;
     const int nrows8 = ((Hq / Hkv) * W + 7) / 8 * 8;
     const size_t sc_smem = (size_t)kBN * kD * 2 + (size_t)nrows8 * kD * 2 + (size_t)nrows8 * 4;
-    if (sc_smem > g_attr_score) {
-        if (cudaFuncSetAttribute(window_score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sc_smem) !=
-            cudaSuccess)
-            return check_launch("select_prefill: attribute");
-        g_attr_score = sc_smem;
+    {
+        std::lock_guard<std::mutex> lk(g_attr_mu);
+        if (sc_smem > g_attr_score[dev]) {
+            if (cudaFuncSetAttribute(window_score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)sc_smem) != cudaSuccess)
+                return check_launch("select_prefill: attribute");
+            g_attr_score[dev] = sc_smem;
+        }
     }
     window_score_kernel<<<dim3((T + kBN - 1) / kBN, B * Hkv), 128, sc_smem, stream>>>(sa);
     return check_launch("select_prefill: window scores");

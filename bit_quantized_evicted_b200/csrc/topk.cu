@@ -20,8 +20,10 @@ namespace {
 
 constexpr int kSelThreads = 1024;
 
+// Order-preserving unsigned key of an fp32 score.  -0 and +0 are one value
+// (the selection compares scores as numbers), so -0 is first made +0.
 __device__ __forceinline__ uint32_t order_key(float f) {
-    uint32_t u = __float_as_uint(f);
+    uint32_t u = __float_as_uint(__fadd_rn(f, 0.0f));
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 

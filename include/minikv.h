@@ -131,10 +131,10 @@ MINIKV_API int minikv_cache_set_ragged(minikv_cache *c, int *seq);
  *   host-side state (also empty).
  * In this mode the loaders (minikv_quant_pack, minikv_evict_pack and their
  * _seq forms) write the loaded rows' state into dseq from their kernel, and
- * each decode call (minikv_decode_attn, _mass, _static) runs one launch
- * configuration fixed by the cache's shape: the kernel reads the state,
- * splits this step's packed tokens over its CTAs, and its last CTA advances
- * every sequence's state.  A step whose flush would pass `cap` leaves that
+ * each decode call runs one launch configuration fixed by the cache's shape:
+ * the kernel reads the state, splits this step's packed tokens over its CTAs,
+ * and its last CTA advances every sequence's state (minikv_decode_attn_static
+ * reads and advances the same state).  A step whose flush would pass `cap` leaves that
  * sequence's state unchanged (its new token is not kept) and sets its status
  * word to 1; the host learns it by reading dseq.  Capacity is therefore not
  * checked on the host in this mode.
@@ -326,7 +326,9 @@ MINIKV_API int minikv_decode_attn_mass(minikv_cache *c, const uint16_t *q, const
  * (cudaGetSymbolAddress, that device current); make it before any stream
  * capture.  All calls share the array: calls whose GPU work overlaps race on
  * it.  Each call clears the array's arrival counters on `stream` first.  No
- * call allocates or frees device memory.
+ * call allocates or frees device memory.  `stream` must belong to the current
+ * device (the array's address is the current device's); otherwise the call
+ * fails with MINIKV_ERR_INVALID_ARG and queues nothing.
  */
 MINIKV_API int minikv_decode_attn_static(minikv_cache *c, const uint16_t *q, const uint16_t *k_new,
                                          const uint16_t *v_new, int Hq, float sm_scale, uint16_t *out,

@@ -165,6 +165,27 @@ def test_topk_exact_with_ties(B, H, T, W, keep):
     assert torch.equal(vk, torch.gather(v, 2, ri[..., None].expand(-1, -1, -1, 128)))
 
 
+@pytest.mark.parametrize("T,W,keep", [(2, 0, 1), (300, 8, 40), (1000, 16, 700), (4100, 32, 600)])
+def test_topk_signed_zeros_tie(T, W, keep):
+    """-0 and +0 are the same score: among them the lower index is kept,
+    exactly as the oracle (which compares the scores as numbers) keeps it."""
+    gen = torch.Generator().manual_seed(T)
+    s = torch.randint(0, 3, (1, 2, T), generator=gen).float() / 4.0   # many exact ties
+    zeros = torch.rand((1, 2, T), generator=gen) < 0.5
+    sign = torch.where(torch.rand((1, 2, T), generator=gen) < 0.5, -1.0, 1.0)
+    s = torch.where(zeros, sign * 0.0, s)   # about half the scores are -0 or +0
+    if T == 2:
+        s[0, :, 0], s[0, :, 1] = -0.0, 0.0   # [-0, +0], keep 1: index 0
+    s = s.to(DEV)
+    k, v = _kv(1, 2, T, 57)
+    idx, kk, vk = mk.topk_evict(s, k, v, W, keep)
+    torch.cuda.synchronize()
+    ref = _select_ref(s.cpu().numpy(), W, keep)
+    np.testing.assert_array_equal(idx.cpu().numpy(), ref)
+    if T == 2:
+        assert idx.cpu().numpy()[0, :, 0].tolist() == [0, 0]
+
+
 # ------------------------------------------------------------- decode
 
 @pytest.mark.parametrize("B,Hq,Hkv,N,G,R,steps", [

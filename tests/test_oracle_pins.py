@@ -132,6 +132,29 @@ def test_quantizer_exact_ramp(oracle):
             assert np.array_equal(codes, c)
 
 
+def test_quantizer_exact_half_way_quotients_round_to_even(oracle):
+    """Groups whose (x - zero)/scale lands exactly on 0.5, 1.5 and 2.5: the
+    reading of the quantizer rounds those ties to even, so the codes are
+    0, 2, 2 (rounding half away from zero would give 1, 2, 3).  Every value,
+    the scale and (x - zero)/scale are exact in fp16/fp32, so the expected
+    codes below are written by hand."""
+    cases = [
+        # zero, scale, x / scale offsets from zero, expected codes
+        (0.0, 0.25, [0.0, 0.5, 1.5, 2.5, 3.0, 1.0, 2.0], [0, 0, 2, 2, 3, 1, 2]),
+        (-1.0, 0.5, [0.0, 0.5, 1.5, 2.5, 3.0], [0, 0, 2, 2, 3]),
+        (2.0, 3.0, [0.0, 0.5, 1.5, 2.5, 3.0], [0, 0, 2, 2, 3]),
+        (-6.0, 0.0625, [3.0, 2.5, 0.5, 1.5, 0.0, 2.5], [3, 2, 0, 2, 0, 2]),
+    ]
+    for zero, s, offs, want in cases:
+        xd = zero + np.asarray(offs) * s
+        x = f16(xd)
+        assert np.array_equal(x.astype(np.float64), xd)   # exact in fp16
+        s_bits, z_bits, codes = oracle.quantize_group(x)
+        assert np.uint16(s_bits).view(np.float16) == np.float16(s)
+        assert np.uint16(z_bits).view(np.float16) == np.float16(zero)
+        assert codes.tolist() == want, (zero, s, codes.tolist())
+
+
 # ------------------------------------------------------------ O7 packing
 
 def _unpack(words, D):
