@@ -196,37 +196,40 @@ __device__ __forceinline__ void h8_to_f(uint4 v, float *x) {
 }
 
 // Pack one key group: G tokens x 128 channels -> codes (token-major words),
-// one (scale, zero) per channel.  Called by all 128 threads of a CTA.
+// one (scale, zero) per channel.  Called by all NT threads of a CTA (NT a
+// multiple of 128; threads 0..127 take one channel each in step 1).
 // at(t, c) points to channel c of token t (global or shared memory); the 8
 // channels of each aligned 8-channel chunk are contiguous and 16-byte aligned.
 // scr: 512 floats of shared scratch.
 //   1. thread c: min / max of channel c over the G tokens -> (zero, scale);
 //   2. thread i: code words i, i + 128, ... (token w / 8, channels 16 (w % 8)
 //      .. +15), each from two 16-byte loads and 16 independent quantizations.
-template <class AtFn>
+template <int NT = 128, class AtFn>
 __device__ __forceinline__ void pack_key_group(AtFn at, int G, uint32_t *codes /* [G][8] */,
                                                uint16_t *scale_out /* [128] */, uint16_t *zero_out,
                                                float *scr /* [512] shared */) {
     const int c = threadIdx.x;
-    float mn = INFINITY, mx = -INFINITY;
+    if (c < kD) {
+        float mn = INFINITY, mx = -INFINITY;
 #pragma unroll 8
-    for (int t = 0; t < G; ++t) {
-        const float x = h2f(*at(t, c));
-        mn = fminf(mn, x);
-        mx = fmaxf(mx, x);
+        for (int t = 0; t < G; ++t) {
+            const float x = h2f(*at(t, c));
+            mn = fminf(mn, x);
+            mx = fmaxf(mx, x);
+        }
+        mn = canon_zero(mn);
+        mx = canon_zero(mx);
+        const uint16_t sb = quant_scale(mn, mx);
+        scale_out[c] = sb;
+        zero_out[c] = f2h(mn);
+        const QThr th = quant_thresholds(h2f(sb));
+        scr[c] = mn;
+        scr[128 + c] = th.t1;
+        scr[256 + c] = th.t2;
+        scr[384 + c] = th.t3;
     }
-    mn = canon_zero(mn);
-    mx = canon_zero(mx);
-    const uint16_t sb = quant_scale(mn, mx);
-    scale_out[c] = sb;
-    zero_out[c] = f2h(mn);
-    const QThr th = quant_thresholds(h2f(sb));
-    scr[c] = mn;
-    scr[128 + c] = th.t1;
-    scr[256 + c] = th.t2;
-    scr[384 + c] = th.t3;
     __syncthreads();
-    for (int wi = c; wi < G * 8; wi += 128) {
+    for (int wi = c; wi < G * 8; wi += NT) {
         const int t = wi >> 3, c0 = 16 * (wi & 7);
         float x[16];
         h8_to_f(*reinterpret_cast<const uint4 *>(at(t, c0)), x);
@@ -243,16 +246,16 @@ __device__ __forceinline__ void pack_key_group(AtFn at, int G, uint32_t *codes /
 }
 
 // Pack value tokens: each of n tokens is quantized per block of Gv channels.
-// Called by all 128 threads: thread 4j + k of a pass takes token (pass * 32 + j)
+// Called by all NT threads: thread 4j + k of a pass takes token (pass * NT/4 + j)
 // and its channels 32k .. 32k+31 (two code words); min / max of a block wider
 // than 32 channels are combined over the Gv/32 threads that share it.
 // Gv in {16, 32, 64, 128}.  at() as for pack_key_group.
-template <class AtFn>
+template <int NT = 128, class AtFn>
 __device__ __forceinline__ void pack_value_tokens(AtFn at, int n, int Gv, uint32_t *codes /* [n][8] */,
                                                   uint16_t *scale_out /* [n][128/Gv] */, uint16_t *zero_out) {
     const int k = threadIdx.x & 3;
     const int nb = kD / Gv;   // blocks per token
-    for (int t0 = 0; t0 < n; t0 += 32) {
+    for (int t0 = 0; t0 < n; t0 += NT / 4) {
         const int t = t0 + (threadIdx.x >> 2);
         const bool live = t < n;
         float x[32];

@@ -4,42 +4,49 @@
 // FlashAttention) and the gptget.net summary of arXiv 2411.18077, section
 // 方法论 (sub-channel key / per-token value 2-bit quantization, compact layout).
 //
-// One launch per layer-step, one CTA of 4 warps per work item:
-//   * residual CTAs, n_rc per (sequence, KV head) "unit": 64-token chunks of the
-//     fp16 residual ring, staged by cp.async into swizzled shared memory; the
-//     chunk holding the new token appends it to the ring, chunk 0 packs the
-//     oldest G tokens to 2 bits when the residual is full (same code as
-//     minikv_quant_pack);
-//   * packed CTAs, sized to fill the GPU once: the packed tokens of all units,
-//     cut into 32-token slices, are laid end to end and split evenly into P
-//     contiguous ranges (one per CTA).  Each warp owns a 4-stage TMA-bulk
-//     pipeline (cp.async.bulk + mbarrier) over its slices of the range.
-// Every CTA writes one partial softmax state (m, l, sum p*v) per unit it
-// touched; the last CTA to arrive at a unit (self-resetting atomic counter)
-// merges them into `out`.
+// Work list.  Every (sequence, KV head) "unit" contributes, in order,
+//   * residual items: 5 fp16 residual tokens each (the new token included), and
+//   * packed items:   32 packed tokens each (one slice of one key group).
+// The items of all units are laid end to end and cut, by weight (packed 8,
+// residual 7: their measured costs), into one contiguous range per SM.  One
+// CTA of 16 warps runs on each SM.  Its warps claim the items of its range one
+// at a time from a shared-memory counter (so warps the scheduler favours simply
+// take more items, and all finish together) and stream them through per-warp
+// 3-stage cp.async pipelines (16 bytes per lane per copy, written to
+// bank-conflict-free positions).  Each warp keeps an online-softmax state per
+// query head.  At the end of each unit the 16 warps merge their states in
+// shared memory and the CTA writes one partial (m, l, sum p*v) per head; the
+// last CTA to arrive at a unit (self-resetting atomic counter) merges the
+// unit's partials into `out`, and when the residual ring is full it also packs
+// the oldest G residual tokens into a new key group.
 //
-// Slice math (per warp, 32 tokens = 2 m-tiles of 16, g <= 4 query heads):
-//   codes -> fp16 SUBNORMALS: one AND puts a 2-bit code at mantissa bit p in
-//     {4, 6, 8} of both halves of a 32-bit word, i.e. the value code * 2^(p-24)
-//     (mma.sync consumes fp16 subnormals exactly);
-//   scores  S[tok, col] = sum_c code_c 2^(p_c-24) b_c,   b_c = q_c s_c 2^(8-p_c)
-//     split hi + lo in fp16 (HMUL2 / HFMA2): columns 0..3 hold the hi parts of
-//     heads 0..3, columns 4..7 the lo parts; the accumulator starts at the
-//     zero-point term sum_c q_c z_c, itself one mma per 16 channels (A = the
-//     key-zero row broadcast to all 16 rows, B = q);
-//   output  O^T[ch, col] = sum_t code_{t,ch} 2^(p-24) P'[t, col],  P' = p_t * v_scale_t
-//     (hi/lo), moved from the score fragment layout into the B layout by
-//     movmatrix; out_ch = (O^T[ch,h] + O^T[ch,h+4]) 2^(24-p) + sum_t p_t v_zero_t.
-// A 16-token m-tile takes its tokens in the order perm8 so that both the
-// key-word and the value-word shared loads of a warp hit 32 distinct banks.
+// Packed-item math (per warp, 32 tokens = 2 m-tiles of 16, g <= 4 heads):
+//   codes -> fp16 SUBNORMALS: one AND puts a 2-bit code at mantissa bit p of
+//     both halves of a 32-bit word (value code * 2^(p-24); the tensor cores
+//     take fp16 subnormals exactly);
+//   scores S[tok, n] = sum_c code_c 2^(p_c-24) b_c over mma.sync.m16n8k16, with
+//     the 8 B columns interleaved per head: column 2h holds the fp16 "hi" part
+//     of q_h,c s_c 2^-p_c, column 2h+1 the exact remainder ("lo"), so the lane
+//     that owns head h holds both parts of its score (no shuffle) and every
+//     (token, head) probability is computed once;
+//   the key zero-point term sum_c q_c z_c is one mma per 16 channels (A = the
+//     zero row broadcast to all rows, B = q);
+//   output O^T[ch, n] = sum_t code_{t,ch} 2^(p-24) P'[t, n], P' = p_t v_scale_t
+//     split hi / lo the same way and moved into the B layout by movmatrix;
+//     out_ch = (O^T[ch, 2h] + O^T[ch, 2h+1]) 2^(24-p) + sum_t p_t v_zero_t.
+// Residual items use the fp16 rows directly: K through ldmatrix, V through
+// 128-bit loads arranged into the same accumulator layout as packed values.
 //
-// Attention-mass variant (decode_kernel<true>, minikv_decode_attn_mass): every
-// CTA also stores the absolute log2 score of each token it scores, per query
-// head, into a workspace array; the merging CTA of a unit stores the unit's
-// final (max, sum) per head; mass_kernel then adds
-// sum_h 2^(x_h,t - M_h) / L_h to the caller's running score of token t, the
-// H2O-style accumulated attention the MiniKV summary's experiments compare with.
+// Attention-mass variant (minikv_decode_attn_mass): every warp also stores the
+// absolute log2 score of each token it scores, per query head; the merging
+// CTA of a unit stores the unit's final (max, sum) per head; mass_kernel then
+// adds sum_h 2^(x_h,t - M_h) / L_h to the caller's running score of token t,
+// the H2O-style accumulated attention the MiniKV summary's experiments compare
+// with.
 #include <math.h>
+
+#include <mutex>
+#include <vector>
 
 #include "common.cuh"
 
@@ -47,37 +54,40 @@ namespace minikv {
 
 namespace {
 
-constexpr int kThreads = 128;
-constexpr int kSlice = 32;         // packed tokens per warp work item
-constexpr int kWarpStages = 4;
-constexpr int kResChunk = 64;      // residual tokens per residual CTA
-constexpr int kPartStride = 132;   // floats per (unit, slot, head): y[128], m, l
-constexpr int kMaxPackedCtas = 4096;
+constexpr int kWarps = 16;
+constexpr int kThreads = 32 * kWarps;
+constexpr int kSlice = 32;           // packed tokens per packed item
+constexpr int kResTok = 5;           // residual tokens per residual item
+constexpr int kStages = 3;           // per-warp pipeline depth
+constexpr int kStageBytes = 2688;    // one packed item (a residual item takes 2560)
+constexpr int kWP = 8, kWR = 7;      // partition weights of a packed / residual item (measured cost ratio)
+constexpr int kMinShare = 8 * kWP;   // least weight per CTA
+constexpr int kPartStride = 132;     // floats per (unit, slot, head): y[128], m, l
+constexpr int kMaxCtas = 512;
+constexpr float kLazy = 8.f;         // log2 headroom before a head's reference max moves
+constexpr int kWyStride = kD + 4;    // floats per (warp, head) row of the warp states
 
-struct __align__(16) SliceBuf {
-    uint32_t kc[kSlice * 8];   // key codes, token-major
-    uint32_t vc[kSlice * 8];   // value codes
-    uint16_t ks[kD];           // key scales of the slice's group
-    uint16_t kz[kD];           // key zeros of the slice's group
-    uint16_t vs[kSlice];       // value scales
-    uint16_t vz[kSlice];       // value zeros
+// packed stage: K codes [32 rows x 32 B] (rows permuted by kpos), V codes the
+// same, k_scale / k_zero 16 chunks each (permuted by schunk), v_scale, v_zero
+constexpr int kOffKc = 0, kOffVc = 1024, kOffKs = 2048, kOffKz = 2304, kOffVs = 2560, kOffVz = 2624;
+// residual stage: K rows [5][256 B] (chunks XOR-swizzled by row), V rows (chunks rotated by rvrot)
+constexpr int kOffRk = 0, kOffRv = kResTok * 256;
+static_assert(2 * kResTok * 256 <= kStageBytes, "residual item fits a stage");
+
+// One unit's share of a CTA's range ("segment").
+struct Seg {
+    int u, b, ub, items, nri, nq, r, rs, first, S_u, hi;
 };
-constexpr uint32_t kSliceBytes = sizeof(SliceBuf);
-static_assert(kSliceBytes == 2688, "slice buffer layout");
 
 struct __align__(16) Smem {
-    union {
-        SliceBuf st[4][kWarpStages];
-        struct {
-            uint16_t k[kResChunk * kD];   // XOR-swizzled rows (see swz)
-            uint16_t v[kResChunk * kD];
-        } res;
-    };
-    uint16_t qn[8][kD];      // query rows of the current unit (rows >= g are zero)
-    uint64_t full[4][kWarpStages];
-    float wm[4][4], wl[4][4];
-    float wy[4][4][kD];
+    unsigned char stage[kWarps][kStages][kStageBytes];
+    unsigned char qbuf[kWarps][kStages][4 * 256];   // query rows of a unit: [head][16 chunks], chunk c at c ^ head
+    float wm[kWarps][4], wl[kWarps][4];
+    float wy[kWarps][4][kWyStride];                 // per warp and head; padded: conflict-free 16-byte stores
+    uint4 zero;
     int flag;
+    int next;   // next item of the CTA's range to claim
+    Seg seg;    // the unit being processed
 };
 
 struct Args {
@@ -90,121 +100,171 @@ struct Args {
     uint16_t *out;
     float *part;
     unsigned *counters;
-    int *err;
     unsigned *grid_counter;   // device-state mode: CTAs of this launch that have finished (self-resetting)
     int *dseq;                // device-state mode: per-sequence state [B][4] in device memory
-    float *xs;          // mass variant: absolute log2 scores [unit][g][xs_stride]
-    float *stats;       // mass variant: per unit max[4], sum[4], token count (int bits), pad
+    float *xs;                // mass variant: absolute log2 scores [unit][g][xs_stride]
+    float *stats;             // mass variant: per unit max[4], sum[4], token count (int bits), pad
     int xs_stride;
     int Hkv, g, G, cap, ring;
-    int n_q, r, res_start, flush;
-    int units, n_rc, spu, P, S_max;   // schedule: slices per unit, packed CTAs, partial slots per unit
-    int groups_cap, lg2G;             // cap / G and log2(G)
-    int Ns;                           // total slices (< 2^31)
+    int n_q, r, res_start;    // uniform batch: every sequence's lengths (r counts the new token)
+    int units, P, S_max;      // CTAs that take a share, partial slots per unit
+    int groups_cap, lg2G;     // cap / G and log2(G)
     float scale_log2;
 };
 
-// Ragged batches: each sequence b has its own packed count, residual count (the
-// new token included) and ring origin.  The table travels as a kernel parameter
-// (__grid_constant__, read through the constant cache), so a step needs no
-// host-to-device copy.  sbeg[b] = first flat slice of sequence b's units.
+// Host-planned modes: the first flat item of each CTA's range (P + 1 entries).
+struct CtaTab {
+    int lo[kMaxCtas + 1];
+};
+
+// ---- per-unit item counts
+__host__ __device__ __forceinline__ int unit_nri(int r) { return (r + kResTok - 1) / kResTok; }
+__host__ __device__ __forceinline__ int unit_items(int nq, int r) { return unit_nri(r) + nq / kSlice; }
+__host__ __device__ __forceinline__ long long unit_w(int nq, int r) {
+    return (long long)unit_nri(r) * kWR + (long long)(nq / kSlice) * kWP;
+}
+
+// ---- sequence lengths and item prefix sums, by mode.  Uniform batches read the
+// shared scalars; ragged ones a kernel-parameter table; device-state ones a
+// table each CTA builds in shared memory from the device-resident state.
+struct ArgsUni : Args {
+    CtaTab cta;
+};
+__host__ __device__ __forceinline__ int nseq(const Args &a) { return a.units / a.Hkv; }
+__device__ __forceinline__ int s_nq(const ArgsUni &a, int) { return a.n_q; }
+__device__ __forceinline__ int s_r(const ArgsUni &a, int) { return a.r; }
+__device__ __forceinline__ int s_rs(const ArgsUni &a, int) { return a.res_start; }
+__device__ __forceinline__ int s_ibeg(const ArgsUni &a, int b) { return b * a.Hkv * unit_items(a.n_q, a.r); }
+__device__ __forceinline__ int seq_of_x(const ArgsUni &a, int x) { return x / (a.Hkv * unit_items(a.n_q, a.r)); }
+__device__ __forceinline__ int cta_lo(const ArgsUni &a, int c) { return a.cta.lo[c]; }
+__device__ __forceinline__ int part_P(const ArgsUni &a) { return a.P; }
+
 constexpr int kMaxRaggedSeqs = MINIKV_MAX_RAGGED_SEQS;
 struct SeqTab {
     int n_q[kMaxRaggedSeqs];
     int r[kMaxRaggedSeqs];
     int res_start[kMaxRaggedSeqs];
-    int sbeg[kMaxRaggedSeqs + 1];
+    int ibeg[kMaxRaggedSeqs + 1];   // first flat item of sequence b's units
 };
 struct ArgsVar : Args {
     SeqTab tab;
+    CtaTab cta;
 };
-
-// Per-unit lengths.  Uniform batches read the shared scalars; ragged ones the
-// table.  slice0 = the unit's first slice in the flat list of all units'
-// packed slices; unit_of = the unit holding flat slice x (x < Ns).
-__device__ __forceinline__ int len_nq(const Args &a, int) { return a.n_q; }
-__device__ __forceinline__ int len_r(const Args &a, int) { return a.r; }
-__device__ __forceinline__ int len_rs(const Args &a, int) { return a.res_start; }
-__device__ __forceinline__ int len_spu(const Args &a, int) { return a.spu; }
-__device__ __forceinline__ int seq_spu(const Args &a, int) { return a.spu; }
-__device__ __forceinline__ int slice0(const Args &a, int unit) { return unit * a.spu; }
-__device__ __forceinline__ int unit_of(const Args &a, int x) { return x / a.spu; }
-
-__device__ __forceinline__ int len_nq(const ArgsVar &a, int unit) { return a.tab.n_q[unit / a.Hkv]; }
-__device__ __forceinline__ int len_r(const ArgsVar &a, int unit) { return a.tab.r[unit / a.Hkv]; }
-__device__ __forceinline__ int len_rs(const ArgsVar &a, int unit) { return a.tab.res_start[unit / a.Hkv]; }
-__device__ __forceinline__ int len_spu(const ArgsVar &a, int unit) { return a.tab.n_q[unit / a.Hkv] / kSlice; }
-__device__ __forceinline__ int seq_spu(const ArgsVar &a, int b) { return a.tab.n_q[b] / kSlice; }
-__device__ __forceinline__ int slice0(const ArgsVar &a, int unit) {
-    const int b = unit / a.Hkv;
-    return a.tab.sbeg[b] + (unit - b * a.Hkv) * (a.tab.n_q[b] / kSlice);
-}
-__device__ __forceinline__ int unit_of(const ArgsVar &a, int x) {
-    // largest b with sbeg[b] <= x; since x < sbeg[B], sequence b has slices
-    int lo = 0, hi = a.units / a.Hkv;
+// largest b with beg(b) <= v (beg(0) = 0 <= v < beg(n))
+template <class F>
+__device__ __forceinline__ int seq_search(int n, int v, F beg) {
+    int lo = 0, hi = n;
     while (hi - lo > 1) {
         const int mid = (lo + hi) >> 1;
-        if (a.tab.sbeg[mid] <= x) lo = mid;
+        if (beg(mid) <= v) lo = mid;
         else hi = mid;
     }
-    return lo * a.Hkv + (x - a.tab.sbeg[lo]) / (a.tab.n_q[lo] / kSlice);
+    return lo;
 }
+__device__ __forceinline__ int s_nq(const ArgsVar &a, int b) { return a.tab.n_q[b]; }
+__device__ __forceinline__ int s_r(const ArgsVar &a, int b) { return a.tab.r[b]; }
+__device__ __forceinline__ int s_rs(const ArgsVar &a, int b) { return a.tab.res_start[b]; }
+__device__ __forceinline__ int s_ibeg(const ArgsVar &a, int b) { return a.tab.ibeg[b]; }
+__device__ __forceinline__ int seq_of_x(const ArgsVar &a, int x) {
+    return seq_search(nseq(a), x, [&](int b) { return a.tab.ibeg[b]; });
+}
+__device__ __forceinline__ int cta_lo(const ArgsVar &a, int c) { return a.cta.lo[c]; }
+__device__ __forceinline__ int part_P(const ArgsVar &a) { return a.P; }
 
-// Device-state mode: the per-sequence state lives in device memory (dseq), so
-// one launch configuration serves every step and the calls can be captured in
-// a CUDA graph.  Each CTA copies the state into shared memory behind Smem
-// (DevTab) before it starts; the partition of the packed slices over the
-// packed CTAs is then computed from it, on the device.
+// Device-state mode: the table sits behind Smem in dynamic shared memory:
+// DevTab, then n_q[B], r[B], res_start[B], ibeg[B + 1], cta_lo[P + 1] (int).
 struct ArgsDev : Args {};
-struct DevTab {   // followed by n_q[B], r[B], res_start[B], sbeg[B + 1]
-    int Ns, P;    // packed slices this step, packed CTAs that take a share
+struct DevTab {
+    long long Wt;
+    int P;
+    int pad;
 };
 __device__ __forceinline__ unsigned char *dyn_smem() {
     extern __shared__ __align__(128) unsigned char smem_raw[];
     return smem_raw;
 }
 __device__ __forceinline__ DevTab &dev_tab() { return *reinterpret_cast<DevTab *>(dyn_smem() + sizeof(Smem)); }
-__device__ __forceinline__ int *dev_arr(const ArgsDev &a, int k) {   // k = 0 n_q, 1 r, 2 res_start, 3 sbeg
-    return reinterpret_cast<int *>(dyn_smem() + sizeof(Smem) + sizeof(DevTab)) + k * (a.units / a.Hkv);
+__device__ __forceinline__ int *dev_arr(const Args &a, int k) {   // k = 0 n_q, 1 r, 2 res_start, 3 ibeg, 4 cta_lo
+    return reinterpret_cast<int *>(dyn_smem() + sizeof(Smem) + sizeof(DevTab)) + k * nseq(a) + (k > 3 ? 1 : 0);
 }
-__device__ __forceinline__ int len_nq(const ArgsDev &a, int unit) { return dev_arr(a, 0)[unit / a.Hkv]; }
-__device__ __forceinline__ int len_r(const ArgsDev &a, int unit) { return dev_arr(a, 1)[unit / a.Hkv]; }
-__device__ __forceinline__ int len_rs(const ArgsDev &a, int unit) { return dev_arr(a, 2)[unit / a.Hkv]; }
-__device__ __forceinline__ int len_spu(const ArgsDev &a, int unit) { return dev_arr(a, 0)[unit / a.Hkv] / kSlice; }
-__device__ __forceinline__ int seq_spu(const ArgsDev &a, int b) { return dev_arr(a, 0)[b] / kSlice; }
-__device__ __forceinline__ int slice0(const ArgsDev &a, int unit) {
-    const int b = unit / a.Hkv;
-    return dev_arr(a, 3)[b] + (unit - b * a.Hkv) * (dev_arr(a, 0)[b] / kSlice);
+__device__ __forceinline__ int s_nq(const ArgsDev &a, int b) { return dev_arr(a, 0)[b]; }
+__device__ __forceinline__ int s_r(const ArgsDev &a, int b) { return dev_arr(a, 1)[b]; }
+__device__ __forceinline__ int s_rs(const ArgsDev &a, int b) { return dev_arr(a, 2)[b]; }
+__device__ __forceinline__ int s_ibeg(const ArgsDev &a, int b) { return dev_arr(a, 3)[b]; }
+__device__ __forceinline__ int seq_of_x(const ArgsDev &a, int x) {
+    const int *ib = dev_arr(a, 3);
+    return seq_search(nseq(a), x, [&](int b) { return ib[b]; });
 }
-__device__ __forceinline__ int unit_of(const ArgsDev &a, int x) {
-    const int *sbeg = dev_arr(a, 3);
-    int lo = 0, hi = a.units / a.Hkv;
-    while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if (sbeg[mid] <= x) lo = mid;
-        else hi = mid;
-    }
-    return lo * a.Hkv + (x - sbeg[lo]) / (dev_arr(a, 0)[lo] / kSlice);
-}
-
-// the partition of packed slices over packed CTAs (host-planned, or this step's on the device)
-__device__ __forceinline__ int part_Ns(const Args &a) { return a.Ns; }
-__device__ __forceinline__ int part_P(const Args &a) { return a.P; }
-__device__ __forceinline__ int part_Ns(const ArgsDev &) { return dev_tab().Ns; }
+__device__ __forceinline__ int cta_lo(const ArgsDev &a, int c) { return dev_arr(a, 4)[c]; }
 __device__ __forceinline__ int part_P(const ArgsDev &) { return dev_tab().P; }
 
-// column of element `col` of query row h in the swizzled sm.qn rows
-__device__ __forceinline__ int qn_col(int h, int col) { return (((col >> 3) ^ h) << 3) | (col & 7); }
+// ---- positions in the work list
 
-// token order inside an 8-row half of an m-tile: {0,2,1,3,6,4,7,5}
-__device__ __forceinline__ int perm8(int r) { return (0x57461320u >> (4 * r)) & 0xf; }
+// the CTA whose item range holds flat item x: largest c with cta_lo(c) <= x
+template <class A>
+__device__ __forceinline__ int cta_of_item(const A &a, int x) {
+    return seq_search(part_P(a), x, [&](int c) { return cta_lo(a, c); });
+}
+
+// Segment info for the unit holding flat item x (one thread).
+template <class A>
+__device__ void seg_info(const A &a, int x, int xhi, Seg &s) {
+    const int b = seq_of_x(a, x);
+    const int nq = s_nq(a, b), r = s_r(a, b);
+    const int items = unit_items(nq, r);
+    const int kh = (x - s_ibeg(a, b)) / items;
+    s.u = b * a.Hkv + kh;
+    s.b = b;
+    s.ub = s_ibeg(a, b) + kh * items;
+    s.items = items;
+    s.nri = unit_nri(r);
+    s.nq = nq;
+    s.r = r;
+    s.rs = s_rs(a, b);
+    s.hi = min(xhi, s.ub + items);
+    // CTAs that write a partial for the unit: those whose ranges hold its items
+    s.first = cta_of_item(a, s.ub);
+    s.S_u = cta_of_item(a, s.ub + items - 1) - s.first + 1;
+}
+
+// A warp's place in the work list: unit u (= b Hkv + kh), item k of the unit,
+// ub = flat index of the unit's first item.  Moving forward needs no division.
+struct Cursor {
+    int x, u, b, kh, k, ub, items;
+    template <class A>
+    __device__ __forceinline__ void set(const A &a, int x_) {
+        x = x_;
+        b = seq_of_x(a, x);
+        items = unit_items(s_nq(a, b), s_r(a, b));
+        kh = (x - s_ibeg(a, b)) / items;
+        u = b * a.Hkv + kh;
+        ub = s_ibeg(a, b) + kh * items;
+        k = x - ub;
+    }
+    template <class A>
+    __device__ __forceinline__ void advance_to(const A &a, int x_) {
+        k += x_ - x;
+        x = x_;
+        while (k >= items) {
+            k -= items;
+            ub += items;
+            ++u;
+            if (++kh == a.Hkv) {
+                kh = 0;
+                ++b;
+                items = unit_items(s_nq(a, b), s_r(a, b));
+            }
+        }
+    }
+};
+
+// ---- small device helpers
 
 __device__ __forceinline__ float ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
     return y;
 }
-
 __device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
     uint32_t d;
     asm("mul.rn.f16x2 %0, %1, %2;\n" : "=r"(d) : "r"(a), "r"(b));
@@ -215,8 +275,7 @@ __device__ __forceinline__ uint32_t hfma2(uint32_t a, uint32_t b, uint32_t c) {
     asm("fma.rn.f16x2 %0, %1, %2, %3;\n" : "=r"(d) : "r"(a), "r"(b), "r"(c));
     return d;
 }
-
-__device__ __forceinline__ float warp_sum_g(float x) {   // over lanes with equal t (xor 4, 8, 16)
+__device__ __forceinline__ float warp_sum_g(float x) {   // over the lanes of one head (xor 4, 8, 16)
     x += __shfl_xor_sync(0xffffffffu, x, 4);
     x += __shfl_xor_sync(0xffffffffu, x, 8);
     x += __shfl_xor_sync(0xffffffffu, x, 16);
@@ -228,648 +287,639 @@ __device__ __forceinline__ float warp_max_g(float x) {
     x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 16));
     return x;
 }
-
-// word << 4 and word >> 6 as integer multiplies (IMAD / IMAD.HI), which issue
-// on the FMA pipe and leave the busier integer ALU to the masks
-__device__ __forceinline__ uint32_t shl4(uint32_t x) {
+// word >> 10 as an integer multiply-high (IMAD.HI), which issues on the FMA
+// pipe and leaves the busier integer ALU to the masks
+__device__ __forceinline__ uint32_t shr10(uint32_t x) {
     uint32_t y;
-    asm("mul.lo.u32 %0, %1, 16;\n" : "=r"(y) : "r"(x));
+    asm("mul.hi.u32 %0, %1, 4194304;\n" : "=r"(y) : "r"(x));
     return y;
 }
-__device__ __forceinline__ uint32_t shr6(uint32_t x) {
-    uint32_t y;
-    asm("mul.hi.u32 %0, %1, 67108864;\n" : "=r"(y) : "r"(x));
-    return y;
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];\n" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+    return v;
+}
+__device__ __forceinline__ uint2 lds64(uint32_t addr) {
+    uint2 v;
+    asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];\n" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+    return v;
+}
+__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];\n" : "=r"(v) : "r"(addr));
+    return v;
+}
+__device__ __forceinline__ uint32_t w4(const uint4 &v, int i) { return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w; }
+// D (16x8 fp32) += A (16x8 fp16, row) * B (8x8 fp16, col):
+//   a0 = {(g,2t),(g,2t+1)}, a1 = {(g+8,2t),(g+8,2t+1)}, b = {(2t,g),(2t+1,g)}; D as for m16n8k16
+__device__ __forceinline__ void mma1688(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t b) {
+    asm volatile("mma.sync.aligned.m16n8k8.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5}, {%6}, {%0,%1,%2,%3};\n"
+                 : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+                 : "r"(a0), "r"(a1), "r"(b));
+}
+// arrival on a unit / launch counter: release of this CTA's writes (ordered
+// before by a block barrier) and acquire of the earlier arrivals' writes
+__device__ __forceinline__ unsigned atom_inc_acq_rel(unsigned *p, unsigned lim) {
+    unsigned old;
+    asm volatile("atom.acq_rel.gpu.global.inc.u32 %0, [%1], %2;\n" : "=r"(old) : "l"(p), "r"(lim) : "memory");
+    return old;
 }
 
 // Code pair i (i = 0..7) of a 32-bit word of 16 codes -> fp16x2 subnormals
-// (code_i, code_{i+8}) at mantissa bit p_i: i -> p = 4,6,4,6,8,4,6,8.
-// x = word, x1 = word >> 6, x2 = word << 4.
-constexpr uint32_t kM4 = 0x00300030u, kM6 = 0x00C000C0u, kM8 = 0x03000300u;
+// (code_i, code_{i+8}) at mantissa bit pair_pos(i): pairs 0..4 are masked
+// straight out of the word (bits 0, 2, .., 8 of each half), pairs 5..7 out of
+// word >> 10 (bits 0, 2, 4).  x = word, y = word >> 10.
 template <int I>
-__device__ __forceinline__ uint32_t code_pair(uint32_t x, uint32_t x1, uint32_t x2) {
-    if constexpr (I == 0) return x2 & kM4;
-    else if constexpr (I == 1) return x2 & kM6;
-    else if constexpr (I == 2) return x & kM4;
-    else if constexpr (I == 3) return x & kM6;
-    else if constexpr (I == 4) return x & kM8;
-    else if constexpr (I == 5) return x1 & kM4;
-    else if constexpr (I == 6) return x1 & kM6;
-    else return x1 & kM8;
+__device__ __forceinline__ uint32_t code_pair(uint32_t x, uint32_t y) {
+    if constexpr (I < 5) return x & (0x00030003u << (2 * I));
+    else return y & (0x00030003u << (2 * (I - 5)));
 }
-// 2^(8 - p_i) and 2^(24 - p_i)
-__host__ __device__ constexpr float pair_wq(int i) {
-    return (i == 4 || i == 7) ? 1.f : ((i == 1 || i == 3 || i == 6) ? 4.f : 16.f);
-}
-__host__ __device__ constexpr float pair_wo(int i) { return pair_wq(i) * 65536.f; }
+__host__ __device__ constexpr int pair_pos(int i) { return i < 5 ? 2 * i : 2 * (i - 5); }
+// 2^-pos (key B operand: q s 2^-pos stays below the fp16 limit whenever q s
+// does) and 2^(24 - pos) (value output scale)
+__host__ __device__ constexpr float pair_wq(int i) { return 1.f / (float)(1 << pair_pos(i)); }
+__host__ __device__ constexpr float pair_wo(int i) { return (float)(1 << (24 - pair_pos(i))); }
+constexpr float kScoreUnit = 16777216.f;   // packed scores come out as code q s 2^-24
+
+// row of packed token j (0..31) in a stage's code block: tokens 2m of a
+// 16-token tile (and 2m+1) land in distinct bank groups, and so do tokens 4t+o
+__host__ __device__ __forceinline__ int kpos(int j) { return 4 * (j >> 2) + ((j + (j >> 2)) & 3); }
+// position of 8-channel chunk k (0..15) of the key scale / zero rows
+__host__ __device__ __forceinline__ int schunk(int k) { return k ^ ((k & 8) >> 2); }
+// rotation of the 16-byte chunks of residual V row j
+__host__ __device__ __forceinline__ int rvrot(int j) { return ((j >> 1) & 1) + 4 * ((j >> 2) & 1); }
 
 // ---------------------------------------------------------------- partials
 
-// Write this CTA's partial state for `unit` into slot `slot`, then let the
-// last arriving CTA of the unit (S_u arrivals) merge all slots into `out`.
+// The CTA's 16 warp states for the segment's unit (already scaled to the CTA's
+// per-head max and written to sm.wy / wl / wm) are summed into one partial in
+// slot `slot`; the last CTA of the unit to arrive (S_u arrivals) merges the
+// partials into `out` and, if the residual ring is full, packs its oldest G
+// tokens into key group n_q/G.  A unit within one CTA is written out directly.
+// Thread tid handles head tid / 128, channel tid % 128.
 template <bool kMass, class A>
-__device__ void finish_unit(const A &a, Smem &sm, int unit, int slot, int S_u, const float *m_h,
-                            const float *l_h, const float (*y_h)[kD]) {
-    const int tid = threadIdx.x;
-    float *base = a.part + ((size_t)unit * a.S_max + slot) * 4 * kPartStride;
-    for (int h = 0; h < a.g; ++h) {
-        base[h * kPartStride + tid] = y_h[h][tid];
-        if (tid == 0) {
-            base[h * kPartStride + 128] = m_h[h];
-            base[h * kPartStride + 129] = l_h[h];
-        }
-    }
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) sm.flag = (atomicInc(&a.counters[unit], (unsigned)(S_u - 1)) == (unsigned)(S_u - 1));
-    __syncthreads();
-    if (!sm.flag) return;
-    __threadfence();
-    const float *ub = a.part + (size_t)unit * a.S_max * 4 * kPartStride;
-    const int b = unit / a.Hkv, kvh = unit % a.Hkv;
+__device__ void finish_unit(const A &a, Smem &sm, const Seg &s, int slot) {
+    const int tid = threadIdx.x, h = tid >> 7, ch = tid & 127;
+    const int unit = s.u;
+    const int b = s.b, kvh = unit - s.b * a.Hkv;
     const int Hq = a.Hkv * a.g;
-    // one pass over the unit's partials, all heads together, four slots per
-    // round with every load of the round issued before any is used (online
-    // rescaling: the running max moves to the larger of the two)
-    float M[4], L[4], Y[4];
+    __syncthreads();   // warp states written
+    float M = -INFINITY, L = 0.f, Y = 0.f;
 #pragma unroll
-    for (int h = 0; h < 4; ++h) {
-        M[h] = -INFINITY;
-        L[h] = 0.f;
-        Y[h] = 0.f;
+    for (int w = 0; w < kWarps; ++w) {
+        M = fmaxf(M, sm.wm[w][h]);
+        L += sm.wl[w][h];
+        Y += sm.wy[w][h][ch];
     }
-    for (int s0 = 0; s0 < S_u; s0 += 4) {
-        float ms[4][4], ls[4][4], ys[4][4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-#pragma unroll
-            for (int h = 0; h < 4; ++h) {
-                const bool ok = (s0 + j < S_u) && (h < a.g);
-                const float *p = ub + ((s0 + j) * 4 + h) * kPartStride;
-                ms[j][h] = ok ? __ldcg(p + 128) : -INFINITY;
-                ls[j][h] = ok ? __ldcg(p + 129) : 0.f;
-                ys[j][h] = ok ? __ldcg(p + tid) : 0.f;
-            }
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-#pragma unroll
-            for (int h = 0; h < 4; ++h) {
-                const float m = ms[j][h], Mn = fmaxf(M[h], m);
-                const float fo = (M[h] == -INFINITY) ? 0.f : ex2(M[h] - Mn);
-                const float fs = (m == -INFINITY) ? 0.f : ex2(m - Mn);
-                L[h] = fmaf(L[h], fo, ls[j][h] * fs);
-                Y[h] = fmaf(Y[h], fo, ys[j][h] * fs);
-                M[h] = Mn;
-            }
-    }
-#pragma unroll
-    for (int h = 0; h < 4; ++h)
+    if (s.S_u > 1) {
+        float *base = a.part + ((size_t)unit * a.S_max + slot) * 4 * kPartStride + h * kPartStride;
         if (h < a.g) {
-            a.out[((size_t)b * Hq + kvh * a.g + h) * kD + tid] = f2h(__fdividef(Y[h], L[h]));
-            if (kMass && tid == 0) {
-                a.stats[unit * 12 + h] = M[h];
-                a.stats[unit * 12 + 4 + h] = L[h];
+            base[ch] = Y;
+            if (ch == 0) {
+                base[128] = M;
+                base[129] = L;
             }
-        }
-    if (kMass && tid == 0) a.stats[unit * 12 + 8] = __int_as_float(len_nq(a, unit) + len_r(a, unit));
-}
-
-// Merge the four warps' states (sm.wm / wl / wy) and hand the CTA partial on.
-template <bool kMass, class A>
-__device__ void merge_warps_and_finish(const A &a, Smem &sm, int unit, int slot, int S_u) {
-    const int tid = threadIdx.x;
-    __syncthreads();
-    float mh[4], lh[4], yh[4];
-#pragma unroll
-    for (int h = 0; h < 4; ++h) {
-        const float M = fmaxf(fmaxf(sm.wm[0][h], sm.wm[1][h]), fmaxf(sm.wm[2][h], sm.wm[3][h]));
-        float L = 0.f, Y = 0.f;
-#pragma unroll
-        for (int w = 0; w < 4; ++w) {
-            const float f = (sm.wm[w][h] == -INFINITY) ? 0.f : ex2(sm.wm[w][h] - M);
-            L += f * sm.wl[w][h];
-            Y += f * sm.wy[w][h][tid];
-        }
-        mh[h] = M;
-        lh[h] = L;
-        yh[h] = Y;
-    }
-    __syncthreads();
-#pragma unroll
-    for (int h = 0; h < 4; ++h) sm.wy[0][h][tid] = yh[h];
-    finish_unit<kMass>(a, sm, unit, slot, S_u, mh, lh, sm.wy[0]);
-}
-
-// packed CTA c covers slices [c*Ns/P, (c+1)*Ns/P); the CTA holding slice x
-__device__ __forceinline__ int cta_of_slice(long long x, int P, int Ns) {
-    return (int)(((x + 1) * P - 1) / Ns);
-}
-template <class A>
-__device__ __forceinline__ void unit_slots(const A &a, int unit, int &first, int &S_u) {
-    const int spu = len_spu(a, unit);
-    if (spu == 0) {
-        first = 0;
-        S_u = a.n_rc;
-        return;
-    }
-    const int s0 = slice0(a, unit);
-    first = cta_of_slice(s0, part_P(a), part_Ns(a));
-    const int last = cta_of_slice((long long)s0 + spu - 1, part_P(a), part_Ns(a));
-    S_u = a.n_rc + last - first + 1;
-}
-
-// ------------------------------------------------------------- residual CTAs
-
-// Residual chunk rc of a unit: logical residual tokens [64 rc, 64 rc + 64) in
-// fp16; warp w takes 16 of them as one m-tile.  Scores use q (exact in fp16)
-// as the B operand; outputs the same hi/lo P as the packed path.
-template <bool kMass, class A>
-__device__ void residual_chunk_cta(const A &a, Smem &sm, int unit, int rc) {
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int g_ = lane >> 2, t_ = lane & 3;
-    const int b = unit / a.Hkv, kvh = unit % a.Hkv;
-    const int Hq = a.Hkv * a.g;
-    const uint16_t *knew = a.k_new + (size_t)unit * kD;
-    const uint16_t *vnew = a.v_new + (size_t)unit * kD;
-    uint16_t *kres = a.k_res + (size_t)unit * a.ring * kD;
-    uint16_t *vres = a.v_res + (size_t)unit * a.ring * kD;
-    const int r = len_r(a, unit), res_start = len_rs(a, unit), n_q = len_nq(a, unit);
-    const int i0 = rc * kResChunk;
-    const int n = min(kResChunk, r - i0);
-    auto slot = [&](int i) { int s = res_start + i; return s >= a.ring ? s - a.ring : s; };
-    auto krow = [&](int i, int c) -> const uint16_t * { return (i == r - 1 ? knew : kres + (size_t)slot(i) * kD) + c; };
-    auto vrow = [&](int i, int c) -> const uint16_t * { return (i == r - 1 ? vnew : vres + (size_t)slot(i) * kD) + c; };
-
-    {
-        const int ch = tid & 15;
-        int s0 = res_start + i0 + (tid >> 4);
-        if (s0 >= a.ring) s0 -= a.ring;
-#pragma unroll 2
-        for (int row = tid >> 4; row < kResChunk; row += 8) {
-            const bool ok = row < n;
-            const bool newest = i0 + row == r - 1;
-            const uint16_t *ks = newest ? knew : kres + (size_t)s0 * kD;
-            const uint16_t *vs = newest ? vnew : vres + (size_t)s0 * kD;
-            const uint32_t so = (uint32_t)swz(row, ch * 8) * 2u;
-            cp_async16(smem_addr(sm.res.k) + so, (ok ? ks : kres) + ch * 8, ok);
-            cp_async16(smem_addr(sm.res.v) + so, (ok ? vs : vres) + ch * 8, ok);
-            s0 += 8;
-            if (s0 >= a.ring) s0 -= a.ring;
-        }
-    }
-    cp_async_commit();
-    if (i0 <= r - 1 && r - 1 < i0 + n) {   // append the new token to the ring
-        if (tid < 16)
-            reinterpret_cast<uint4 *>(kres + (size_t)slot(r - 1) * kD)[tid] = reinterpret_cast<const uint4 *>(knew)[tid];
-        else if (tid < 32)
-            reinterpret_cast<uint4 *>(vres + (size_t)slot(r - 1) * kD)[tid - 16] =
-                reinterpret_cast<const uint4 *>(vnew)[tid - 16];
-    }
-    // B operand: column g_ < 4 is query head g_ (channels in natural order), columns 4..7 are 0
-    uint32_t bq[8][2];
-    {
-        const int hq = g_ & 3;
-        const bool live = (g_ < 4) && (hq < a.g);
-        const uint32_t *qp =
-            reinterpret_cast<const uint32_t *>(a.q + ((size_t)b * Hq + kvh * a.g + (live ? hq : 0)) * kD);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-            bq[kk][0] = live ? qp[8 * kk + t_] : 0u;
-            bq[kk][1] = live ? qp[8 * kk + t_ + 4] : 0u;
-        }
-    }
-    cp_async_wait<0>();
-    __syncthreads();
-
-    const int hA = 2 * (t_ & 1);
-    float m_w[2] = {-INFINITY, -INFINITY}, l_w[2] = {0.f, 0.f};
-    float acc[8][4];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
-    if (16 * warp < n) {
-        float s[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-            uint32_t kf[4];
-            ldmatrix_x4(kf, smem_addr(sm.res.k + swz(16 * warp + (lane & 7) + 8 * ((lane >> 3) & 1),
-                                                      16 * kk + 8 * (lane >> 4))));
-            mma16816(s, kf, bq[kk][0], bq[kk][1]);
-        }
-        float x[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const float v = s[i] + __shfl_xor_sync(0xffffffffu, s[i], 2);
-            const int row = 16 * warp + g_ + 8 * (i >> 1);
-            x[i] = row < n ? v * a.scale_log2 : -INFINITY;
-            if (kMass) {   // lanes t_ < 2 hold head hA + (i & 1) of token `row`
-                const int h = hA + (i & 1);
-                if (t_ < 2 && h < a.g && row < n)
-                    a.xs[((size_t)unit * a.g + h) * a.xs_stride + n_q + i0 + row] = x[i];
-            }
-        }
-#pragma unroll
-        for (int e = 0; e < 2; ++e) m_w[e] = warp_max_g(fmaxf(x[e], x[e + 2]));
-        uint32_t prow[2];
-#pragma unroll
-        for (int hr = 0; hr < 2; ++hr) {
-            const float p0 = ex2(x[2 * hr] - m_w[0]), p1 = ex2(x[2 * hr + 1] - m_w[1]);
-            l_w[0] += p0;
-            l_w[1] += p1;
-            const uint32_t hv = pack_half2(p0, p1);
-            const float2 f = unpack_half2(hv);
-            const uint32_t lv = pack_half2(p0 - f.x, p1 - f.y);
-            prow[hr] = (t_ >= 2) ? lv : hv;
-        }
-        const uint32_t bv0 = movmatrix_t(prow[0]), bv1 = movmatrix_t(prow[1]);
-#pragma unroll
-        for (int nu = 0; nu < 8; ++nu) {
-            uint32_t va[4];
-            ldmatrix_x4_t(va, smem_addr(sm.res.v + swz(16 * warp + (lane & 7) + 8 * (lane >> 4),
-                                                        16 * nu + 8 * ((lane >> 3) & 1))));
-            mma16816(acc[nu], va, bv0, bv1);
-        }
-    }
-#pragma unroll
-    for (int e = 0; e < 2; ++e) l_w[e] = warp_sum_g(l_w[e]);
-#pragma unroll
-    for (int nu = 0; nu < 8; ++nu)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) acc[nu][i] += __shfl_xor_sync(0xffffffffu, acc[nu][i], 2);
-    if (t_ < 2) {
-#pragma unroll
-        for (int nu = 0; nu < 8; ++nu) {
-            const int ch = 16 * nu + g_;
-            sm.wy[warp][hA][ch] = acc[nu][0];
-            sm.wy[warp][hA + 1][ch] = acc[nu][1];
-            sm.wy[warp][hA][ch + 8] = acc[nu][2];
-            sm.wy[warp][hA + 1][ch + 8] = acc[nu][3];
-        }
-        if (g_ == 0) {
-            sm.wm[warp][hA] = m_w[0];
-            sm.wm[warp][hA + 1] = m_w[1];
-            sm.wl[warp][hA] = l_w[0];
-            sm.wl[warp][hA + 1] = l_w[1];
-        }
-    }
-    if (r == a.ring && n_q + a.G <= a.cap && rc == 0) {
-        // the oldest G residual tokens become key group n_q/G and G value tokens
-        const size_t tok0 = (size_t)unit * a.cap + n_q;
-        const size_t grow = (size_t)unit * (a.cap / a.G) + n_q / a.G;
-        float *scr = reinterpret_cast<float *>(&sm.qn[0][0]);   // unused by residual CTAs otherwise
-        if (a.G <= kResChunk) {   // the group is in this CTA's shared tile (logical rows 0..63)
-            __syncthreads();
-            auto kat = [&](int i, int c) -> const uint16_t * { return sm.res.k + swz(i, c); };
-            auto vat = [&](int i, int c) -> const uint16_t * { return sm.res.v + swz(i, c); };
-            pack_key_group(kat, a.G, a.k_codes_w + tok0 * 8, a.k_scale_w + grow * kD, a.k_zero_w + grow * kD, scr);
-            pack_value_tokens(vat, a.G, kD, a.v_codes_w + tok0 * 8, a.v_scale_w + tok0, a.v_zero_w + tok0);
-        } else {
-            pack_key_group(krow, a.G, a.k_codes_w + tok0 * 8, a.k_scale_w + grow * kD, a.k_zero_w + grow * kD, scr);
-            pack_value_tokens(vrow, a.G, kD, a.v_codes_w + tok0 * 8, a.v_scale_w + tok0, a.v_zero_w + tok0);
-        }
-    }
-    int first, S_u;
-    unit_slots(a, unit, first, S_u);
-    merge_warps_and_finish<kMass>(a, sm, unit, rc, S_u);
-}
-
-// ------------------------------------------------------------------ packed CTA
-
-// Queue the bulk copies of the slice at (unit u, slice j) into this warp's
-// stage.  Called by one lane; no division: G is a power of two.
-template <class A>
-__device__ __forceinline__ void issue_slice(const A &a, Smem &sm, int warp, int stage, int u, int j) {
-    SliceBuf &S = sm.st[warp][stage];
-    uint64_t *bar = &sm.full[warp][stage];
-    const int t0 = j * kSlice;
-    const size_t tok = (size_t)u * a.cap + t0;
-    const size_t grow = (size_t)u * a.groups_cap + (t0 >> a.lg2G);
-    mbar_arrive_expect_tx(bar, kSliceBytes);
-    bulk_g2s(S.kc, a.k_codes + tok * 8, kSlice * 32, bar);
-    bulk_g2s(S.vc, a.v_codes + tok * 8, kSlice * 32, bar);
-    bulk_g2s(S.ks, a.k_scale + grow * kD, kD * 2, bar);
-    bulk_g2s(S.kz, a.k_zero + grow * kD, kD * 2, bar);
-    bulk_g2s(S.vs, a.v_scale + tok, kSlice * 2, bar);
-    bulk_g2s(S.vz, a.v_zero + tok, kSlice * 2, bar);
-}
-
-// A warp's position in the flat slice list, kept as (unit, its sequence b, its
-// KV head kh, slice in unit j) so that stepping needs no division.
-struct Cursor {
-    int u, b, kh, j;
-    template <class A>
-    __device__ __forceinline__ void step(const A &a, int n) {
-        j += n;
-        int spu = seq_spu(a, b);
-        while (j >= spu && u < a.units - 1) {
-            j -= spu;
-            ++u;
-            if (++kh == a.Hkv) {
-                kh = 0;
-                spu = seq_spu(a, ++b);
-            }
-        }
-    }
-};
-
-// q * 2^(8-p) for the key B operand of this lane: head g_ & 3, the channel
-// pair of chunk KK, slot SIG (see code_pair)
-template <int KK, int SIG>
-__device__ __forceinline__ uint32_t qw_pair(const uint16_t *qh, int t_) {
-    constexpr int i = 2 * (KK & 3) + SIG;
-    const int c = 16 * (2 * t_ + (KK >> 2)) + i;
-    constexpr float w = pair_wq(i);
-    return pack_half2(h2f(qh[c]) * w, h2f(qh[c + 8]) * w);
-}
-
-// packed fp32 pairs (two lanes of work per instruction)
-template <bool kMass, class A>
-__device__ void packed_cta(const A &a, Smem &sm, int c) {
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int g_ = lane >> 2, t_ = lane & 3;
-    const int Hq = a.Hkv * a.g;
-    const int Ns = part_Ns(a), P = part_P(a);
-    if (c >= P) return;   // no share this step (device-state mode plans for the largest step)
-    const int cs = (int)((long long)c * Ns / P), ce = (int)((long long)(c + 1) * Ns / P);
-
-    if (tid == 0) {
-        for (int w = 0; w < 4; ++w)
-            for (int s = 0; s < kWarpStages; ++s) mbar_init(&sm.full[w][s], 1);
-        fence_mbar_init();
-    }
-    __syncthreads();
-    // this warp's slices: cs + warp + 4k; `nxt` is the next one to queue
-    Cursor nxt{0, 0, 0, 0};
-    int nxt_x = cs + warp;
-    if (nxt_x < ce) {
-        nxt.u = unit_of(a, nxt_x);
-        nxt.b = nxt.u / a.Hkv;
-        nxt.kh = nxt.u - nxt.b * a.Hkv;
-        nxt.j = nxt_x - slice0(a, nxt.u);
-    }
-    if (lane == 0)
-        for (int k = 0; k < kWarpStages && nxt_x < ce; ++k) {
-            issue_slice(a, sm, warp, k, nxt.u, nxt.j);
-            nxt.step(a, 4);
-            nxt_x += 4;
-        }
-
-    const int hA = 2 * (t_ & 1);
-    const int pg = perm8(g_);
-    const int p2t = perm8(2 * t_), p2t1 = perm8(2 * t_ + 1);
-    const uint32_t lo_neg = (g_ >= 4) ? 0xBC00BC00u : 0u;   // fp16x2 (-1, -1) on lo columns, (0, 0) on hi
-    const bool lo_row = t_ >= 2;
-    int k = 0;   // this warp's slice counter over the whole range
-    bool ok = true;
-
-    int seg = cs;
-    while (seg < ce) {
-        const int unit = unit_of(a, seg);
-        const int u_s0 = slice0(a, unit);
-        const int seg_end = min(ce, u_s0 + len_spu(a, unit));
-        const int b = unit / a.Hkv, kvh = unit % a.Hkv;
-        const uint16_t *qbase = a.q + ((size_t)b * Hq + kvh * a.g) * kD;
-        // query rows of this unit for the zero-point mma (rows >= g zero), 16-byte
-        // chunks XOR-swizzled by row so the ldmatrix of 8 rows is conflict-free
-        for (int e = tid; e < 8 * 16; e += kThreads) {
-            const int h = e / 16, ch = e % 16;
-            uint4 v = make_uint4(0, 0, 0, 0);
-            if (h < a.g) v = reinterpret_cast<const uint4 *>(qbase + (size_t)h * kD)[ch];
-            *reinterpret_cast<uint4 *>(&sm.qn[h][qn_col(h, 8 * ch)]) = v;
-        }
-        uint32_t qw[8][2];
-        {
-            const int hq = g_ & 3;
-            const bool live = hq < a.g;
-            const uint16_t *qh = qbase + (size_t)(live ? hq : 0) * kD;
-#define QW(KK)                                      \
-    qw[KK][0] = live ? qw_pair<KK, 0>(qh, t_) : 0u; \
-    qw[KK][1] = live ? qw_pair<KK, 1>(qh, t_) : 0u;
-            QW(0) QW(1) QW(2) QW(3) QW(4) QW(5) QW(6) QW(7)
-#undef QW
         }
         __syncthreads();
+        if (tid == 0) sm.flag = (atom_inc_acq_rel(&a.counters[unit], (unsigned)(s.S_u - 1)) == (unsigned)(s.S_u - 1));
+        __syncthreads();
+        if (!sm.flag) return;
+        // merge the unit's partials: eight slots per round, every load of a
+        // round issued before any is used (online rescaling)
+        const float *ub = a.part + (size_t)unit * a.S_max * 4 * kPartStride + h * kPartStride;
+        M = -INFINITY;
+        L = 0.f;
+        Y = 0.f;
+        if (h < a.g)
+            for (int s0 = 0; s0 < s.S_u; s0 += 8) {
+                float ms[8], ls[8], ys[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const bool ok = s0 + j < s.S_u;
+                    const float *p = ub + (size_t)(s0 + j) * 4 * kPartStride;
+                    ms[j] = ok ? __ldcg(p + 128) : -INFINITY;
+                    ls[j] = ok ? __ldcg(p + 129) : 0.f;
+                    ys[j] = ok ? __ldcg(p + ch) : 0.f;
+                }
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const float m = ms[j], Mn = fmaxf(M, m);
+                    const float fo = (M == -INFINITY) ? 0.f : ex2(M - Mn);
+                    const float fs = (m == -INFINITY) ? 0.f : ex2(m - Mn);
+                    L = fmaf(L, fo, ls[j] * fs);
+                    Y = fmaf(Y, fo, ys[j] * fs);
+                    M = Mn;
+                }
+            }
+    }
+    if (h < a.g) {
+        a.out[((size_t)b * Hq + kvh * a.g + h) * kD + ch] = f2h(__fdividef(Y, L));
+        if (kMass && ch == 0) {
+            a.stats[unit * 12 + h] = M;
+            a.stats[unit * 12 + 4 + h] = L;
+        }
+    }
+    if (kMass && tid == 0) a.stats[unit * 12 + 8] = __int_as_float(s.nq + s.r);
+    if (s.r == a.ring && s.nq + a.G <= a.cap) {
+        // flush: the oldest G residual tokens (all in the ring: the new token was
+        // appended before its CTA arrived) become key group nq/G and G value tokens
+        const uint16_t *kres = a.k_res + (size_t)unit * a.ring * kD;
+        const uint16_t *vres = a.v_res + (size_t)unit * a.ring * kD;
+        const int rs = s.rs;
+        auto slot_of = [&](int i) { const int t = rs + i; return t >= a.ring ? t - a.ring : t; };
+        auto krow = [&](int i, int c) -> const uint16_t * { return kres + (size_t)slot_of(i) * kD + c; };
+        auto vrow = [&](int i, int c) -> const uint16_t * { return vres + (size_t)slot_of(i) * kD + c; };
+        const size_t tok0 = (size_t)unit * a.cap + s.nq;
+        const size_t grow = (size_t)unit * a.groups_cap + s.nq / a.G;
+        float *scr = &sm.wy[0][0][0];   // the warp states are summed: free as scratch
+        __syncthreads();
+        pack_key_group<kThreads>(krow, a.G, a.k_codes_w + tok0 * 8, a.k_scale_w + grow * kD,
+                                 a.k_zero_w + grow * kD, scr);
+        pack_value_tokens<kThreads>(vrow, a.G, kD, a.v_codes_w + tok0 * 8, a.v_scale_w + tok0, a.v_zero_w + tok0);
+    }
+}
 
-        // running state of heads hA, hA+1: max (log2 units), sum p, sum p*v_zero
-        float m_run[2] = {-INFINITY, -INFINITY};
-        unsigned long long l2 = f2pack(0.f, 0.f), pz2 = f2pack(0.f, 0.f);
+// ------------------------------------------------------------------ issuing
+
+// Per-lane constants of the copies of a packed item.
+struct PackedLane {
+    uint32_t row;       // smem offset of this lane's K / V code chunk (token lane/2, half lane%2)
+    uint32_t sz_dst;    // smem offset of its key-scale / key-zero chunk
+    uint32_t v_dst;     // smem offset of its value scale / zero chunk (lanes 0-7)
+    uint32_t sz_src;    // byte offset of that chunk in a scale / zero row
+    uint32_t v_src;     // byte offset in the value scale / zero run
+};
+
+// Queue the copies of packed item j (tokens 32j..32j+31) of unit u into the
+// stage at `st` (shared address).  Every lane copies 16-byte chunks.
+template <class A>
+__device__ __forceinline__ void issue_packed(const A &a, uint32_t st, int u, int j, int lane, const PackedLane &pl) {
+    const size_t tok = (size_t)u * a.cap + (size_t)j * kSlice;
+    const char *kc = reinterpret_cast<const char *>(a.k_codes) + tok * 32 + 16 * lane;
+    const char *vc = reinterpret_cast<const char *>(a.v_codes) + tok * 32 + 16 * lane;
+    cp_async16(st + kOffKc + pl.row, kc, true);
+    cp_async16(st + kOffKc + 512 + pl.row, kc + 512, true);
+    cp_async16(st + kOffVc + pl.row, vc, true);
+    cp_async16(st + kOffVc + 512 + pl.row, vc + 512, true);
+    const size_t grow = (size_t)u * a.groups_cap + ((j * kSlice) >> a.lg2G);
+    const char *sz = reinterpret_cast<const char *>(lane < 16 ? a.k_scale : a.k_zero) + grow * (kD * 2);
+    cp_async16(st + pl.sz_dst, sz + pl.sz_src, true);
+    if (lane < 8) {
+        const char *vsz = reinterpret_cast<const char *>(lane < 4 ? a.v_scale : a.v_zero) + tok * 2;
+        cp_async16(st + pl.v_dst, vsz + pl.v_src, true);
+    }
+}
+
+// Residual item i of unit u: logical residual tokens 5i .. 5i+4 (those below r;
+// the rest are zero-filled).  Lanes 0-15 copy chunk `lane` of each K row,
+// lanes 16-31 chunk `lane - 16` of each V row.  Token r-1 is this step's new
+// token, read from k_new / v_new.
+template <class A>
+__device__ __forceinline__ void issue_residual(const A &a, uint32_t st, int u, int i, int r, int rs, int lane) {
+    const int part = lane >> 4, c = lane & 15;
+    const uint16_t *newrow = (part ? a.v_new : a.k_new) + (size_t)u * kD + 8 * c;
+    const uint16_t *ring = (part ? a.v_res : a.k_res) + (size_t)u * a.ring * kD + 8 * c;
+    const int t0 = i * kResTok;
+    int slot = rs + t0;
+    if (slot >= a.ring) slot -= a.ring;
+#pragma unroll
+    for (int j = 0; j < kResTok; ++j) {
+        const int ti = t0 + j;
+        const bool ok = ti < r;
+        const uint16_t *src = (ti == r - 1 || !ok) ? newrow : ring + (size_t)slot * kD;
+        const uint32_t dst = part == 0 ? st + kOffRk + j * 256 + 16 * (c ^ j)
+                                       : st + kOffRv + j * 256 + 16 * ((c + rvrot(j)) & 15);
+        cp_async16(dst, src, ok);
+        if (++slot == a.ring) slot = 0;
+    }
+}
+
+// Query rows of unit u (heads >= g zero-filled) into a q buffer: chunk c of
+// head h at position c ^ h.
+template <class A>
+__device__ __forceinline__ void issue_q(const A &a, uint32_t qb, int u, int lane) {
+    const int b = u / a.Hkv, kh = u - b * a.Hkv;
+    const uint16_t *qrow = a.q + ((size_t)b * a.Hkv * a.g + (size_t)kh * a.g) * kD;
+#pragma unroll
+    for (int e0 = 0; e0 < 64; e0 += 32) {
+        const int e = e0 + lane, h = e >> 4, c = e & 15;
+        const bool ok = h < a.g;
+        cp_async16(qb + (h * 16 + (c ^ h)) * 16, qrow + (ok ? h : 0) * kD + 8 * c, ok);
+    }
+}
+
+// ------------------------------------------------------------------ the CTA
+
+template <bool kMass, class A>
+__device__ void run_cta(const A &a, Smem &sm, int c) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int g_ = lane >> 2, t_ = lane & 3;
+    const int xlo = cta_lo(a, c), xhi = cta_lo(a, c + 1);
+    if (tid == 0) {
+        sm.zero = make_uint4(0, 0, 0, 0);
+        sm.next = xlo + kWarps * (kStages - 1);   // the first kStages-1 items of each warp are fixed
+        seg_info(a, xlo, xhi, sm.seg);
+    }
+    __syncthreads();
+
+    const uint32_t st0 = smem_addr(&sm.stage[warp][0][0]);
+    const uint32_t qb0 = smem_addr(&sm.qbuf[warp][0][0]);
+    const uint32_t zero_addr = smem_addr(&sm.zero);
+
+    // ---- producer: claims items of [xlo, xhi) and queues them kStages - 1 ahead
+    PackedLane pl;
+    pl.row = kpos(lane >> 1) * 32 + 16 * (lane & 1);
+    pl.sz_dst = (lane < 16 ? kOffKs : kOffKz) + 16 * schunk(lane & 15);
+    pl.sz_src = 16 * (lane & 15);
+    pl.v_dst = (lane < 4 ? kOffVs : kOffVz) + 16 * (lane & 3);
+    pl.v_src = 16 * (lane & 3);
+    Cursor pc;
+    pc.set(a, min(xlo + warp, xhi - 1));
+    int pq_unit = -1, pq_slot = -1, pstage = 0, nclaim = 0;
+    int xq0 = xhi, xq1 = xhi, xq2 = xhi;   // claimed items in flight, oldest first (xhi = none)
+    auto issue_next = [&]() {
+        int x;
+        if (nclaim < kStages - 1) {
+            x = xlo + warp + kWarps * nclaim;
+        } else {
+            if (lane == 0) x = atomicAdd(&sm.next, 1);
+            x = __shfl_sync(0xffffffffu, x, 0);
+        }
+        if (x < xhi) {
+            pc.advance_to(a, x);
+            const uint32_t st = st0 + pstage * kStageBytes;
+            if (pc.u != pq_unit) {   // first item of a new unit for this warp: bring its query rows too
+                pq_unit = pc.u;
+                pq_slot = pq_slot == kStages - 1 ? 0 : pq_slot + 1;
+                issue_q(a, qb0 + pq_slot * 1024, pc.u, lane);
+            }
+            const int r = s_r(a, pc.b), nri = unit_nri(r);
+            if (pc.k < nri) issue_residual(a, st, pc.u, pc.k, r, s_rs(a, pc.b), lane);
+            else issue_packed(a, st, pc.u, pc.k - nri, lane, pl);
+        } else {
+            x = xhi;
+        }
+        cp_async_commit();
+        pstage = pstage == kStages - 1 ? 0 : pstage + 1;
+        if (nclaim == 0) xq0 = x;
+        else if (nclaim == 1) xq1 = x;
+        else xq2 = x;
+        ++nclaim;
+    };
+#pragma unroll
+    for (int s = 0; s < kStages - 1; ++s) issue_next();
+
+    // ---- consumer constants of this lane
+    const float sl2 = a.scale_log2, sl2w = a.scale_log2 * kScoreUnit;
+    const uint32_t lo_neg = (g_ & 1) ? 0xBC00BC00u : 0u;   // fp16x2 (-1, -1) in lo columns, (0, 0) in hi
+    const int hB = g_ >> 1;                                // head of this lane's B column
+    const uint32_t kA = kpos(2 * g_) * 32 + 8 * t_, kB = kpos(2 * g_ + 1) * 32 + 8 * t_;
+    const uint32_t vo0 = kpos(4 * t_) * 32 + 4 * g_, vo1 = kpos(4 * t_ + 1) * 32 + 4 * g_;
+    const uint32_t vo2 = kpos(4 * t_ + 2) * 32 + 4 * g_, vo3 = kpos(4 * t_ + 3) * 32 + 4 * g_;
+    // chunks 4t_ + 2 half (+1) of the key scales (channels 16(2t_+half) .. +15): schunk
+    // swaps the two halves of lanes t_ >= 2
+    const uint32_t ks_h0 = 64 * t_ + 32 * (t_ >> 1), ks_h1 = 64 * t_ + 32 * (1 - (t_ >> 1));
+    // ldmatrix rows of the q B operand: matrix m = lane >> 3 (chunk 4jj + m), row n = lane & 7 ->
+    // head n/2 for even n, zero for odd n (the lo columns)
+    const int qn = lane & 7;
+    const bool q_zero = qn & 1;
+    const uint32_t q_row_off = ((qn >> 1) * 16 + ((lane >> 3) ^ (qn >> 1))) * 16;
+    // ldmatrix of the key-zero quads: matrices (chunk 2j, chunk 2j, chunk 2j+1, chunk 2j+1)
+    const uint32_t z_lane_off = 16 * (lane >> 4);
+    // residual K rows: matrices (chunk 2kk rows, zero, chunk 2kk+1 rows, zero)
+    const int rk_row = lane & 7, rk_m = lane >> 3;
+    const bool rk_live = !(rk_m & 1) && rk_row < kResTok;
+    uint32_t qw[8][2];   // per-segment score B base: (q_c 2^-pos, q_{c+8} 2^-pos), head hB
+
+    int cq_unit = -1, cq_slot = -1, cstage = 0;
+    for (;;) {
+        const Seg sg = sm.seg;
+        const int u = sg.u, ub = sg.ub, nri = sg.nri, nq = sg.nq, r = sg.r, rs = sg.rs;
+
         float acc[8][4];
 #pragma unroll
         for (int i = 0; i < 8; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
+        float m_ref = -INFINITY, l = 0.f, pz = 0.f;
+        bool vunit = false;   // acc holds packed-value units (x 2^(pos-24)) once a packed item was seen
+        uint32_t qb = 0;      // this segment's q buffer (shared address)
 
-        for (int x = cs + warp + 4 * k; ok && x < seg_end; x += 4, ++k) {
-            const int stage = k % kWarpStages;
-            ok = mbar_wait(&sm.full[warp][stage], (k / kWarpStages) & 1);
-            if (!ok) break;
-            const SliceBuf &S = sm.st[warp][stage];
-
-            // ---- zero-point term sum_c q_c z_c: A = the key-zero row in all 16 rows
-            float zc[4] = {0.f, 0.f, 0.f, 0.f};
+        while (xq0 < sg.hi) {
+            const int x = xq0;
+            issue_next();
+            cp_async_wait<kStages - 1>();
+            __syncwarp();
+            const uint32_t S = st0 + cstage * kStageBytes;
+            if (u != cq_unit) {   // first item of the segment for this warp: its query rows arrived with it
+                cq_unit = u;
+                cq_slot = cq_slot == kStages - 1 ? 0 : cq_slot + 1;
+                qb = qb0 + cq_slot * 1024;
+                const uint32_t qh = qb + hB * 256;
+                const uint4 qa0 = lds128(qh + ((4 * t_) ^ hB) * 16);
+                const uint4 qb0v = lds128(qh + ((4 * t_ + 1) ^ hB) * 16);
+                const uint4 qa1 = lds128(qh + ((4 * t_ + 2) ^ hB) * 16);
+                const uint4 qb1v = lds128(qh + ((4 * t_ + 3) ^ hB) * 16);
 #pragma unroll
-            for (int kp = 0; kp < 4; ++kp) {
-                uint32_t za[4], zb[4], qf[4];
-                ldmatrix_x4(za, smem_addr(&S.kz[32 * kp + 8 * (lane >> 4)]));
-                ldmatrix_x4(qf, smem_addr(&sm.qn[lane & 7][qn_col(lane & 7, 32 * kp + 8 * (lane >> 3))]));
-                mma16816(zc, za, qf[0], qf[1]);
-                ldmatrix_x4(zb, smem_addr(&S.kz[32 * kp + 16 + 8 * (lane >> 4)]));
-                mma16816(zc, zb, qf[2], qf[3]);
+                for (int kk = 0; kk < 8; ++kk) {
+                    const int half = kk >> 2, Q = kk & 3;
+                    const uint32_t wa = w4(half ? qa1 : qa0, Q), wb = w4(half ? qb1v : qb0v, Q);
+                    const float w0 = pair_wq(2 * Q), w1 = pair_wq(2 * Q + 1);
+                    const __half2 s0 = __floats2half2_rn(w0, w0), s1 = __floats2half2_rn(w1, w1);
+                    qw[kk][0] = hmul2(__byte_perm(wa, wb, 0x5410), *reinterpret_cast<const uint32_t *>(&s0));
+                    qw[kk][1] = hmul2(__byte_perm(wa, wb, 0x7632), *reinterpret_cast<const uint32_t *>(&s1));
+                }
             }
-            // ---- scores: both m-tiles, one k-chunk at a time; B operand made just in time
-            float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
-            {
-                const uint2 ka0 = *reinterpret_cast<const uint2 *>(&S.kc[pg * 8 + 2 * t_]);
-                const uint2 kb0 = *reinterpret_cast<const uint2 *>(&S.kc[(pg + 8) * 8 + 2 * t_]);
-                const uint2 ka1 = *reinterpret_cast<const uint2 *>(&S.kc[(pg + 16) * 8 + 2 * t_]);
-                const uint2 kb1 = *reinterpret_cast<const uint2 *>(&S.kc[(pg + 24) * 8 + 2 * t_]);
+            const uint32_t q_addr = q_zero ? zero_addr : qb + q_row_off;
+            const uint32_t q_step = q_zero ? 0u : 64u;
+            const int k = x - ub;
+
+            if (k < nri) {
+                // ================= residual item: tokens t0 .. t0+n-1 in fp16
+                const int t0 = k * kResTok, n = min(kResTok, r - t0);
+                if (r - 1 >= t0 && r - 1 < t0 + kResTok) {   // the new token: append it to the ring
+                    const int j = r - 1 - t0, part = lane >> 4, cch = lane & 15;
+                    int sl = rs + r - 1;
+                    if (sl >= a.ring) sl -= a.ring;
+                    const uint32_t src = part == 0 ? S + kOffRk + j * 256 + 16 * (cch ^ j)
+                                                   : S + kOffRv + j * 256 + 16 * ((cch + rvrot(j)) & 15);
+                    const uint4 v = lds128(src);
+                    *reinterpret_cast<uint4 *>((part ? a.v_res : a.k_res) + ((size_t)u * a.ring + sl) * kD + 8 * cch) =
+                        v;
+                }
+                float sr[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    const uint32_t a0 = half ? ka0.y : ka0.x, b0 = half ? kb0.y : kb0.x;
-                    const uint32_t a1 = half ? ka1.y : ka1.x, b1 = half ? kb1.y : kb1.x;
-                    const uint32_t a0r = shr6(a0), a0l = shl4(a0), b0r = shr6(b0), b0l = shl4(b0);
-                    const uint32_t a1r = shr6(a1), a1l = shl4(a1), b1r = shr6(b1), b1l = shl4(b1);
-#define KSTEP(Q)                                                                                               \
-    {                                                                                                          \
-        const int kk = 4 * half + Q;                                                                           \
-        const int ch = 16 * (2 * t_ + half) + 2 * Q;                                                           \
-        const uint32_t sa = *reinterpret_cast<const uint32_t *>(&S.ks[ch]);                                    \
-        const uint32_t sb = *reinterpret_cast<const uint32_t *>(&S.ks[ch + 8]);                                \
-        const uint32_t e0 = __byte_perm(sa, sb, 0x5410), e1 = __byte_perm(sa, sb, 0x7632);                     \
-        const uint32_t bk0 = hfma2(qw[kk][0], e0, hmul2(hmul2(qw[kk][0], e0), lo_neg));                        \
-        const uint32_t bk1 = hfma2(qw[kk][1], e1, hmul2(hmul2(qw[kk][1], e1), lo_neg));                        \
-        const uint32_t f0[4] = {code_pair<2 * Q>(a0, a0r, a0l), code_pair<2 * Q>(b0, b0r, b0l),                \
-                                code_pair<2 * Q + 1>(a0, a0r, a0l), code_pair<2 * Q + 1>(b0, b0r, b0l)};       \
-        mma16816(s0, f0, bk0, bk1);                                                                            \
-        const uint32_t f1[4] = {code_pair<2 * Q>(a1, a1r, a1l), code_pair<2 * Q>(b1, b1r, b1l),                \
-                                code_pair<2 * Q + 1>(a1, a1r, a1l), code_pair<2 * Q + 1>(b1, b1r, b1l)};       \
-        mma16816(s1, f1, bk0, bk1);                                                                            \
+                for (int kq = 0; kq < 4; ++kq) {
+                    uint32_t qf[4];
+                    ldmatrix_x4(qf, q_addr + kq * q_step);
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const int kk = 2 * kq + e;
+                        uint32_t ka[4];
+                        ldmatrix_x4(ka, rk_live ? S + kOffRk + rk_row * 256 + 16 * ((2 * kk + (rk_m >> 1)) ^ rk_row)
+                                                : zero_addr);
+                        mma16816(sr, ka, qf[2 * e], qf[2 * e + 1]);
+                    }
+                }
+                const bool valid = g_ < n;
+                const float xa = valid ? sr[0] * sl2 : -INFINITY;   // absolute log2 score of token g_, head t_
+                float xv = xa - m_ref;
+                if (__any_sync(0xffffffffu, xv > kLazy)) {
+                    const float mn = fmaxf(m_ref, warp_max_g(xa));
+                    const float al = ex2(m_ref - mn);
+                    l *= al;
+                    pz *= al;
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        acc[i][0] *= al;
+                        acc[i][1] *= al;
+                        acc[i][2] *= al;
+                        acc[i][3] *= al;
+                    }
+                    m_ref = mn;
+                    xv = xa - mn;
+                }
+                if (kMass && valid && t_ < a.g)
+                    a.xs[((size_t)u * a.g + t_) * a.xs_stride + nq + t0 + g_] = xa;
+                const float p = valid ? ex2(xv) : 0.f;
+                l += p;
+                const float ph = __half2float(__float2half_rn(p));
+                const uint32_t bp = movmatrix_t(pack_half2(p, p - ph));
+                // V^T fragments (m16n8k8): channel rows 16g_+I (a0) and 16g_+8+I (a1), tokens 2t_, 2t_+1
+                uint4 A0 = make_uint4(0, 0, 0, 0), A1 = A0, B0 = A0, B1 = A0;
+                const int ta = 2 * t_, tb = 2 * t_ + 1;
+                if (ta < kResTok) {
+                    const uint32_t rowa = S + kOffRv + ta * 256;
+                    A0 = lds128(rowa + 16 * ((2 * g_ + rvrot(ta)) & 15));
+                    A1 = lds128(rowa + 16 * ((2 * g_ + 1 + rvrot(ta)) & 15));
+                }
+                if (tb < kResTok) {
+                    const uint32_t rowb = S + kOffRv + tb * 256;
+                    B0 = lds128(rowb + 16 * ((2 * g_ + rvrot(tb)) & 15));
+                    B1 = lds128(rowb + 16 * ((2 * g_ + 1 + rvrot(tb)) & 15));
+                }
+#define RSTEP(I)                                                                                \
+    mma1688(acc[I], __byte_perm(w4(A0, I >> 1), w4(B0, I >> 1), (I & 1) ? 0x7632 : 0x5410),     \
+            __byte_perm(w4(A1, I >> 1), w4(B1, I >> 1), (I & 1) ? 0x7632 : 0x5410), bp);
+                RSTEP(0) RSTEP(1) RSTEP(2) RSTEP(3) RSTEP(4) RSTEP(5) RSTEP(6) RSTEP(7)
+#undef RSTEP
+            } else {
+                // ================= packed item: tokens 32j .. 32j+31 of the unit
+                const int j = k - nri;
+                if (!vunit) {   // from here on acc holds packed-value units: code 2^(pos-24) per channel pair
+                    vunit = true;
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const float f = 1.f / pair_wo(i);
+                        acc[i][0] *= f;
+                        acc[i][1] *= f;
+                        acc[i][2] *= f;
+                        acc[i][3] *= f;
+                    }
+                }
+                // ---- zero-point term sum_c q_c z_c (A = the key-zero chunk in every row)
+                float zc4[4] = {0.f, 0.f, 0.f, 0.f};
+                const uint32_t zb = S + kOffKz + z_lane_off;
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) {
+                    uint32_t qf[4];
+                    ldmatrix_x4(qf, q_addr + jj * q_step);
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const int jc = 2 * jj + e;                     // k-chunk: chunks 2jc, 2jc+1
+                        const int jp = jc < 4 ? jc : (jc ^ 1);         // their position pair under schunk
+                        uint32_t za[4];
+                        ldmatrix_x4(za, zb + 32 * jp);
+                        mma16816(zc4, za, qf[2 * e], qf[2 * e + 1]);
+                    }
+                }
+                // ---- scores: both m-tiles, one k-chunk at a time; B operand made just in time
+                float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
+                {
+                    const uint2 ka0 = lds64(S + kOffKc + kA), kb0 = lds64(S + kOffKc + kB);
+                    const uint2 ka1 = lds64(S + kOffKc + 512 + kA), kb1 = lds64(S + kOffKc + 512 + kB);
+#pragma unroll
+                    for (int half = 0; half < 2; ++half) {
+                        const uint32_t ksh = half ? ks_h1 : ks_h0;
+                        const uint4 sA = lds128(S + kOffKs + ksh);        // channels 16w .. 16w+7, w = 2t_ + half
+                        const uint4 sB = lds128(S + kOffKs + ksh + 16);   // 16w+8 .. 16w+15
+                        const uint32_t a0 = half ? ka0.y : ka0.x, b0 = half ? kb0.y : kb0.x;
+                        const uint32_t a1 = half ? ka1.y : ka1.x, b1 = half ? kb1.y : kb1.x;
+                        const uint32_t a0r = shr10(a0), b0r = shr10(b0), a1r = shr10(a1), b1r = shr10(b1);
+#define KSTEP(Q)                                                                                    \
+    {                                                                                               \
+        const int kk = 4 * half + Q;                                                                \
+        const uint32_t e0 = __byte_perm(w4(sA, Q), w4(sB, Q), 0x5410);                              \
+        const uint32_t e1 = __byte_perm(w4(sA, Q), w4(sB, Q), 0x7632);                              \
+        const uint32_t bk0 = hfma2(qw[kk][0], e0, hmul2(hmul2(qw[kk][0], e0), lo_neg));             \
+        const uint32_t bk1 = hfma2(qw[kk][1], e1, hmul2(hmul2(qw[kk][1], e1), lo_neg));             \
+        const uint32_t f0[4] = {code_pair<2 * Q>(a0, a0r), code_pair<2 * Q>(b0, b0r),               \
+                                code_pair<2 * Q + 1>(a0, a0r), code_pair<2 * Q + 1>(b0, b0r)};      \
+        mma16816(s0, f0, bk0, bk1);                                                                 \
+        const uint32_t f1[4] = {code_pair<2 * Q>(a1, a1r), code_pair<2 * Q>(b1, b1r),               \
+                                code_pair<2 * Q + 1>(a1, a1r), code_pair<2 * Q + 1>(b1, b1r)};      \
+        mma16816(s1, f1, bk0, bk1);                                                                 \
     }
-                    KSTEP(0) KSTEP(1) KSTEP(2) KSTEP(3)
+                        KSTEP(0) KSTEP(1) KSTEP(2) KSTEP(3)
 #undef KSTEP
+                    }
                 }
-            }
-            // ---- x = score * scale - mr (log2 units, relative to the running max mr;
-            //      0 stands in until a first max is known)
-            const float mr0 = (m_run[0] == -INFINITY) ? 0.f : m_run[0];
-            const float mr1 = (m_run[1] == -INFINITY) ? 0.f : m_run[1];
-            float x_[2][4];
+                // ---- x = log2 score relative to the reference max m_ref (tokens 2g_, 2g_+1, 16+2g_, 17+2g_)
+                const float zcs = zc4[0] * sl2;
+                const float sc[4] = {s0[0] + s0[1], s0[2] + s0[3], s1[0] + s1[1], s1[2] + s1[3]};
+                float xv[4];
+                {
+                    const float bias = zcs - m_ref;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const float v0 = fmaf(zc[i], 1.f / 65536.f, s0[i]), v1 = fmaf(zc[i], 1.f / 65536.f, s1[i]);
-                const float w0 = v0 + __shfl_xor_sync(0xffffffffu, v0, 2);
-                const float w1 = v1 + __shfl_xor_sync(0xffffffffu, v1, 2);
-                x_[0][i] = fmaf(w0, a.scale_log2 * 65536.f, (i & 1) ? -mr1 : -mr0);
-                x_[1][i] = fmaf(w1, a.scale_log2 * 65536.f, (i & 1) ? -mr1 : -mr0);
-            }
-            if (kMass) {   // lanes t_ < 2: head hA + (i & 1), token 16 mt + 8 (i >> 1) + perm8(g_)
-                const int h = hA;
-                if (t_ < 2) {
-                    float *xrow = a.xs + ((size_t)unit * a.g + h) * a.xs_stride + (size_t)(x - u_s0) * kSlice + pg;
-#pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        if (h + (i & 1) < a.g) {
-                            const float ref = (i & 1) ? mr1 : mr0;
-                            xrow[(i & 1) * a.xs_stride + 8 * (i >> 1)] = x_[0][i] + ref;
-                            xrow[(i & 1) * a.xs_stride + 16 + 8 * (i >> 1)] = x_[1][i] + ref;
-                        }
+                    for (int i = 0; i < 4; ++i) xv[i] = fmaf(sc[i], sl2w, bias);
                 }
-            }
-            // ---- online softmax: rescale only when a head's running max grows
-            float mx0 = fmaxf(fmaxf(x_[0][0], x_[0][2]), fmaxf(x_[1][0], x_[1][2]));
-            float mx1 = fmaxf(fmaxf(x_[0][1], x_[0][3]), fmaxf(x_[1][1], x_[1][3]));
-            mx0 = warp_max_g(mx0) + mr0;   // slice max, absolute
-            mx1 = warp_max_g(mx1) + mr1;
-            if (__any_sync(0xffffffffu, mx0 > m_run[0] || mx1 > m_run[1])) {
-                const float n0 = fmaxf(m_run[0], mx0), n1 = fmaxf(m_run[1], mx1);
-                const float al0 = ex2(m_run[0] - n0), al1 = ex2(m_run[1] - n1);   // 0 on the first slice
-                const float d0 = n0 - mr0, d1 = n1 - mr1;                            // shift of the reference
-                m_run[0] = n0;
-                m_run[1] = n1;
-                l2 = fmul2(l2, f2pack(al0, al1));
-                pz2 = fmul2(pz2, f2pack(al0, al1));
+                const float mx = fmaxf(fmaxf(xv[0], xv[1]), fmaxf(xv[2], xv[3]));
+                if (__any_sync(0xffffffffu, mx > kLazy)) {
+                    float xa[4];
 #pragma unroll
-                for (int nu = 0; nu < 8; ++nu) {
-                    acc[nu][0] *= al0;
-                    acc[nu][1] *= al1;
-                    acc[nu][2] *= al0;
-                    acc[nu][3] *= al1;
+                    for (int i = 0; i < 4; ++i) xa[i] = fmaf(sc[i], sl2w, zcs);
+                    const float mn = fmaxf(m_ref, warp_max_g(fmaxf(fmaxf(xa[0], xa[1]), fmaxf(xa[2], xa[3]))));
+                    const float al = ex2(m_ref - mn);
+                    l *= al;
+                    pz *= al;
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        acc[i][0] *= al;
+                        acc[i][1] *= al;
+                        acc[i][2] *= al;
+                        acc[i][3] *= al;
+                    }
+                    m_ref = mn;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) xv[i] = xa[i] - mn;
                 }
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    x_[0][i] -= (i & 1) ? d1 : d0;
-                    x_[1][i] -= (i & 1) ? d1 : d0;
+                if (kMass && t_ < a.g) {
+                    float *xrow = a.xs + ((size_t)u * a.g + t_) * a.xs_stride + (size_t)j * kSlice + 2 * g_;
+                    xrow[0] = xv[0] + m_ref;
+                    xrow[1] = xv[1] + m_ref;
+                    xrow[16] = xv[2] + m_ref;
+                    xrow[17] = xv[3] + m_ref;
                 }
-            }
-            // ---- P' = p * v_scale (hi / lo) and O^T += code^T P'
+                // ---- P' = p * v_scale (hi / lo) and O^T += code^T P'
 #pragma unroll
-            for (int mt = 0; mt < 2; ++mt) {
-                const int base = 16 * mt;
-                uint32_t prow[2];
-#pragma unroll
-                for (int hr = 0; hr < 2; ++hr) {
-                    const int tok = base + 8 * hr + pg;
-                    const float vsc = h2f(S.vs[tok]), vzr = h2f(S.vz[tok]);
-                    const unsigned long long p2 = f2pack(ex2(x_[mt][2 * hr]), ex2(x_[mt][2 * hr + 1]));
-                    l2 = fadd2(l2, p2);
-                    pz2 = ffma2(p2, f2pack(vzr, vzr), pz2);
-                    const unsigned long long y2 = fmul2(p2, f2pack(vsc, vsc));
-                    float y0, y1;
-                    f2unpack(y2, y0, y1);
-                    const uint32_t hv = pack_half2(y0, y1);
-                    const float2 f = unpack_half2(hv);
-                    float r0, r1;
-                    f2unpack(fadd2(y2, f2pack(-f.x, -f.y)), r0, r1);
-                    const uint32_t lv = pack_half2(r0, r1);
-                    prow[hr] = lo_row ? lv : hv;
-                }
-                const uint32_t bv0 = movmatrix_t(prow[0]), bv1 = movmatrix_t(prow[1]);
-                const uint32_t wA = S.vc[(base + p2t) * 8 + g_], wB = S.vc[(base + p2t1) * 8 + g_];
-                const uint32_t wC = S.vc[(base + 8 + p2t) * 8 + g_], wD = S.vc[(base + 8 + p2t1) * 8 + g_];
-                const uint32_t l1 = __byte_perm(wA, wB, 0x5410), h1 = __byte_perm(wA, wB, 0x7632);
-                const uint32_t l2w = __byte_perm(wC, wD, 0x5410), h2 = __byte_perm(wC, wD, 0x7632);
-                const uint32_t l1a = shr6(l1), l1b = shl4(l1), h1a = shr6(h1), h1b = shl4(h1);
-                const uint32_t l2a = shr6(l2w), l2b = shl4(l2w), h2a = shr6(h2), h2b = shl4(h2);
-#define VSTEP(NU)                                                                             \
-    {                                                                                         \
-        const uint32_t af[4] = {code_pair<NU>(l1, l1a, l1b), code_pair<NU>(h1, h1a, h1b),     \
-                                code_pair<NU>(l2w, l2a, l2b), code_pair<NU>(h2, h2a, h2b)};   \
-        mma16816(acc[NU], af, bv0, bv1);                                                      \
+                for (int mt = 0; mt < 2; ++mt) {
+                    const uint32_t vsw = lds32(S + kOffVs + 2 * (16 * mt + 2 * g_));
+                    const uint32_t vzw = lds32(S + kOffVz + 2 * (16 * mt + 2 * g_));
+                    const float2 vsf = unpack_half2(vsw), vzf = unpack_half2(vzw);
+                    const float p0 = ex2(xv[2 * mt]), p1 = ex2(xv[2 * mt + 1]);
+                    l += p0 + p1;
+                    pz = fmaf(p0, vzf.x, fmaf(p1, vzf.y, pz));
+                    const float y0 = p0 * vsf.x, y1 = p1 * vsf.y;
+                    const float2 hf = unpack_half2(pack_half2(y0, y1));
+                    const uint32_t bv0 = movmatrix_t(pack_half2(y0, y0 - hf.x));
+                    const uint32_t bv1 = movmatrix_t(pack_half2(y1, y1 - hf.y));
+                    const uint32_t vb = S + kOffVc + 512 * mt;
+                    const uint32_t wA = lds32(vb + vo0), wC = lds32(vb + vo1), wB = lds32(vb + vo2),
+                                   wD = lds32(vb + vo3);
+                    const uint32_t l1 = __byte_perm(wA, wB, 0x5410), h1 = __byte_perm(wA, wB, 0x7632);
+                    const uint32_t l2 = __byte_perm(wC, wD, 0x5410), h2 = __byte_perm(wC, wD, 0x7632);
+                    const uint32_t l1r = shr10(l1), h1r = shr10(h1), l2r = shr10(l2), h2r = shr10(h2);
+#define VSTEP(NU)                                                                   \
+    {                                                                               \
+        const uint32_t af[4] = {code_pair<NU>(l1, l1r), code_pair<NU>(h1, h1r),     \
+                                code_pair<NU>(l2, l2r), code_pair<NU>(h2, h2r)};    \
+        mma16816(acc[NU], af, bv0, bv1);                                            \
     }
-                VSTEP(0) VSTEP(1) VSTEP(2) VSTEP(3) VSTEP(4) VSTEP(5) VSTEP(6) VSTEP(7)
+                    VSTEP(0) VSTEP(1) VSTEP(2) VSTEP(3) VSTEP(4) VSTEP(5) VSTEP(6) VSTEP(7)
 #undef VSTEP
+                }
             }
             __syncwarp();
-            if (lane == 0 && nxt_x < ce) {
-                issue_slice(a, sm, warp, stage, nxt.u, nxt.j);
-                nxt.step(a, 4);
-                nxt_x += 4;
-            }
+            cstage = cstage == kStages - 1 ? 0 : cstage + 1;
+            xq0 = xq1;   // the next claimed item moves to the head
+            xq1 = xq2;
+            --nclaim;
         }
-        if (!ok && lane == 0 && a.err) atomicExch(a.err, 1);
 
-        // ---- warp epilogue: y[head][channel] = (O^T_hi + O^T_lo) 2^(24-p) + sum p * v_zero
-        float l_run[2], pz[2];
-        f2unpack(l2, l_run[0], l_run[1]);
-        f2unpack(pz2, pz[0], pz[1]);
+        // ---- warp epilogue: scale to the CTA's per-head max, then
+        //      y[head t_][channel] = (O^T_hi + O^T_lo) * unit + sum p * v_zero
+        const float lh = warp_sum_g(l), pzh = warp_sum_g(pz);
+        if (g_ == 0) sm.wm[warp][t_] = m_ref;
+        __syncthreads();
+        float Mc = -INFINITY;
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-            l_run[e] = warp_sum_g(l_run[e]);
-            pz[e] = warp_sum_g(pz[e]);
-        }
-#define VOUT(NU)                                                                      \
-    _Pragma("unroll") for (int i = 0; i < 4; ++i) {                                   \
-        const float y = acc[NU][i] + __shfl_xor_sync(0xffffffffu, acc[NU][i], 2);     \
-        acc[NU][i] = y * pair_wo(NU) + pz[i & 1];                                     \
-    }
-        VOUT(0) VOUT(1) VOUT(2) VOUT(3) VOUT(4) VOUT(5) VOUT(6) VOUT(7)
-#undef VOUT
-        if (t_ < 2) {
+        for (int w = 0; w < kWarps; ++w) Mc = fmaxf(Mc, sm.wm[w][t_]);
+        const float f = (m_ref == -INFINITY) ? 0.f : ex2(m_ref - Mc);
+        const float pzf = pzh * f;
+        {
+            float y[16];
 #pragma unroll
-            for (int nu = 0; nu < 8; ++nu) {
-                const int ch = 16 * g_ + nu;
-                sm.wy[warp][hA][ch] = acc[nu][0];
-                sm.wy[warp][hA + 1][ch] = acc[nu][1];
-                sm.wy[warp][hA][ch + 8] = acc[nu][2];
-                sm.wy[warp][hA + 1][ch + 8] = acc[nu][3];
+            for (int i = 0; i < 8; ++i) {
+                const float fi = (vunit ? pair_wo(i) : 1.f) * f;
+                y[i] = fmaf(acc[i][0] + acc[i][1], fi, pzf);       // channel 16g_ + i
+                y[8 + i] = fmaf(acc[i][2] + acc[i][3], fi, pzf);   // channel 16g_ + 8 + i
             }
-            if (g_ == 0) {
-                sm.wm[warp][hA] = m_run[0];
-                sm.wm[warp][hA + 1] = m_run[1];
-                sm.wl[warp][hA] = l_run[0];
-                sm.wl[warp][hA + 1] = l_run[1];
-            }
+            float4 *dst = reinterpret_cast<float4 *>(&sm.wy[warp][t_][16 * g_]);
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) dst[q4] = make_float4(y[4 * q4], y[4 * q4 + 1], y[4 * q4 + 2], y[4 * q4 + 3]);
         }
-        int first, S_u;
-        unit_slots(a, unit, first, S_u);
-        merge_warps_and_finish<kMass>(a, sm, unit, a.n_rc + (c - first), S_u);
-        seg = seg_end;
+        if (g_ == 0) sm.wl[warp][t_] = lh * f;
+        finish_unit<kMass>(a, sm, sg, c - sg.first);
+        if (sg.hi >= xhi) break;
+        __syncthreads();   // every thread has read sm.seg and the warp states
+        if (tid == 0) seg_info(a, sg.hi, xhi, sm.seg);
+        __syncthreads();
     }
+    cp_async_wait<0>();
 }
 
-template <bool kMass, class A>
-__device__ __forceinline__ void decode_body(const A &a) {
-    extern __shared__ __align__(128) unsigned char smem_raw[];
-    Smem &sm = *reinterpret_cast<Smem *>(smem_raw);
-    // packed CTAs first: they carry most of the work; the short residual CTAs fill in behind them
-    if ((int)blockIdx.x < a.P) packed_cta<kMass>(a, sm, blockIdx.x);
-    else {
-        const int i = blockIdx.x - a.P;
-        residual_chunk_cta<kMass>(a, sm, i / a.n_rc, i % a.n_rc);
-    }
-}
+__device__ __forceinline__ void wait_prior_grid() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
 
 template <bool kMass>
-__global__ void __launch_bounds__(kThreads, 4) decode_kernel(const Args a) {
-    decode_body<kMass>(a);
+__global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_constant__ ArgsUni a) {
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    wait_prior_grid();
+    run_cta<kMass>(a, *reinterpret_cast<Smem *>(smem_raw), blockIdx.x);
 }
 
-// Device-state mode: copy the state in, run the CTA's work, and let the last CTA
+// ragged batch: per-sequence lengths in the parameter table
+template <bool kMass>
+__global__ void __launch_bounds__(kThreads, 1) decode_ragged_kernel(const __grid_constant__ ArgsVar a) {
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    wait_prior_grid();
+    run_cta<kMass>(a, *reinterpret_cast<Smem *>(smem_raw), blockIdx.x);
+}
+
+// First flat item whose start weight is >= w, from the device-state table.
+// Weights stay below 2^45, so the double divisions are exact: for integers
+// N < 2^53 and D > 0, floor(fl(N / D)) = floor(N / D).
+__device__ int dev_first_item(const ArgsDev &a, const long long *wbeg, long long w) {
+    const int B = nseq(a);
+    const int *nqa = dev_arr(a, 0), *ra = dev_arr(a, 1), *ib = dev_arr(a, 3);
+    if (w >= wbeg[B]) return ib[B];
+    int lo = 0, hi = B;   // largest b with wbeg[b] <= w
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (wbeg[mid] <= w) lo = mid;
+        else hi = mid;
+    }
+    const int b = lo, nq = nqa[b], r = ra[b];
+    const long long W = unit_w(nq, r);
+    const long long off = w - wbeg[b];
+    const int kh = (int)floor((double)off / (double)W);
+    const long long rem = off - kh * W;
+    const int nri = unit_nri(r);
+    int k;
+    if (rem <= (long long)(nri - 1) * kWR) k = (int)((rem + kWR - 1) / kWR);
+    else k = nri + (int)((rem - (long long)nri * kWR + kWP - 1) / kWP);
+    return ib[b] + kh * unit_items(nq, r) + k;
+}
+
+// Device-state mode: build the table, run the CTA's work, and let the last CTA
 // of the launch advance the state of every sequence (append; flush G tokens
 // where the ring is full).  A flush that would pass `cap` is not done: the
 // sequence keeps its state and its status word is set to 1.
 template <bool kMass>
-__global__ void __launch_bounds__(kThreads, 4) decode_dev_kernel(const ArgsDev a) {
+__global__ void __launch_bounds__(kThreads, 1) decode_dev_kernel(const ArgsDev a) {
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    wait_prior_grid();
     const int tid = threadIdx.x;
-    const int B = a.units / a.Hkv;
-    int *nq = dev_arr(a, 0), *rr = dev_arr(a, 1), *rs = dev_arr(a, 2), *sbeg = dev_arr(a, 3);
+    const int B = nseq(a);
+    int *nq = dev_arr(a, 0), *rr = dev_arr(a, 1), *rs = dev_arr(a, 2), *ib = dev_arr(a, 3), *clo = dev_arr(a, 4);
+    __shared__ long long wbeg[kMaxRaggedSeqs + 1];
     for (int b = tid; b < B; b += kThreads) {
         const int4 st = __ldcg(reinterpret_cast<const int4 *>(a.dseq) + b);
         nq[b] = st.x;
@@ -877,37 +927,54 @@ __global__ void __launch_bounds__(kThreads, 4) decode_dev_kernel(const ArgsDev a
         rs[b] = st.z;
     }
     __syncthreads();
-    if (tid < 32) {   // sbeg = exclusive prefix of Hkv * slices, one warp, 32 sequences per pass
-        int carry = 0;
+    if (tid < 32) {   // exclusive prefix sums of items and weights, 32 sequences per pass
+        int ci = 0;
+        long long cw = 0;
         for (int b0 = 0; b0 < B; b0 += 32) {
             const int b = b0 + tid;
-            const int v = b < B ? a.Hkv * (nq[b] / kSlice) : 0;
-            int x = v;
+            const int vi = b < B ? a.Hkv * unit_items(nq[b], rr[b]) : 0;
+            const long long vw = b < B ? (long long)a.Hkv * unit_w(nq[b], rr[b]) : 0;
+            int xi = vi;
+            long long xw = vw;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
-                const int y = __shfl_up_sync(0xffffffffu, x, o);
-                if (tid >= o) x += y;
+                const int yi = __shfl_up_sync(0xffffffffu, xi, o);
+                const long long yw = __shfl_up_sync(0xffffffffu, xw, o);
+                if (tid >= o) {
+                    xi += yi;
+                    xw += yw;
+                }
             }
-            if (b < B) sbeg[b] = carry + x - v;
-            carry += __shfl_sync(0xffffffffu, x, 31);
+            if (b < B) {
+                ib[b] = ci + xi - vi;
+                wbeg[b] = cw + xw - vw;
+            }
+            ci += __shfl_sync(0xffffffffu, xi, 31);
+            cw += __shfl_sync(0xffffffffu, xw, 31);
         }
         if (tid == 0) {
-            sbeg[B] = carry;
+            ib[B] = ci;
+            wbeg[B] = cw;
             DevTab &t = dev_tab();
-            t.Ns = carry;
-            long long P = a.P;   // packed CTAs of the grid; at least 4 slices each
-            if (P > (carry + 3) / 4) P = (carry + 3) / 4;
-            t.P = (int)P;
+            t.Wt = cw;
+            long long P = a.P;   // CTAs of the grid; each share at least kMinShare
+            if (P > cw / kMinShare) P = cw / kMinShare;
+            t.P = (int)(P < 1 ? 1 : P);
         }
     }
     __syncthreads();
-    decode_body<kMass>(a);
+    {
+        const int P = dev_tab().P;
+        const long long Wt = dev_tab().Wt;
+        for (int cc = tid; cc <= P; cc += kThreads)
+            clo[cc] = dev_first_item(a, wbeg, (long long)floor((double)cc * (double)Wt / (double)P));
+    }
+    __syncthreads();
+    if ((int)blockIdx.x < dev_tab().P) run_cta<kMass>(a, *reinterpret_cast<Smem *>(smem_raw), blockIdx.x);
     __syncthreads();
     if (tid == 0) {
-        __threadfence();
         const unsigned n = gridDim.x;
-        if (atomicInc(a.grid_counter, n - 1) == n - 1) {
-            __threadfence();
+        if (atom_inc_acq_rel(a.grid_counter, n - 1) == n - 1) {
             for (int b = 0; b < B; ++b) {
                 int4 st = make_int4(nq[b], rr[b], rs[b], __ldcg(a.dseq + 4 * b + 3));   // status stays set
                 if (rr[b] == a.ring) {
@@ -926,17 +993,11 @@ __global__ void __launch_bounds__(kThreads, 4) decode_dev_kernel(const ArgsDev a
     }
 }
 
-// ragged batch: per-sequence lengths in the parameter table
-template <bool kMass>
-__global__ void __launch_bounds__(kThreads, 4) decode_ragged_kernel(const __grid_constant__ ArgsVar a) {
-    decode_body<kMass>(a);
-}
-
 // mass[unit][t] += sum_h 2^(xs[unit][h][t] - M_h) / L_h for the n_u tokens
 // the unit attended to this step (n_u, M_h, L_h from the merging CTA's stats);
 // grid (ceil(max n_u / 1024), units), four consecutive tokens per thread,
 // all G_ score loads issued before any use.  Launched as a programmatic
-// dependent of decode_kernel<true>: its launch overlaps the decode kernel's
+// dependent of the decode kernel: its launch overlaps the decode kernel's
 // tail and griddepcontrol.wait holds it until that grid has finished and its
 // writes are visible.  xs rows are 16-byte aligned (xs_stride4 float4s each);
 // entries from n up to the row end hold no score and are never used.
@@ -977,44 +1038,54 @@ __global__ void __launch_bounds__(256) mass_kernel(const float4 *__restrict__ xs
     }
 }
 
-int g_slots = 0;   // resident decode CTAs on the device (SMs x CTAs per SM)
-bool g_attr_done = false;
+// ------------------------------------------------------------ host planning
 
-template <class K>
-bool set_smem_attr(K kernel) {
-    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(Smem)) ==
-           cudaSuccess;
+// Per-device set-up (a function attribute applies to the device current when
+// it is set; the SM count is looked up per device), guarded for calls from
+// several host threads.
+std::mutex g_dev_mu;
+bool g_attr_done[kMaxDevices] = {};
+int g_sms[kMaxDevices] = {};
+
+size_t dev_smem_bytes(int B, int P) {
+    return sizeof(Smem) + sizeof(DevTab) + (4 * (size_t)B + 1 + (size_t)P + 1) * sizeof(int);
 }
 
-// the kernels' shared memory is above the 48 KB default: opt in once
-int ensure_attr() {
-    if (!g_attr_done) {
-        const int dev_max = (int)(sizeof(Smem) + sizeof(DevTab) + (4 * kMaxRaggedSeqs + 1) * sizeof(int));
-        if (!set_smem_attr(decode_kernel<false>) || !set_smem_attr(decode_kernel<true>) ||
-            !set_smem_attr(decode_ragged_kernel<false>) || !set_smem_attr(decode_ragged_kernel<true>) ||
-            cudaFuncSetAttribute(decode_dev_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, dev_max) !=
+// the kernels' shared memory is above the 48 KB default: opt in once per device
+int ensure_attr(int dev) {
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    if (!g_attr_done[dev]) {
+        const int smax = (int)dev_smem_bytes(kMaxRaggedSeqs, kMaxCtas);
+        const int s = (int)sizeof(Smem);
+        if (cudaFuncSetAttribute(decode_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, s) != cudaSuccess ||
+            cudaFuncSetAttribute(decode_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, s) != cudaSuccess ||
+            cudaFuncSetAttribute(decode_ragged_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, s) !=
                 cudaSuccess ||
-            cudaFuncSetAttribute(decode_dev_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, dev_max) !=
+            cudaFuncSetAttribute(decode_ragged_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, s) !=
+                cudaSuccess ||
+            cudaFuncSetAttribute(decode_dev_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smax) !=
+                cudaSuccess ||
+            cudaFuncSetAttribute(decode_dev_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smax) !=
                 cudaSuccess)
             return check_launch("decode_attn: cudaFuncSetAttribute");
-        g_attr_done = true;
+        g_attr_done[dev] = true;
     }
     return MINIKV_OK;
 }
 
-int resident_slots() {
-    if (g_slots == 0) {
-        int dev = 0, sms = 148, per = 4;
-        if (ensure_attr() == MINIKV_OK && cudaGetDevice(&dev) == cudaSuccess) {
-            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, decode_kernel<false>, kThreads, sizeof(Smem)) !=
-                    cudaSuccess || per < 1)
-                per = 4;
-        }
-        cudaGetLastError();
-        g_slots = (sms > 0 ? sms : 148) * per;
+// one decode CTA per SM
+int sm_count(int dev) {
+    {
+        std::lock_guard<std::mutex> lk(g_dev_mu);
+        if (g_sms[dev] > 0) return g_sms[dev];
     }
-    return g_slots;
+    int sms = 148;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1) sms = 148;
+    cudaGetLastError();
+    if (sms > kMaxCtas) sms = kMaxCtas;
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    g_sms[dev] = sms;
+    return sms;
 }
 
 // Host state of sequence b: the table of a ragged cache, else the shared scalars.
@@ -1023,97 +1094,78 @@ int seq_nres(const minikv_cache *c, int b) { return c->seq ? c->seq[3 * b + 1] :
 int seq_rs(const minikv_cache *c, int b) { return c->seq ? c->seq[3 * b + 2] : c->res_start; }
 
 struct Plan {
-    int units, n_rc, spu, P, S_max, Ns;
-    int max_n;   // most tokens any unit attends to this step
+    int units, P, S_max;
+    int max_n;               // most tokens any unit attends to this step
+    std::vector<int> lo;     // host-planned modes: first item of each CTA (P + 1 entries)
 };
 
-// shared memory of decode_dev_kernel for a batch of B sequences
-size_t dev_smem_bytes(int B) { return sizeof(Smem) + sizeof(DevTab) + (4 * (size_t)B + 1) * sizeof(int); }
-
-// resident decode_dev_kernel CTAs for this shared-memory size (looked up once
-// per size, so that calls under stream capture make no occupancy query)
-int dev_slots(size_t smem) {
-    static size_t last_smem = 0;
-    static int last_slots = 0;
-    if (smem == last_smem && last_slots > 0) return last_slots;
-    int dev = 0, sms = 148, per = 4;
-    if (ensure_attr() == MINIKV_OK && cudaGetDevice(&dev) == cudaSuccess) {
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, decode_dev_kernel<false>, kThreads, smem) !=
-                cudaSuccess || per < 1)
-            per = 1;
-    }
-    cudaGetLastError();
-    last_smem = smem;
-    last_slots = (sms > 0 ? sms : 148) * per;
-    return last_slots;
+// CTAs that take a share: one per SM, at least kMinShare weight each
+long long cta_count(long long Wt, int slots) {
+    long long P = slots;
+    if (P > Wt / kMinShare) P = Wt / kMinShare;
+    if (P > kMaxCtas) P = kMaxCtas;
+    return P < 1 ? 1 : P;
 }
 
-Plan plan(const minikv_cache *c) {
+// Partial slots per unit for a unit of weight W when every CTA share is at
+// least `share` wide: the CTA ranges its items can fall into.
+int slots_bound(long long W, long long share) { return (int)(W / share + 2); }
+
+Plan plan(const minikv_cache *c, int dev) {
     Plan p;
     p.units = c->B * c->Hkv;
+    const int ring = c->R + c->G;
     if (c->dseq) {
         // device-state mode: one configuration for every state the cache can hold;
-        // the kernel partitions this step's slices itself
-        const int ring = c->R + c->G;
-        const int spu_cap = c->cap / kSlice;
-        p.n_rc = (ring + kResChunk - 1) / kResChunk;
-        p.spu = 0;
-        p.Ns = p.units * spu_cap;
-        p.P = 0;
-        if (p.Ns > 0) {
-            long long P = dev_slots(dev_smem_bytes(c->B));
-            if (P > (p.Ns + 3) / 4) P = (p.Ns + 3) / 4;
-            if (P > kMaxPackedCtas) P = kMaxPackedCtas;
-            p.P = (int)(P < 1 ? 1 : P);
-        }
-        int per_unit = p.Ns > 0 ? spu_cap / 3 + 2 : 0;
-        if (per_unit > p.P) per_unit = p.P;
-        p.S_max = p.n_rc + per_unit;
+        // the kernel partitions this step's items itself
+        const long long Wmax = unit_w(c->cap, ring);
+        p.P = (int)cta_count((long long)p.units * Wmax, sm_count(dev));
+        p.S_max = slots_bound(Wmax, kMinShare);
+        if (p.S_max > p.P) p.S_max = p.P;
         p.max_n = c->cap + ring;
         return p;
     }
-    const int nb = c->seq ? c->B : 1;   // distinct sequence states
-    int max_r = 0;
-    long long Ns = 0;
+    const bool ragged = c->seq != nullptr;
+    // per-sequence item and weight prefix sums (uniform: one state for every sequence)
+    std::vector<long long> wbeg(c->B + 1, 0);
+    std::vector<int> ibeg(c->B + 1, 0);
+    long long Wmax = 0;
     p.max_n = 0;
-    for (int b = 0; b < nb; ++b) {
-        const int r = seq_nres(c, b) + 1;
-        if (r > max_r) max_r = r;
-        if (seq_nq(c, b) + r > p.max_n) p.max_n = seq_nq(c, b) + r;
-        Ns += (long long)c->Hkv * (seq_nq(c, b) / kSlice);
+    for (int b = 0; b < c->B; ++b) {
+        const int s = ragged ? b : 0;
+        const int r = seq_nres(c, s) + 1, nq = seq_nq(c, s);
+        if (nq + r > p.max_n) p.max_n = nq + r;
+        const long long W = unit_w(nq, r);
+        if (W > Wmax) Wmax = W;
+        wbeg[b + 1] = wbeg[b] + (long long)c->Hkv * W;
+        ibeg[b + 1] = ibeg[b] + c->Hkv * unit_items(nq, r);
     }
-    if (!c->seq) Ns *= c->B;
-    p.n_rc = (max_r + kResChunk - 1) / kResChunk;
-    p.spu = c->seq ? 0 : c->n_packed / kSlice;   // slices per unit (uniform batches)
-    p.Ns = (int)Ns;                             // the caller bounds units * cap / 32 below 2^31
-    p.P = 0;
-    if (p.Ns > 0) {
-        // packed CTAs fill every resident slot, all in one wave, so that each SM
-        // holds the same packed work; the short residual CTAs run as a second
-        // wave behind them.  (Three of four slots, with residual CTAs mixed into
-        // the first wave, measured about 10 % slower: the scheduler does not
-        // spread such a mix evenly over the SMs.)
-        const int slots = resident_slots();
-        long long P = slots;
-        const long long most = (p.Ns + 3) / 4;   // at least 4 slices per CTA
-        if (P > most) P = most;
-        if (P > kMaxPackedCtas) P = kMaxPackedCtas;
-        if (P < 1) P = 1;
-        p.P = (int)P;
+    const long long Wt = wbeg[c->B];
+    p.P = (int)cta_count(Wt, sm_count(dev));
+    p.S_max = slots_bound(Wmax, Wt / p.P);
+    if (p.S_max > p.P) p.S_max = p.P;
+    // first item whose start weight is >= floor(i Wt / P), for each CTA boundary i
+    p.lo.resize(p.P + 1);
+    int b = 0;
+    for (int i = 0; i <= p.P; ++i) {
+        const long long w = (long long)((__int128)i * Wt / p.P);
+        if (w >= Wt) {
+            p.lo[i] = ibeg[c->B];
+            continue;
+        }
+        while (wbeg[b + 1] <= w) ++b;
+        const int s = ragged ? b : 0;
+        const int r = seq_nres(c, s) + 1, nq = seq_nq(c, s);
+        const long long W = unit_w(nq, r);
+        const long long off = w - wbeg[b];
+        const int kh = (int)(off / W);
+        const long long rem = off - kh * W;
+        const int nri = unit_nri(r);
+        int k;
+        if (rem <= (long long)(nri - 1) * kWR) k = (int)((rem + kWR - 1) / kWR);
+        else k = nri + (int)((rem - (long long)nri * kWR + kWP - 1) / kWP);
+        p.lo[i] = ibeg[b] + kh * unit_items(nq, r) + k;
     }
-    // partial slots per unit: the residual chunks plus the most packed CTAs any unit meets
-    int per_unit = 0;
-    long long lo = 0;
-    for (int u = 0; p.Ns > 0 && u < p.units; ++u) {
-        const int spu = seq_nq(c, c->seq ? u / c->Hkv : 0) / kSlice;
-        if (spu == 0) continue;
-        const long long hi = lo + spu - 1;
-        const int first = (int)(((lo + 1) * p.P - 1) / p.Ns), last = (int)(((hi + 1) * p.P - 1) / p.Ns);
-        if (last - first + 1 > per_unit) per_unit = last - first + 1;
-        lo = hi + 1;
-    }
-    p.S_max = p.n_rc + per_unit;
     return p;
 }
 
@@ -1123,15 +1175,20 @@ Plan plan(const minikv_cache *c) {
 // the launch-wide counter of the device-state mode.
 size_t decode_counter_bytes(int B, int Hkv) { return (((size_t)B * Hkv * 4 + 4 + 255) / 256) * 256; }
 
+// Partial slots per unit for any state up to max_tokens tokens per unit: each
+// CTA share is at least kMinShare weight, so a unit of weight W meets at most
+// W / kMinShare + 2 CTAs.
+static size_t slots_for(int max_tokens) {
+    const int res_max = max_tokens < 1024 ? max_tokens : 1024;   // the ring holds at most 1024 tokens
+    const long long W = unit_w(max_tokens, res_max < 1 ? 1 : res_max);
+    long long s = W / kMinShare + 2;
+    if (s > kMaxCtas) s = kMaxCtas;
+    return (size_t)s;
+}
+
 size_t decode_workspace_bytes(int B, int Hkv, int max_tokens) {
     const size_t units = (size_t)B * Hkv;
-    const int res_max = max_tokens < 1024 ? max_tokens : 1024;   // the ring holds at most 1024 tokens
-    const size_t n_rc = (res_max + kResChunk - 1) / kResChunk + 1;
-    // every packed CTA holds at least 3 slices (the plan gives each about 4 or more)
-    const size_t spu = (size_t)max_tokens / kSlice + 1;
-    size_t per_unit = spu / 3 + 2;
-    if (per_unit > (size_t)kMaxPackedCtas) per_unit = kMaxPackedCtas;
-    return decode_counter_bytes(B, Hkv) + units * (n_rc + per_unit) * 4 * kPartStride * 4;
+    return decode_counter_bytes(B, Hkv) + units * slots_for(max_tokens) * 4 * kPartStride * 4;
 }
 
 // Extra workspace of the attention-mass variant: per unit max[4], sum[4] and the
@@ -1147,38 +1204,31 @@ size_t decode_mass_workspace_bytes(int B, int Hq, int Hkv, int max_tokens) {
 
 // Workspace bytes the next decode call on this cache state will use.
 size_t decode_call_workspace_bytes(const minikv_cache *c) {
-    const Plan p = plan(c);
+    const int dev = current_device();
+    const Plan p = plan(c, dev < 0 ? 0 : dev);
     return decode_counter_bytes(c->B, c->Hkv) + (size_t)p.units * p.S_max * 4 * kPartStride * 4;
 }
 
 namespace {
 
-template <class A>
-int launch_decode(const A &a, const Plan &p, bool with_mass, cudaStream_t stream);
-
-template <>
-int launch_decode<Args>(const Args &a, const Plan &p, bool with_mass, cudaStream_t stream) {
-    const int grid = p.units * p.n_rc + p.P;
-    if (with_mass) decode_kernel<true><<<grid, kThreads, sizeof(Smem), stream>>>(a);
-    else decode_kernel<false><<<grid, kThreads, sizeof(Smem), stream>>>(a);
-    return check_launch(with_mass ? "decode_attn_mass" : "decode_attn");
-}
-
-template <>
-int launch_decode<ArgsVar>(const ArgsVar &a, const Plan &p, bool with_mass, cudaStream_t stream) {
-    const int grid = p.units * p.n_rc + p.P;
-    if (with_mass) decode_ragged_kernel<true><<<grid, kThreads, sizeof(Smem), stream>>>(a);
-    else decode_ragged_kernel<false><<<grid, kThreads, sizeof(Smem), stream>>>(a);
-    return check_launch(with_mass ? "decode_attn_mass (ragged)" : "decode_attn (ragged)");
-}
-
-template <>
-int launch_decode<ArgsDev>(const ArgsDev &a, const Plan &p, bool with_mass, cudaStream_t stream) {
-    const int grid = p.units * p.n_rc + p.P;
-    const size_t smem = dev_smem_bytes(a.units / a.Hkv);
-    if (with_mass) decode_dev_kernel<true><<<grid, kThreads, smem, stream>>>(a);
-    else decode_dev_kernel<false><<<grid, kThreads, smem, stream>>>(a);
-    return check_launch(with_mass ? "decode_attn_mass (device state)" : "decode_attn (device state)");
+// Every decode launch is a programmatic dependent of the work before it on the
+// stream: its CTAs may be placed while the previous kernel drains, and
+// griddepcontrol.wait at their top holds them until that kernel has finished
+// and its writes are visible.
+template <class K, class A>
+int launch_pdl(K kernel, const A &a, int grid, size_t smem, cudaStream_t stream, const char *what) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaLaunchKernelEx(&cfg, kernel, a);
+    return check_launch(what);
 }
 
 int launch_mass(const Args &a, const Plan &p, float *mass, long long mass_stride, cudaStream_t stream) {
@@ -1215,15 +1265,17 @@ int decode_launch(minikv_cache *c, const uint16_t *q, const uint16_t *k_new, con
         if (seq_nres(c, b) + 1 == ring && seq_nq(c, b) + c->G > c->cap)
             return fail(MINIKV_ERR_CAPACITY, "decode_attn: flushing a key group of sequence %d would exceed cap=%d",
                         b, c->cap);
-    const Plan p = plan(c);
+    const int dev = current_device();
+    if (dev < 0) return fail(MINIKV_ERR_CUDA, "decode_attn: no current CUDA device");
+    const int arc = ensure_attr(dev);
+    if (arc) return arc;
+    const Plan p = plan(c, dev);
     const size_t cnt_bytes = decode_counter_bytes(c->B, c->Hkv);
     const size_t part_bytes = (size_t)p.units * p.S_max * 4 * kPartStride * 4;
     size_t need = cnt_bytes + part_bytes;
     if (mass) need += mass_stats_bytes(c->B, c->Hkv) + mass_scores_bytes(c->B, c->Hkv, g, p.max_n);
     if (ws == nullptr || ws_bytes < need)
         return fail(MINIKV_ERR_INVALID_ARG, "decode_attn: workspace of %zu bytes needed, %zu given", need, ws_bytes);
-    const int arc = ensure_attr();
-    if (arc) return arc;
 
     Args a;
     a.k_codes = c->k_codes; a.v_codes = c->v_codes;
@@ -1236,39 +1288,47 @@ int decode_launch(minikv_cache *c, const uint16_t *q, const uint16_t *k_new, con
     a.grid_counter = a.counters + p.units;
     a.dseq = c->dseq;
     a.part = reinterpret_cast<float *>(static_cast<char *>(ws) + cnt_bytes);
-    a.err = nullptr;
     a.stats = mass ? reinterpret_cast<float *>(static_cast<char *>(ws) + cnt_bytes + part_bytes) : nullptr;
     a.xs = mass ? reinterpret_cast<float *>(static_cast<char *>(ws) + cnt_bytes + part_bytes +
                                             mass_stats_bytes(c->B, c->Hkv))
                 : nullptr;
     a.xs_stride = (p.max_n + 3) & ~3;
     a.Hkv = c->Hkv; a.g = g; a.G = c->G; a.cap = c->cap; a.ring = ring;
-    a.n_q = c->n_packed; a.r = c->n_res + 1; a.res_start = c->res_start; a.flush = (a.r == ring);
+    a.n_q = c->n_packed; a.r = c->n_res + 1; a.res_start = c->res_start;
     a.groups_cap = c->cap / c->G;
     a.lg2G = 31 - __builtin_clz((unsigned)c->G);
-    a.units = p.units; a.n_rc = p.n_rc; a.spu = p.spu; a.P = p.P; a.S_max = p.S_max; a.Ns = p.Ns;
+    a.units = p.units; a.P = p.P; a.S_max = p.S_max;
     a.scale_log2 = sm_scale * kLog2e;
 
     int rc;
     if (c->dseq) {
         ArgsDev ad;
         static_cast<Args &>(ad) = a;
-        rc = launch_decode(ad, p, mass != nullptr, stream);
+        const size_t smem = dev_smem_bytes(c->B, p.P);
+        rc = mass ? launch_pdl(decode_dev_kernel<true>, ad, p.P, smem, stream, "decode_attn_mass (device state)")
+                  : launch_pdl(decode_dev_kernel<false>, ad, p.P, smem, stream, "decode_attn (device state)");
         if (rc) return rc;
         return mass ? launch_mass(a, p, mass, (long long)c->cap + ring, stream) : MINIKV_OK;
     } else if (c->seq) {
         ArgsVar av;
         static_cast<Args &>(av) = a;
-        av.tab.sbeg[0] = 0;
+        av.tab.ibeg[0] = 0;
         for (int b = 0; b < c->B; ++b) {
-            av.tab.n_q[b] = seq_nq(c, b);
-            av.tab.r[b] = seq_nres(c, b) + 1;
+            const int nq = seq_nq(c, b), r = seq_nres(c, b) + 1;
+            av.tab.n_q[b] = nq;
+            av.tab.r[b] = r;
             av.tab.res_start[b] = seq_rs(c, b);
-            av.tab.sbeg[b + 1] = av.tab.sbeg[b] + c->Hkv * (av.tab.n_q[b] / kSlice);
+            av.tab.ibeg[b + 1] = av.tab.ibeg[b] + c->Hkv * unit_items(nq, r);
         }
-        rc = launch_decode(av, p, mass != nullptr, stream);
+        for (int i = 0; i <= p.P; ++i) av.cta.lo[i] = p.lo[i];
+        rc = mass ? launch_pdl(decode_ragged_kernel<true>, av, p.P, sizeof(Smem), stream, "decode_attn_mass (ragged)")
+                  : launch_pdl(decode_ragged_kernel<false>, av, p.P, sizeof(Smem), stream, "decode_attn (ragged)");
     } else {
-        rc = launch_decode(a, p, mass != nullptr, stream);
+        ArgsUni au;
+        static_cast<Args &>(au) = a;
+        for (int i = 0; i <= p.P; ++i) au.cta.lo[i] = p.lo[i];
+        rc = mass ? launch_pdl(decode_kernel<true>, au, p.P, sizeof(Smem), stream, "decode_attn_mass")
+                  : launch_pdl(decode_kernel<false>, au, p.P, sizeof(Smem), stream, "decode_attn");
     }
     if (rc) return rc;
     // host-side state: append, then flush G tokens where the ring is full

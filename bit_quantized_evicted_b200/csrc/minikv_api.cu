@@ -96,8 +96,8 @@ int decode_validate(minikv_cache *c, const uint16_t *q, const uint16_t *k_new, c
     if (Hq / c->Hkv > 4) return fail(MINIKV_ERR_UNSUPPORTED, "decode_attn: more than 4 query heads per KV head");
     if (c->Gv != c->D) return fail(MINIKV_ERR_UNSUPPORTED, "decode_attn: value group Gv=%d (needs Gv = D)", c->Gv);
     if ((size_t)c->B * c->Hkv > 65535) return fail(MINIKV_ERR_UNSUPPORTED, "decode_attn: B*Hkv above 65535");
-    if ((size_t)c->B * c->Hkv * (c->cap / 32) >= (1u << 31))
-        return fail(MINIKV_ERR_UNSUPPORTED, "decode_attn: B*Hkv*cap/32 must stay below 2^31");
+    if ((size_t)c->B * c->Hkv * (c->cap / 32 + (c->R + c->G + 4) / 5) >= (1u << 31))
+        return fail(MINIKV_ERR_UNSUPPORTED, "decode_attn: B*Hkv*(cap/32 + (R+G)/5) must stay below 2^31");
     const int nb = c->dseq ? 0 : (c->seq ? c->B : 1);   // a device-resident state is checked on the device
     for (int b = 0; b < nb; ++b) {
         const int n_packed = c->seq ? c->seq[3 * b] : c->n_packed, n_res = c->seq ? c->seq[3 * b + 1] : c->n_res;

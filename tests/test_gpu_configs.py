@@ -187,6 +187,28 @@ def test_config3_4_packed_decode(wid, B, Hq, Hkv, N, steps):
         _decode_steps(wid, layer, cache, slices, B, Hq, Hkv, steps, checks)
 
 
+def test_quant_only_32k_decode():
+    """The keep-100 % (quantization only) workload at its own size: Mistral-7B GQA
+    shape, all 32768 context tokens kept (32640 packed + 128 fp16 per unit), 40
+    decode steps crossing a key-group flush at step 31, two layers, sampled
+    units.  It has the most packed tokens per unit of any workload, so the most
+    CTAs meet in each unit's split-KV merge."""
+    wid, B, Hq, Hkv, N, steps = 106, 16, 32, 8, 32768, 40
+    G, R = 32, 128
+    units = [(0, 0), (7, 3), (B - 1, Hkv - 1)]
+    for layer in (0, 1):
+        cache, k, v = _packed_cache(wid, layer, B, Hkv, N, G, R, steps)
+        assert (cache.n_packed, cache.n_res) == (32640, 128)
+        slices = {(b, h): O.SliceCache.from_kept(_np(k[b, h]), _np(v[b, h]), R, G, 128) for (b, h) in units}
+        for (b, h), sc in slices.items():
+            _check_slice(cache, b, h, sc)
+        del k, v
+        _decode_steps(wid, layer, cache, slices, B, Hq, Hkv, steps, {0, 1, 30, 31, 32, steps - 1})
+        assert cache.n_packed == 32640 + G   # one key group was flushed in every unit
+        del cache
+        torch.cuda.empty_cache()
+
+
 def test_config5_pyramid_long_prompt():
     """LLaMA2-7B shape, B=4, prompt 44000, keep from 30% (layer 0) to 5% (layer 31), W=32, G=32, R=128,
     prefill select + pack + 512 decode steps on layers 0, 15 and 31."""
