@@ -53,6 +53,10 @@ DECODE_PRESETS = {
                               head_dim=128, context=16384, keep_pct=15, G=32, Gv=128, R=128),
     "pyramid_44k_decode": dict(workload="pyramid_44k_decode", layers=32, batch=4, q_heads=32, kv_heads=32,
                                head_dim=128, context=44000, keep_pct="pyramid", G=32, Gv=128, R=128),
+    # the pyramid decode at the largest batch that fits the free HBM (sized at run time)
+    "pyramid_44k_maxbatch_decode": dict(workload="pyramid_44k_maxbatch_decode", layers=32, batch="max", q_heads=32,
+                                        kv_heads=32, head_dim=128, context=44000, keep_pct="pyramid", G=32, Gv=128,
+                                        R=128),
     # every token kept, only quantized (the KIVI-like point of the method): 32K context
     "quant_only_32k_decode": dict(workload="quant_only_32k_decode", layers=32, batch=16, q_heads=32, kv_heads=8,
                                   head_dim=128, context=32768, keep_pct=100, G=32, Gv=128, R=128),
@@ -250,7 +254,7 @@ def decode_keeps():
 
 
 def decode_config(extra=None, step_bytes=None):
-    c = {k: v for k, v in DECODE.items()}
+    c = {k: v for k, v in DECODE.items() if k != "eager"}
     keeps = decode_keeps()
     c["keep"] = keeps[0] if len(set(keeps)) == 1 else f"{keeps[0]}..{keeps[-1]} (per layer)"
     if "contexts" in DECODE:
@@ -273,20 +277,30 @@ def run_reference(args):
     per_step = max(0.05, min(0.5, 120.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
         oracle_decode_rate(per_step, threads)
-    rates, units = [], 0
+    rates, units, timed = [], 0, 0.0
     for _ in range(args.steps):
-        r, n, _ = oracle_decode_rate(per_step, threads)
+        r, n, dt = oracle_decode_rate(per_step, threads)
         rates.append(r)
         units += n
+        timed += dt
     rate = statistics.median(rates)
     v = cpu_tokens_per_s(rate)
+    per_full_step = DECODE["layers"] * DECODE["batch"] * DECODE["kv_heads"]
     sample = (f"{units} decode unit-steps (one sequence x KV head of one layer: 6553 kept tokens, 4 query heads, fp64) "
               f"over {args.steps} steps of {per_step:.2f} s on {threads} threads; tokens/s = unit-steps/s x batch / "
               f"(32 layers x 16 x 8 units)")
+    # the same config object as the GPU arm's (same workload, same timed-step bytes)
+    cfg = decode_config({"parallelism": f"replicas x{args.gpus}"},
+                        step_bytes=timed_step_bytes(args.warmup, args.steps))
     line = {"metric": METRIC, "value": v, "unit": "tokens/s", "impl": "reference", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * DECODE["batch"] / v,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": decode_config(),
+            "config": cfg,
+            # value and ms_per_step are rates scaled up from the timed sample: one full step is
+            # per_full_step unit-steps, far more than the sample holds
+            "extrapolated": {"value": True, "ms_per_step": True, "timed_seconds": timed, "unit_steps_timed": units,
+                             "unit_steps_per_full_step": per_full_step,
+                             "unit_steps_per_s": rate},
             "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": sample},
             "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -294,29 +308,59 @@ def run_reference(args):
 
 # ------------------------------------------------------------- GPU arm
 
+# The largest batch of the pyramid workload that fits the free device memory
+# (the long-prompt workload's batch is raised until HBM is full).  Every sequence
+# costs its 32 per-layer caches (sized for 512 decode steps of growth), its
+# share of the decode workspace and its step inputs / outputs; a fixed reserve
+# covers the transient of loading one sequence and the allocator's slack.
+MAXBATCH_RESERVE = 6 << 30
+MAX_SEQS = 256   # most sequences a device-state batch may hold
+
+
+def max_batch(mk, free_bytes, preset=None, steps=512, pool=8):
+    d = preset or DECODE
+    L, Hq, Hkv, G, Gv, R = d["layers"], d["q_heads"], d["kv_heads"], d["G"], d["Gv"], d["R"]
+    keeps = [keep_of(d["context"], d["keep_pct"], l, L) for l in range(L)]
+    caps = [((n + steps + 8) // G + 2) * G for n in keeps]
+    lib = mk.lib()
+    per_seq = sum(int(lib.minikv_cache_bytes(1, Hkv, 128, G, Gv, R, cap)) for cap in caps)
+    per_seq += mk.workspace_size(mk.OP_DECODE_ATTN, 1, Hq, Hkv, max(caps) + R + G)
+    per_seq += (pool + 4) * L * (Hq + 2 * Hkv) * 128 * 2 + 4 * L * Hq * 128 * 2
+    B = int((free_bytes - MAXBATCH_RESERVE) // per_seq)
+    return max(1, min(MAX_SEQS, B)), per_seq
+
+
 def make_decode_state(torch, mk, synth, device, warmup, steps):
-    L, B, Hq, Hkv = DECODE["layers"], DECODE["batch"], DECODE["q_heads"], DECODE["kv_heads"]
+    L, Hq, Hkv = DECODE["layers"], DECODE["q_heads"], DECODE["kv_heads"]
     G, Gv, R = DECODE["G"], DECODE["Gv"], DECODE["R"]
+    if DECODE["batch"] == "max":
+        free, _ = torch.cuda.mem_get_info(device)
+        DECODE["batch"], per_seq = max_batch(mk, free, steps=max(512, warmup + 2 * steps + 2))
+        DECODE["max_batch_rule"] = (f"largest batch that fits {free / 1e9:.1f} GB of free HBM at "
+                                    f"{per_seq / 1e9:.3f} GB per sequence (caches sized for 512 steps)")
+    B = DECODE["batch"]
     keeps = decode_keeps()
-    total_steps = warmup + 2 * steps + 2
-    cap_max = ((max(keeps) + total_steps) // G + 2) * G
+    total_steps = max(warmup + 2 * steps + 2, 512 if "max_batch_rule" in DECODE else 0)
+    cap_max = ((max(keeps) + total_steps + 8) // G + 2) * G
     op = mk.OP_DECODE_ATTN_MASS if DECODE.get("mass") else mk.OP_DECODE_ATTN
     ws = torch.zeros(mk.workspace_size(op, B, Hq, Hkv, cap_max + R + G), dtype=torch.uint8, device=device)
     wid = 4 if DECODE["workload"] == "mistral7b_gqa_decode" else 40 + list(DECODE_PRESETS).index(DECODE["workload"])
     caches = []
     sk = seq_keeps()
+    per_seq_load = sk is not None or "max_batch_rule" in DECODE
     for l in range(L):
         N = keeps[l]
-        cap = ((N + total_steps) // G + 2) * G
+        cap = ((N + total_steps + 8) // G + 2) * G
         c = mk.MiniKVCache(B, Hkv, cap, G=G, Gv=Gv, R=R, Hq=Hq, device=device, ws=ws)
         if not DECODE.get("eager"):
             c.set_device_state()   # per-sequence state on the GPU: steps replay from CUDA graphs
-        elif sk is not None:
+        elif per_seq_load:
             c.set_ragged()
-        if sk is not None:   # ragged: each sequence loaded into its own row with its own length
+        if per_seq_load:   # each sequence loaded into its own row (its own length for a ragged batch)
             for b in range(B):
-                kb = synth.keys_fp16((Hkv, sk[b], 128), synth.seed_of(wid, l, synth.T_K, 0, b), device)
-                vb = synth.normal_fp16((Hkv, sk[b], 128), synth.seed_of(wid, l, synth.T_V, 0, b), device)
+                n = sk[b] if sk is not None else N
+                kb = synth.keys_fp16((Hkv, n, 128), synth.seed_of(wid, l, synth.T_K, 0, b), device)
+                vb = synth.normal_fp16((Hkv, n, 128), synth.seed_of(wid, l, synth.T_V, 0, b), device)
                 mk.quant_pack_seq(c, b, kb, vb)
                 del kb, vb
             k = v = None
@@ -383,6 +427,28 @@ class LengthMirror:
                     s[1] -= self.G
 
 
+def mirror_for_preset():
+    """A LengthMirror of the current decode workload's starting lengths."""
+    sk = seq_keeps()
+    B = DECODE["batch"]
+    return LengthMirror([sk if sk is not None else [n] * B for n in decode_keeps()], DECODE["G"], DECODE["R"])
+
+
+def timed_step_bytes(warmup, steps):
+    """Algorithmic bytes per timed step of the current decode workload: the
+    mean over the timed steps, after `warmup` steps (host bookkeeping only, so
+    that the reference arm states the same config as the GPU arm)."""
+    m = mirror_for_preset()
+    L, Hkv, mass = DECODE["layers"], DECODE["kv_heads"], bool(DECODE.get("mass"))
+    for _ in range(warmup):
+        m.advance()
+    tot = 0
+    for _ in range(steps):
+        tot += sum(m.layer_bytes(l, Hkv, mass) for l in range(L))
+        m.advance()
+    return tot / max(1, steps)
+
+
 def decode_call(mk, c, q, kn, vn, out, ws, stream):
     if c.mass is not None:
         mk.decode_attn_mass(c, q, kn, vn, c.mass, out=out, ws=ws, stream=stream)
@@ -390,7 +456,7 @@ def decode_call(mk, c, q, kn, vn, out, ws, stream):
         mk.decode_attn(c, q, kn, vn, out=out, ws=ws, stream=stream)
 
 
-def run_prefill(torch, mk, synth, device):
+def run_prefill(torch, mk, synth, device, pk):
     """Prompt rows of one prefill workload: per layer select_prefill, topk_evict
     and quant_pack, each timed with CUDA events (3 warm-up layers first).  A
     layer's q, k, v are generated (untimed) just before its calls."""
@@ -444,43 +510,57 @@ def run_prefill(torch, mk, synth, device):
         layer(l, ev[l])
     sel = sum(e[0].elapsed_time(e[1]) for e in ev)
     top = sum(e[1].elapsed_time(e[2]) for e in ev)
-    pk = sum(e[2].elapsed_time(e[3]) for e in ev)
+    pk_ms = sum(e[2].elapsed_time(e[3]) for e in ev)
     fused = sum(e[3].elapsed_time(e[4]) for e in ev)
     flops = L * (2.0 * T * T * 128 * H * B + 2.0 * W * T * 128 * H * B)    # causal QK^T + PV, plus the window pass
+    tflops = flops / (sel * 1e-3) / 1e12
     del q, k, v, o
     return {"workload": PREFILL["workload"], "config": {**PREFILL, "keep": keeps[0] if len(set(keeps)) == 1 else
                                                         f"{keeps[0]}..{keeps[-1]} (per layer)"},
             "select_prefill_ms": sel, "select_prefill_ms_per_layer": sel / L,
-            "select_prefill_tflops": flops / (sel * 1e-3) / 1e12,
-            "topk_evict_ms": top, "quant_pack_ms": pk, "evict_pack_ms": fused, "layers": L}
+            "select_prefill_tflops": tflops,
+            # select_prefill per layer (flash-attention pass + window pass) against the dense bf16 peak
+            # (fp16 tensor-core rate = bf16 rate); each layer is timed alone after an L2 flush: burst peak
+            "roofline": {"bound": "tensor", "kernel": "fa_tc_kernel + window_score_kernel", "achieved": tflops,
+                         "peak": pk["bf16"], "unit": "TFLOP/s", "frac": tflops / pk["bf16"], "traffic": None,
+                         "algorithmic_flops_per_layer": flops / L, "peak_source": pk["src"] + " (bf16 burst)"},
+            "topk_evict_ms": top, "quant_pack_ms": pk_ms, "evict_pack_ms": fused, "layers": L}
 
 
-def run_gpu(args):
-    import torch
-    import torch.distributed as dist
+class GpuCtx:
+    """One process's GPU, rank and barrier for the timed regions."""
 
+    def __init__(self):
+        import torch
+        import torch.distributed as dist
+        self.torch, self.dist = torch, dist
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        torch.cuda.set_device(self.local)
+        self.device = torch.device("cuda", self.local)
+        if self.world > 1:
+            import datetime
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=self.device)
+
+    def barrier(self):
+        if self.world > 1:
+            self.dist.barrier()
+
+
+def measure_decode(ctx, args, steps, warmup, with_e2e=True):
+    """Run the current decode workload (DECODE): warm-up steps, then `steps`
+    timed steps (barrier + synchronize on both sides, max over ranks), then the
+    same number of end-to-end steps through the public API with the inputs
+    copied from pinned host memory and the outputs copied back.  Returns the
+    measurements (rank-independent fields only)."""
+    torch, device = ctx.torch, ctx.device
     from bit_quantized_evicted_b200 import minikv as mk
     from bit_quantized_evicted_b200 import synth
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
-    device = torch.device("cuda", local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=device)
-
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
-    mk.lib()
-    pk = peaks()
+    caches, ws, qin, knin, vnin, out = make_decode_state(torch, mk, synth, device, warmup, steps)
     L, B, Hkv = DECODE["layers"], DECODE["batch"], DECODE["kv_heads"]
-    caches, ws, qin, knin, vnin, out = make_decode_state(torch, mk, synth, device, args.warmup, args.steps)
-    sk = seq_keeps()
-    mirror = LengthMirror([sk if sk is not None else [n] * B for n in decode_keeps()], DECODE["G"], DECODE["R"])
+    mirror = mirror_for_preset()
     with_mass = bool(DECODE.get("mass"))
     eager = bool(DECODE.get("eager"))
     P = qin.shape[0]
@@ -500,15 +580,15 @@ def run_gpu(args):
     def step_bytes():
         return [mirror.layer_bytes(l, Hkv, with_mass) for l in range(L)]
 
-    for s in range(args.warmup):
+    for s in range(warmup):
         layer_calls(qin, knin, vnin, s % P)
         mirror.advance()
     torch.cuda.synchronize()
 
-    # Graph mode (default): the caches keep their state on the GPU, so one
-    # captured step per input-pool slot replays correctly at every later step.
-    # Timing events are recorded between replays, not inside the graphs (event
-    # nodes inside a graph would sit between the kernels and slow the step).
+    # Graph mode: the caches keep their state on the GPU, so one captured step
+    # per input-pool slot replays correctly at every later step.  Timing events
+    # are recorded between replays, not inside the graphs (event nodes inside a
+    # graph would sit between the kernels and slow the step).
     graphs = []
     if not eager:
         for p in range(P):
@@ -520,16 +600,16 @@ def run_gpu(args):
 
     # ---- device-timed region
     stream = torch.cuda.current_stream(device)
-    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(L)] for _ in range(args.steps)]
-    sev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(L)] for _ in range(steps)]
+    sev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
     nbytes = []
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier()
+    ctx.barrier()
     torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
+    with ClockSampler(ctx.local) as clk:
         t0.record(stream)
-        for s in range(args.steps):
-            p = (args.warmup + s) % P
+        for s in range(steps):
+            p = (warmup + s) % P
             nbytes.append(step_bytes())
             if eager:
                 layer_calls(qin, knin, vnin, p, evs[s])
@@ -540,86 +620,148 @@ def run_gpu(args):
             mirror.advance()
         t1.record(stream)
         torch.cuda.synchronize()
-    barrier()
+    ctx.barrier()
     ms = t0.elapsed_time(t1)
     launch_bytes = [b for sb in nbytes for b in sb]
     if eager:
-        kern_ms = [evs[s][l][0].elapsed_time(evs[s][l][1]) for s in range(args.steps) for l in range(L)]
+        kern_ms = [evs[s][l][0].elapsed_time(evs[s][l][1]) for s in range(steps) for l in range(L)]
     else:   # a replay runs the L layer launches back to back: its time / L per launch (gaps included)
-        kern_ms = [sev[s][0].elapsed_time(sev[s][1]) / L for s in range(args.steps)]
+        kern_ms = [sev[s][0].elapsed_time(sev[s][1]) / L for s in range(steps)]
     ms = max_over_ranks(ms, device)
-    tok_s = job_tokens_per_s(B, args.steps, world, ms)
+    tok_s = job_tokens_per_s(B, steps, ctx.world, ms)
     alg_bytes = sum(sum(sb) for sb in nbytes)
     mean_launch_bytes = sum(launch_bytes) / len(launch_bytes)
     mean_launch_s = statistics.mean(kern_ms) * 1e-3
-    achieved = mean_launch_bytes / mean_launch_s / 1e9
-    step_gbs = alg_bytes / (ms * 1e-3) / 1e9
+    res = {"value": tok_s, "ms_per_step": ms / steps, "step_bytes": alg_bytes / steps,
+           "hbm_gbs": alg_bytes / (ms * 1e-3) / 1e9, "mean_launch_bytes": mean_launch_bytes,
+           "mean_launch_us": mean_launch_s * 1e6, "achieved_gbs": mean_launch_bytes / mean_launch_s / 1e9,
+           "clocks": clk.summary(), "launches": L * steps * (2 if with_mass else 1), "eager": eager}
     del graphs
 
-    # ---- end to end: inputs from pinned host memory, outputs back, each step.
-    # Two buffer sets: while step s computes, a copy stream brings step s+1's
-    # inputs in and takes step s-1's outputs out (stream order and events keep
-    # each buffer's copies and its compute apart).
-    hq = qin.cpu().pin_memory()
-    hk = knin.cpu().pin_memory()
-    hv = vnin.cpu().pin_memory()
-    dq = [torch.empty_like(qin[:1]) for _ in range(2)]
-    dk = [torch.empty_like(knin[:1]) for _ in range(2)]
-    dv = [torch.empty_like(vnin[:1]) for _ in range(2)]
-    dout = [torch.empty_like(out) for _ in range(2)]
-    hout = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
-    h2d = (dq[0].numel() + dk[0].numel() + dv[0].numel()) * 2
-    d2h = out.numel() * 2
-    g_e2e = []
-    if not eager:
-        for i in range(2):
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g):
+    if with_e2e:
+        # ---- end to end: inputs from pinned host memory, outputs back, each step.
+        # Two buffer sets: while step s computes, a copy stream brings step s+1's
+        # inputs in and takes step s-1's outputs out (stream order and events keep
+        # each buffer's copies and its compute apart).
+        hq = qin.cpu().pin_memory()
+        hk = knin.cpu().pin_memory()
+        hv = vnin.cpu().pin_memory()
+        dq = [torch.empty_like(qin[:1]) for _ in range(2)]
+        dk = [torch.empty_like(knin[:1]) for _ in range(2)]
+        dv = [torch.empty_like(vnin[:1]) for _ in range(2)]
+        dout = [torch.empty_like(out) for _ in range(2)]
+        hout = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
+        h2d = (dq[0].numel() + dk[0].numel() + dv[0].numel()) * 2
+        d2h = out.numel() * 2
+        g_e2e = []
+        if not eager:
+            for i in range(2):
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g):
+                    layer_calls(dq[i], dk[i], dv[i], 0, o=dout[i])
+                g_e2e.append(g)
+        copy = torch.cuda.Stream(device)
+        in_ready = [torch.cuda.Event() for _ in range(2)]
+        done = [torch.cuda.Event() for _ in range(2)]
+        torch.cuda.synchronize()
+        ctx.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        copy.wait_stream(stream)
+        for s in range(steps):
+            i, p = s % 2, s % P
+            with torch.cuda.stream(copy):
+                dq[i].copy_(hq[p:p + 1], non_blocking=True)
+                dk[i].copy_(hk[p:p + 1], non_blocking=True)
+                dv[i].copy_(hv[p:p + 1], non_blocking=True)
+                in_ready[i].record(copy)
+            stream.wait_event(in_ready[i])
+            if eager:
                 layer_calls(dq[i], dk[i], dv[i], 0, o=dout[i])
-            g_e2e.append(g)
-    copy = torch.cuda.Stream(device)
-    in_ready = [torch.cuda.Event() for _ in range(2)]
-    done = [torch.cuda.Event() for _ in range(2)]
-    torch.cuda.synchronize()
-    barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    copy.wait_stream(stream)
-    for s in range(args.steps):
-        i, p = s % 2, s % P
-        with torch.cuda.stream(copy):
-            dq[i].copy_(hq[p:p + 1], non_blocking=True)
-            dk[i].copy_(hk[p:p + 1], non_blocking=True)
-            dv[i].copy_(hv[p:p + 1], non_blocking=True)
-            in_ready[i].record(copy)
-        stream.wait_event(in_ready[i])
-        if eager:
-            layer_calls(dq[i], dk[i], dv[i], 0, o=dout[i])
-        else:
-            g_e2e[i].replay()
-        done[i].record(stream)
-        with torch.cuda.stream(copy):
-            copy.wait_event(done[i])
-            hout[i].copy_(dout[i], non_blocking=True)
-    stream.wait_stream(copy)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    barrier()
-    del g_e2e
-    e2e_ms = e0.elapsed_time(e1)
-    e2e_ms = max_over_ranks(e2e_ms, device)
-    e2e_tok_s = job_tokens_per_s(B, args.steps, world, e2e_ms)
+            else:
+                g_e2e[i].replay()
+            done[i].record(stream)
+            with torch.cuda.stream(copy):
+                copy.wait_event(done[i])
+                hout[i].copy_(dout[i], non_blocking=True)
+        stream.wait_stream(copy)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ctx.barrier()
+        del g_e2e
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1), device)
+        res["e2e"] = {"value": job_tokens_per_s(B, steps, ctx.world, e2e_ms), "unit": "tokens/s",
+                      "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
     status_bad = sum(sum(c.status()) for c in caches)
     if status_bad:
         raise RuntimeError(f"{status_bad} sequences hit the cache capacity")
+    del caches, ws, qin, knin, vnin, out
+    torch.cuda.empty_cache()
+    return res
 
-    prefill = run_prefill(torch, mk, synth, device) if not args.no_prefill else None
+
+def launch_name(eager):
+    return ("eager: one Python call per layer" if eager else
+            "one CUDA graph replay per step (all layer calls captured, state on the GPU)")
+
+
+def select_preset(name, args):
+    DECODE.clear()
+    DECODE.update(DECODE_PRESETS[name])
+    if args.layers is not None and name == args.workload:
+        DECODE["layers"] = args.layers
+    if args.mass and name == args.workload:
+        DECODE["mass"] = True
+    if args.launch == "eager" or (args.launch == "auto" and AUTO_EAGER and "contexts" not in DECODE
+                                  and DECODE["batch"] != "max"):
+        DECODE["eager"] = True
+
+
+# Workloads measured as compact sub-lines of the default run (so that their
+# numbers are driver-observed): LLaMA2-13B MHA decode and the pyramid (B = 4).
+SUBLINE_WORKLOADS = ("llama2_13b_decode", "pyramid_44k_decode")
+SUBLINE_STEPS = 16
+# --launch auto: one Python call per layer for uniform batches (its kernel is
+# faster than the device-state kernel a graph replays, and the host keeps up),
+# graph replay for ragged batches (the per-call host cost is higher there)
+AUTO_EAGER = True
+
+
+def run_gpu(args):
+    from bit_quantized_evicted_b200 import minikv as mk
+
+    ctx = GpuCtx()
+    torch = ctx.torch
+    mk.lib()
+    pk = peaks()
+    main = measure_decode(ctx, args, args.steps, args.warmup)
+    B, L = DECODE["batch"], DECODE["layers"]
+    cfg_extra = {"parallelism": f"replicas x{ctx.world}"}
+    main_cfg = decode_config(cfg_extra, step_bytes=main["step_bytes"])
+    eager = main["eager"]
+
+    prefill = run_prefill(torch, mk, __import__("bit_quantized_evicted_b200.synth", fromlist=["x"]), ctx.device, pk) \
+        if not args.no_prefill else None
     if prefill:
-        prefill["tensor_frac_of_bf16_peak"] = prefill["select_prefill_tflops"] / pk["bf16"]
+        prefill["tensor_frac_of_bf16_peak"] = prefill["roofline"]["frac"]
+
+    sublines = {}
+    if args.workload == "mistral7b_gqa_decode" and not args.no_sublines and not args.mass and args.layers is None:
+        for name in SUBLINE_WORKLOADS:
+            select_preset(name, args)
+            r = measure_decode(ctx, args, SUBLINE_STEPS, 3, with_e2e=False)
+            sublines[name] = {"value": r["value"], "unit": "tokens/s", "ms_per_step": r["ms_per_step"],
+                              "steps": SUBLINE_STEPS, "warmup": 3, "hbm_gbs": r["hbm_gbs"],
+                              "roofline": {"bound": "hbm", "kernel": "decode_kernel", "achieved": r["achieved_gbs"],
+                                           "peak": pk["hbm"], "unit": "GB/s", "frac": r["achieved_gbs"] / pk["hbm"],
+                                           "mean_launch_us": r["mean_launch_us"]},
+                              "launch": launch_name(r["eager"]),
+                              "config": decode_config(cfg_extra, step_bytes=r["step_bytes"])}
+        select_preset(args.workload, args)
 
     cpu = None
-    if (rank == 0 and world == 1 and not args.no_cpu_baseline and DECODE["workload"] == "mistral7b_gqa_decode"
-            and not DECODE.get("mass")):
+    if (ctx.rank == 0 and ctx.world == 1 and not args.no_cpu_baseline and args.workload == "mistral7b_gqa_decode"
+            and not args.mass):
         threads = os.cpu_count() or 1
         rate, n, dt = oracle_decode_rate(args.cpu_seconds, threads)
         cpu = {"value": cpu_tokens_per_s(rate), "unit": "tokens/s", "cores": threads, "kind": "oracle",
@@ -630,33 +772,31 @@ def run_gpu(args):
     csrc = os.path.join(ROOT, "bit_quantized_evicted_b200", "csrc")
     traffic, traffic_note = recorded_traffic(
         "decode_kernel", [os.path.join(csrc, "decode.cu"), os.path.join(csrc, "common.cuh")])
-    if DECODE.get("mass"):
+    if args.mass:
         traffic, traffic_note = None, "no capture of the attention-mass variant (decode_kernel<true> + mass_kernel)"
-    if rank == 0:
+    if ctx.rank == 0:
         line = {
-            "metric": METRIC, "value": tok_s, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "u2+f16 (2-bit codes, fp16 scales/residual, fp32 accumulate)",
-            "data": "synthetic",
-            "config": decode_config({"parallelism": f"replicas x{world}",
-                                     "launch": "eager: one Python call per layer" if eager else
-                                     "one CUDA graph replay per step (32 captured layer calls, state on the GPU)"},
-                                    step_bytes=alg_bytes / args.steps),
-            "hbm_gbs": step_gbs, "hbm_frac_of_peak": step_gbs / pk["hbm"],
-            "roofline": {"bound": "hbm", "kernel": "decode_kernel", "achieved": achieved, "peak": pk["hbm"],
-                         "unit": "GB/s", "frac": achieved / pk["hbm"], "traffic": traffic,
-                         "algorithmic_bytes_per_launch": mean_launch_bytes,
-                         "mean_launch_us": mean_launch_s * 1e6, "peak_source": pk["src"],
+            "metric": METRIC, "value": main["value"], "unit": "tokens/s", "n_gpus": ctx.world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": main["ms_per_step"], "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None,
+            "dtype": "u2+f16 (2-bit codes, fp16 scales/residual, fp32 accumulate)", "data": "synthetic",
+            "config": main_cfg, "launch": launch_name(eager),
+            "hbm_gbs": main["hbm_gbs"], "hbm_frac_of_peak": main["hbm_gbs"] / pk["hbm"],
+            "roofline": {"bound": "hbm", "kernel": "decode_kernel", "achieved": main["achieved_gbs"],
+                         "peak": pk["hbm"], "unit": "GB/s", "frac": main["achieved_gbs"] / pk["hbm"],
+                         "traffic": traffic, "algorithmic_bytes_per_launch": main["mean_launch_bytes"],
+                         "mean_launch_us": main["mean_launch_us"], "peak_source": pk["src"],
                          "traffic_source": traffic_note},
             "cpu_baseline": cpu,
-            "e2e": {"value": e2e_tok_s, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-            "gpu_launches": L * args.steps * (2 if DECODE.get("mass") else 1),
-            "clocks": clk.summary(),
+            "e2e": main["e2e"],
+            "gpu_launches": main["launches"],
+            "clocks": main["clocks"],
             "prefill": prefill,
+            "sublines": sublines or None,
         }
         print(json.dumps(line), flush=True)
-    if world > 1:
-        dist.destroy_process_group()
+    if ctx.world > 1:
+        ctx.dist.destroy_process_group()
 
 
 def main():
@@ -672,8 +812,8 @@ def main():
                     help="decode workload (the default one carries the bench line's target)")
     ap.add_argument("--launch", default="auto", choices=["auto", "graph", "eager"],
                     help="graph: state on the GPU, one captured CUDA graph replayed per step; eager: one Python "
-                         "call per layer, host-side state; auto: graph for ragged batches (eager is host-bound "
-                         "there), eager otherwise (its kernel is a little faster)")
+                         "call per layer, host-side state; auto: eager for uniform batches, graph for ragged and "
+                         "max-batch ones")
     ap.add_argument("--mass", action="store_true",
                     help="decode with minikv_decode_attn_mass (H2O-style running attention mass per token)")
     ap.add_argument("--prefill-workload", default="llama2_7b_prefill_select", choices=list(PREFILL_PRESETS))
@@ -681,17 +821,12 @@ def main():
                     help="decode layers (fewer only for small profiling runs; default: the workload's)")
     ap.add_argument("--prefill-layers", type=int, default=None,
                     help="prefill layers (fewer only for small profiling runs; default: the workload's)")
+    ap.add_argument("--no-sublines", action="store_true",
+                    help="skip the compact LLaMA2-13B and pyramid decode sub-lines of the default run")
     args = ap.parse_args()
-    DECODE.clear()
-    DECODE.update(DECODE_PRESETS[args.workload])
+    select_preset(args.workload, args)
     PREFILL.clear()
     PREFILL.update(PREFILL_PRESETS[args.prefill_workload])
-    if args.layers is not None:
-        DECODE["layers"] = args.layers
-    if args.mass:
-        DECODE["mass"] = True
-    if args.launch == "eager" or (args.launch == "auto" and "contexts" not in DECODE):
-        DECODE["eager"] = True
     if args.prefill_layers is not None:
         PREFILL["layers"] = args.prefill_layers
     if args.warmup < 3:

@@ -200,10 +200,19 @@ __device__ __forceinline__ int part_P(const ArgsDev &) { return dev_tab().P; }
 
 // ---- positions in the work list
 
-// the CTA whose item range holds flat item x: largest c with cta_lo(c) <= x
+// The CTA whose item range holds flat item x: largest c with cta_lo(c) <= x.
+// The ranges have equal weight and an item's weight is 7/8 .. 1 of the mean,
+// so x P / items lands within a step or two of c; the walk from there reads
+// one table entry at a time (the same for the whole warp: kernel-parameter
+// reads with a per-thread index would be serialized).
 template <class A>
 __device__ __forceinline__ int cta_of_item(const A &a, int x) {
-    return seq_search(part_P(a), x, [&](int c) { return cta_lo(a, c); });
+    const int P = part_P(a), n = cta_lo(a, P);
+    int c = (int)floor((double)x * (double)P / (double)n);
+    c = c < 0 ? 0 : (c >= P ? P - 1 : c);
+    while (c > 0 && cta_lo(a, c) > x) --c;
+    while (c < P - 1 && cta_lo(a, c + 1) <= x) ++c;
+    return c;
 }
 
 // Segment info for the unit holding flat item x (one thread).
@@ -515,13 +524,6 @@ __device__ void run_cta(const A &a, Smem &sm, int c) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g_ = lane >> 2, t_ = lane & 3;
     const int xlo = cta_lo(a, c), xhi = cta_lo(a, c + 1);
-    if (tid == 0) {
-        sm.zero = make_uint4(0, 0, 0, 0);
-        sm.next = xlo + kWarps * (kStages - 1);   // the first kStages-1 items of each warp are fixed
-        seg_info(a, xlo, xhi, sm.seg);
-    }
-    __syncthreads();
-
     const uint32_t st0 = smem_addr(&sm.stage[warp][0][0]);
     const uint32_t qb0 = smem_addr(&sm.qbuf[warp][0][0]);
     const uint32_t zero_addr = smem_addr(&sm.zero);
@@ -567,7 +569,16 @@ __device__ void run_cta(const A &a, Smem &sm, int c) {
         ++nclaim;
     };
 #pragma unroll
-    for (int s = 0; s < kStages - 1; ++s) issue_next();
+    for (int s = 0; s < kStages - 1; ++s) issue_next();   // the first copies go out before any set-up
+
+    // set-up of the first segment while they are in flight (the dynamic claims
+    // start after the barrier below)
+    if (tid == 0) {
+        sm.zero = make_uint4(0, 0, 0, 0);
+        sm.next = xlo + kWarps * (kStages - 1);   // the first kStages-1 items of each warp are fixed
+        seg_info(a, xlo, xhi, sm.seg);
+    }
+    __syncthreads();
 
     // ---- consumer constants of this lane
     const float sl2 = a.scale_log2, sl2w = a.scale_log2 * kScoreUnit;

@@ -209,6 +209,45 @@ def test_quant_only_32k_decode():
         torch.cuda.empty_cache()
 
 
+def test_pyramid_max_batch_decode():
+    """The long-prompt pyramid workload at the largest batch that fits the free
+    HBM (the bench's own sizing rule), in the launch configuration the bench
+    times (per-sequence state on the GPU): layer 0 (keep 13200 of 44000), every
+    sequence loaded, 3 decode steps, sampled units against the oracle."""
+    import bench
+    wid, H, T, G, R, steps = 107, 32, 44000, 32, 128, 3
+    free, _ = torch.cuda.mem_get_info()
+    B, _ = bench.max_batch(mk, free, preset=bench.DECODE_PRESETS["pyramid_44k_maxbatch_decode"])
+    assert B >= 64   # ~0.75 GB per sequence for all 32 layers: well over 64 fit in 180 GB
+    N = O.pyramid_keep(T, 0, 32)
+    cap = ((N + 512 + 8) // G + 2) * G
+    cache = mk.MiniKVCache(B, H, cap, G=G, R=R, Hq=H).set_device_state()
+    units = [(0, 0), (B // 2, 17), (B - 1, H - 1)]
+    slices = {}
+    for b in range(B):
+        kb = synth.keys_fp16((H, N, 128), synth.seed_of(wid, 0, synth.T_K, 0, b), DEV)
+        vb = synth.normal_fp16((H, N, 128), synth.seed_of(wid, 0, synth.T_V, 0, b), DEV)
+        mk.quant_pack_seq(cache, b, kb, vb)
+        for (ub, h) in units:
+            if ub == b:
+                slices[(b, h)] = O.SliceCache.from_kept(_np(kb[h]), _np(vb[h]), R, G, 128)
+        del kb, vb
+    for s in range(steps):
+        q, kn, vn = _step_inputs(wid, 0, s, B, H, H)
+        out = mk.decode_attn(cache, q, kn, vn)
+        outn, qn, knn, vnn = out.float().cpu().numpy(), _np(q), _np(kn), _np(vn)
+        for (b, h), sc in slices.items():
+            ref = sc.step(qn[b, h:h + 1], knn[b, h], vnn[b, h], TAU)
+            err = float(np.max(np.abs(outn[b, h:h + 1] - ref)))
+            assert err <= ATOL, (s, b, h, err)
+    torch.cuda.synchronize()
+    assert cache.status() == [0] * B
+    for (b, h), sc in slices.items():
+        assert cache.seq_state(b)[:2] == (sc.n_q, sc.r)
+    del cache
+    torch.cuda.empty_cache()
+
+
 def test_config5_pyramid_long_prompt():
     """LLaMA2-7B shape, B=4, prompt 44000, keep from 30% (layer 0) to 5% (layer 31), W=32, G=32, R=128,
     prefill select + pack + 512 decode steps on layers 0, 15 and 31."""
