@@ -14,6 +14,10 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libminikv.so")
+# The same library with the flash-attention pipeline's bounded waits cut to one
+# poll: its waits give up while their copies are in flight, which exercises the
+# abort path (drain, status word) without any fault.  Only the tests load it.
+WAIT_PROBE_LIB = os.path.join(PKG, "libminikv_waitprobe.so")
 SOURCES = ["minikv_api.cu", "pack.cu", "prefill.cu", "topk.cu", "decode.cu", "decode_static.cu"]
 HEADERS = ["common.cuh", "tc.cuh"]
 NVCC = os.environ.get("NVCC", "nvcc")
@@ -45,19 +49,25 @@ def build(force: bool = False, ptxas_verbose: bool = False) -> str:
             if ptxas_verbose:
                 cmd += ["-Xptxas", "-v"]
             jobs.append(cmd)
+    probe_src = os.path.join(CSRC, "prefill.cu")
+    probe_obj = os.path.join(BUILD, "prefill_waitprobe.o")
+    if force or _stale(probe_obj, [probe_src, *hdrs]):
+        jobs.append([NVCC, *FLAGS, "-DMINIKV_WAIT_LIMIT=1", "-c", probe_src, "-o", probe_obj])
     with cf.ThreadPoolExecutor(max_workers=min(8, max(1, len(jobs)))) as ex:
         for res in ex.map(lambda c: subprocess.run(c, capture_output=True, text=True), jobs):
             if res.returncode != 0:
                 raise RuntimeError(f"nvcc failed:\n{res.stdout}\n{res.stderr}")
             if ptxas_verbose:
                 print(res.stderr)
-    if force or jobs or _stale(LIB, objs):
-        tmp = LIB + f".tmp{os.getpid()}"
-        cmd = [NVCC, "-shared", "-gencode", "arch=compute_100a,code=sm_100a", "-o", tmp, *objs, "-lcudart"]
-        res = subprocess.run(cmd, capture_output=True, text=True)
-        if res.returncode != 0:
-            raise RuntimeError(f"link failed:\n{res.stdout}\n{res.stderr}")
-        os.replace(tmp, LIB)
+    probe_objs = [probe_obj if o.endswith(os.sep + "prefill.o") else o for o in objs]
+    for lib, parts in ((LIB, objs), (WAIT_PROBE_LIB, probe_objs)):
+        if force or jobs or _stale(lib, parts):
+            tmp = lib + f".tmp{os.getpid()}"
+            cmd = [NVCC, "-shared", "-gencode", "arch=compute_100a,code=sm_100a", "-o", tmp, *parts, "-lcudart"]
+            res = subprocess.run(cmd, capture_output=True, text=True)
+            if res.returncode != 0:
+                raise RuntimeError(f"link failed:\n{res.stdout}\n{res.stderr}")
+            os.replace(tmp, lib)
     return LIB
 
 

@@ -29,6 +29,7 @@ int select_launch(const float *scores, int B, int Hkv, int T, int W, int keep, i
 int prefill_launch(const uint16_t *q, const uint16_t *k, const uint16_t *v, int B, int Hq, int Hkv, int T, int W,
                    float sm_scale, uint16_t *o, float *scores, void *ws, cudaStream_t stream);
 size_t prefill_workspace_bytes(int B, int Hq, int W);
+size_t prefill_lse_bytes(int B, int Hq, int W);
 int topk_launch(const float *scores, const uint16_t *k, const uint16_t *v, int B, int Hkv, int T, int W, int keep,
                 int32_t *idx, uint16_t *k_kept, uint16_t *v_kept, cudaStream_t stream);
 int decode_launch(minikv_cache *c, const uint16_t *q, const uint16_t *k_new, const uint16_t *v_new, int Hq,
@@ -228,6 +229,22 @@ int minikv_select_prefill(const uint16_t *q, const uint16_t *k, const uint16_t *
     if (ws_bytes < need)
         return fail(MINIKV_ERR_INVALID_ARG, "select_prefill: workspace of %zu bytes needed, %zu given", need, ws_bytes);
     return prefill_launch(q, k, v, B, Hq, Hkv, T, W, sm_scale, o, scores, ws, static_cast<cudaStream_t>(stream));
+}
+
+int minikv_select_prefill_status(const void *ws, size_t ws_bytes, int B, int Hq, int W, void *stream,
+                                 unsigned *status) {
+    g_err[0] = 0;
+    if (!ws || !status) return fail(MINIKV_ERR_INVALID_ARG, "select_prefill_status: null pointer");
+    if (B < 1 || Hq < 1 || W < 1) return fail(MINIKV_ERR_INVALID_ARG, "select_prefill_status: B=%d Hq=%d W=%d", B, Hq, W);
+    if (ws_bytes < prefill_workspace_bytes(B, Hq, W))
+        return fail(MINIKV_ERR_INVALID_ARG, "select_prefill_status: workspace of %zu bytes is smaller than the call's",
+                    ws_bytes);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const char *word = static_cast<const char *>(ws) + prefill_lse_bytes(B, Hq, W);
+    cudaError_t e = cudaMemcpyAsync(status, word, sizeof(unsigned), cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return fail(MINIKV_ERR_CUDA, "select_prefill_status: %s", cudaGetErrorString(e));
+    return MINIKV_OK;
 }
 
 int minikv_topk_evict(const float *scores, const uint16_t *k, const uint16_t *v, int B, int Hkv, int T, int D, int W,

@@ -77,21 +77,31 @@ struct FaSmem {
     uint16_t v[kVStages][2][kTileN * 64];   // [stage][64-wide d block]: MN-major B of P V
     uint64_t q_full, k_full[kKStages], k_empty[kKStages], v_full[kVStages], v_empty[kVStages];
     uint64_t s_full[2], p_full[2], o_done[2];
+    uint64_t drain;   // the MMA issuer's last commit, waited on before tensor memory is freed
     uint32_t tmem_base;
     int abort;
 };
 
 struct FaArgs {
-    float *lse2;   // [B, Hq, W] window rows, log2 domain
+    float *lse2;        // [B, Hq, W] window rows, log2 domain
+    unsigned *status;   // bit 0: a bounded wait expired in some CTA (its outputs are not valid)
     int Hq, Hkv, T, W, nqt;
     float scale_log2;
 };
+
+// Polls of an mbarrier before a wait of the pipeline gives up (seconds at the
+// default).  A build with a tiny limit makes the waits run out while the copies
+// and MMAs they wait for are still in flight: the abort path below then drains
+// them and the status word reports the expiry.
+#ifndef MINIKV_WAIT_LIMIT
+#define MINIKV_WAIT_LIMIT (1u << 26)
+#endif
 
 // Bounded wait shared by a CTA: once any wait times out, every later wait
 // returns false at once so all roles reach the final barrier.
 __device__ __forceinline__ bool fa_wait(FaSmem &s, uint64_t *bar, uint32_t parity) {
     if (*reinterpret_cast<volatile int *>(&s.abort)) return false;
-    if (mbar_wait(bar, parity)) return true;
+    if (mbar_wait(bar, parity, MINIKV_WAIT_LIMIT)) return true;
     *reinterpret_cast<volatile int *>(&s.abort) = 1;
     return false;
 }
@@ -137,6 +147,7 @@ __global__ void __launch_bounds__(kFaThreads, 1)
             mbar_init(&s.p_full[i], 128);
             mbar_init(&s.o_done[i], 1);
         }
+        mbar_init(&s.drain, 1);
         s.abort = 0;
         fence_mbar_init();
     }
@@ -155,25 +166,39 @@ __global__ void __launch_bounds__(kFaThreads, 1)
             mbar_arrive_expect_tx(&s.q_full, 2 * kTileM * 128);
             tc::tma_load_3d(s.q[0], &map_q, 0, qt * kTileM, bh, &s.q_full);
             tc::tma_load_3d(s.q[1], &map_q, 64, qt * kTileM, bh, &s.q_full);
+            int issued = 0;
             for (int j = 0; j < nkb; ++j) {
                 const int ks = j % kKStages;
                 if (j >= kKStages && !fa_wait(s, &s.k_empty[ks], (j / kKStages - 1) & 1)) break;
                 mbar_arrive_expect_tx(&s.k_full[ks], 2 * kTileN * 128);
                 tc::tma_load_3d(s.k[ks][0], &map_k, 0, j * kTileN, kvh, &s.k_full[ks]);
                 tc::tma_load_3d(s.k[ks][1], &map_k, 64, j * kTileN, kvh, &s.k_full[ks]);
+                issued = j + 1;
+            }
+            if (*reinterpret_cast<volatile int *>(&s.abort)) {
+                // a wait gave up: let the loads this thread queued land before the CTA exits
+                // (each stage holds at most one unconsumed load; waits on a finished phase return at once)
+                mbar_wait(&s.q_full, 0);
+                for (int j = issued > kKStages ? issued - kKStages : 0; j < issued; ++j)
+                    mbar_wait(&s.k_full[j % kKStages], (j / kKStages) & 1);
             }
         }
         __syncwarp();
     } else if (warp == 2) {
         // ---------------- V producer (its own thread: a V slot frees later than a K slot)
         if (lane == 0) {
+            int issued = 0;
             for (int j = 0; j < nkb; ++j) {
                 const int vs = j % kVStages;
                 if (j >= kVStages && !fa_wait(s, &s.v_empty[vs], (j / kVStages - 1) & 1)) break;
                 mbar_arrive_expect_tx(&s.v_full[vs], 2 * kTileN * 128);
                 tc::tma_load_3d(s.v[vs][0], &map_v, 0, j * kTileN, kvh, &s.v_full[vs]);
                 tc::tma_load_3d(s.v[vs][1], &map_v, 64, j * kTileN, kvh, &s.v_full[vs]);
+                issued = j + 1;
             }
+            if (*reinterpret_cast<volatile int *>(&s.abort))
+                for (int j = issued > kVStages ? issued - kVStages : 0; j < issued; ++j)
+                    mbar_wait(&s.v_full[j % kVStages], (j / kVStages) & 1);
         }
         __syncwarp();
     } else if (warp == 1) {
@@ -228,6 +253,10 @@ __global__ void __launch_bounds__(kFaThreads, 1)
                     tc::commit(&s.k_empty[ks]);
                 }
             }
+            // every MMA this thread issued has finished with shared and tensor memory
+            // before the CTA frees them (on the abort path too)
+            tc::commit(&s.drain);
+            mbar_wait(&s.drain, 0);
         }
         __syncwarp();
     } else {
@@ -360,6 +389,7 @@ __global__ void __launch_bounds__(kFaThreads, 1)
     __syncthreads();
     tc::fence_after_sync();
     if (warp == 1) tc::tmem_dealloc(tmem, 512);
+    if (tid == 0 && s.abort) atomicOr(a.status, 1u);
 }
 
 // ---------------------------------------------------------------- kernel 2
@@ -492,7 +522,10 @@ int make_map(CUtensorMap *m, const void *base, int rows, int planes, const char 
 
 }  // namespace
 
-size_t prefill_workspace_bytes(int B, int Hq, int W) { return ((size_t)B * Hq * W * 4 + 255) / 256 * 256; }
+// Workspace: the window rows' log-sum-exp [B, Hq, W] fp32, then a 256-byte
+// block whose first word is the call's status (see minikv_select_prefill_status).
+size_t prefill_lse_bytes(int B, int Hq, int W) { return ((size_t)B * Hq * W * 4 + 255) / 256 * 256; }
+size_t prefill_workspace_bytes(int B, int Hq, int W) { return prefill_lse_bytes(B, Hq, W) + 256; }
 
 int prefill_launch(const uint16_t *q, const uint16_t *k, const uint16_t *v, int B, int Hq, int Hkv, int T, int W,
                    float sm_scale, uint16_t *o, float *scores, void *ws, cudaStream_t stream) {
@@ -503,6 +536,9 @@ int prefill_launch(const uint16_t *q, const uint16_t *k, const uint16_t *v, int 
         return rc;
     FaArgs fa;
     fa.lse2 = static_cast<float *>(ws);
+    fa.status = reinterpret_cast<unsigned *>(static_cast<char *>(ws) + prefill_lse_bytes(B, Hq, W));
+    if (cudaMemsetAsync(fa.status, 0, sizeof(unsigned), stream) != cudaSuccess)
+        return check_launch("select_prefill: clearing the status word");
     fa.Hq = Hq; fa.Hkv = Hkv; fa.T = T; fa.W = W;
     fa.nqt = (T + kTileM - 1) / kTileM;
     fa.scale_log2 = sm_scale * kLog2e;

@@ -47,6 +47,7 @@ _SIGS = {
     "minikv_quant_pack_seq": (_I, [ctypes.POINTER(CacheStruct), _I, _P, _P, _I, _P]),
     "minikv_evict_pack_seq": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, ctypes.POINTER(CacheStruct), _I, _P]),
     "minikv_select_prefill": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P, _Z, _P]),
+    "minikv_select_prefill_status": (_I, [_P, _Z, _I, _I, _I, _P, ctypes.POINTER(ctypes.c_uint)]),
     "minikv_topk_evict": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _Z, _P]),
     "minikv_evict_pack": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, ctypes.POINTER(CacheStruct), _P]),
     "minikv_decode_attn": (_I, [ctypes.POINTER(CacheStruct), _P, _P, _P, _I, _F, _P, _P, _Z, _P]),
@@ -275,6 +276,16 @@ def select_prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, W: int, sm
         _dev(scores, torch.float32, "scores"), _dev(ws, torch.uint8, "ws"), ws.numel(),
         _stream(stream, q.device)))
     return o, scores
+
+
+def select_prefill_status(ws: torch.Tensor, B: int, Hq: int, W: int, stream=None, library=None) -> int:
+    """Status word of the last select_prefill on `ws` (synchronizes the stream):
+    0 = finished, bit 0 = a bounded wait in the flash-attention pass expired."""
+    st = ctypes.c_uint(0)
+    L = library or lib()
+    _check(L.minikv_select_prefill_status(_dev(ws, torch.uint8, "ws"), ws.numel(), B, Hq, W,
+                                          _stream(stream, ws.device), ctypes.byref(st)))
+    return int(st.value)
 
 
 def topk_evict(scores: torch.Tensor, k: torch.Tensor, v: torch.Tensor, W: int, keep: int,

@@ -189,7 +189,8 @@ MINIKV_API int minikv_quant_pack_seq(minikv_cache *c, int b, const uint16_t *k, 
  * the window rows' probabilities from it and sums them per key.
  *   sm_scale > 0 (the usual 1/sqrt(D)).
  *   ws: device scratch of minikv_workspace_size(MINIKV_OP_SELECT_PREFILL, ...)
- *       bytes, no initial contents required.
+ *       bytes, no initial contents required; it also holds the call's status
+ *       word (minikv_select_prefill_status).
  * Errors: INVALID_ARG (null, W < 1, W > T, Hq % Hkv, sm_scale <= 0, ws too
  * small), UNSUPPORTED (D != 128), CUDA (tensor-map encoding or launch failed).
  */
@@ -197,6 +198,23 @@ MINIKV_API int minikv_select_prefill(const uint16_t *q, const uint16_t *k, const
                           int B, int Hq, int Hkv, int T, int D, int W, float sm_scale,
                           uint16_t *o, float *scores, void *ws, size_t ws_bytes,
                           void *stream);
+
+/*
+ * minikv_select_prefill_status -- did the last minikv_select_prefill on this
+ * workspace finish its work?  The flash-attention pass waits on its own copies
+ * and tensor-core operations with bounded waits; if a wait gives up (a copy
+ * that never lands), the CTA drains what it started, skips its outputs and
+ * sets bit 0 of a status word in `ws`, instead of hanging or trapping.
+ * minikv_select_prefill clears the word on its stream before its kernels.
+ * Source: none on the pages (failure reporting of this library).
+ *   ws, ws_bytes, B, Hq, W: as passed to that minikv_select_prefill.
+ *   *status (host): 0 = every CTA finished; bit 0 = a bounded wait expired, the
+ *   call's o / scores are not valid.
+ * Queues a 4-byte device-to-host copy on `stream` and synchronizes the stream.
+ * Errors: INVALID_ARG (null, shape, ws smaller than the call's), CUDA.
+ */
+MINIKV_API int minikv_select_prefill_status(const void *ws, size_t ws_bytes, int B, int Hq, int W, void *stream,
+                                            unsigned *status);
 
 /*
  * minikv_topk_evict -- adaptive KV: keep the tokens that matter.

@@ -116,8 +116,19 @@ def test_prefill_and_topk_argument_errors():
     assert L.minikv_topk_evict(p, p, p, 1, 4, 512, 96, 32, 64, p, p, p, None, 0, None) == mk.ERR_UNSUPPORTED
 
 
+def test_select_prefill_status_argument_errors():
+    L = mk.lib()
+    st = ctypes.c_uint(0)
+    p = ctypes.c_void_p(1 << 20)
+    assert L.minikv_select_prefill_status(None, 4352, 1, 32, 32, None, ctypes.byref(st)) == mk.ERR_INVALID_ARG
+    assert L.minikv_select_prefill_status(p, 4352, 1, 32, 32, None, None) == mk.ERR_INVALID_ARG
+    assert L.minikv_select_prefill_status(p, 4351, 1, 32, 32, None, ctypes.byref(st)) == mk.ERR_INVALID_ARG
+    assert L.minikv_select_prefill_status(p, 4352, 0, 32, 32, None, ctypes.byref(st)) == mk.ERR_INVALID_ARG
+
+
 def test_workspace_sizes():
-    assert mk.workspace_size(mk.OP_SELECT_PREFILL, 1, 32, 32, 4096, 128, 32) == 4096
+    # window rows' log-sum-exp (32 heads x 32 rows x 4 B), then the 256-byte status block
+    assert mk.workspace_size(mk.OP_SELECT_PREFILL, 1, 32, 32, 4096, 128, 32) == 4096 + 256
     assert mk.workspace_size(mk.OP_TOPK_EVICT, 1, 32, 32, 4096, 128, 32) == 0
     assert mk.workspace_size(mk.OP_DECODE_ATTN, 16, 32, 8, 6656 + 160, 128) > 16 * 8 * 4
 
