@@ -8,7 +8,9 @@
 //   * residual items: 5 fp16 residual tokens each (the new token included), and
 //   * packed items:   32 packed tokens each (one slice of one key group).
 // The items of all units are laid end to end and cut, by weight (packed 8,
-// residual 7: their measured costs), into one contiguous range per SM.  One
+// residual 7: their measured costs; 256 more at each unit boundary, for the
+// extra segment end and merge it costs the CTA whose range crosses it), into
+// one contiguous range per SM.  One
 // CTA of 16 warps runs on each SM.  Its warps claim the items of its range one
 // at a time from a shared-memory counter (so warps the scheduler favours simply
 // take more items, and all finish together) and stream them through per-warp
@@ -29,8 +31,9 @@
 //     of q_h,c s_c 2^-p_c, column 2h+1 the exact remainder ("lo"), so the lane
 //     that owns head h holds both parts of its score (no shuffle) and every
 //     (token, head) probability is computed once;
-//   the key zero-point term sum_c q_c z_c is one mma per 16 channels (A = the
-//     zero row broadcast to all rows, B = q);
+//   the key zero-point term sum_c q_c z_c takes two mma: A rows are (head,
+//     16-channel chunk) of q, B columns are chunks of the zero row, and the
+//     term of a head is the sum of four diagonal entries (two shuffles);
 //   output O^T[ch, n] = sum_t code_{t,ch} 2^(p-24) P'[t, n], P' = p_t v_scale_t
 //     split hi / lo the same way and moved into the B layout by movmatrix;
 //     out_ch = (O^T[ch, 2h] + O^T[ch, 2h+1]) 2^(24-p) + sum_t p_t v_zero_t.
@@ -45,6 +48,7 @@
 // with.
 #include <math.h>
 
+#include <atomic>
 #include <mutex>
 #include <vector>
 
@@ -61,7 +65,9 @@ constexpr int kResTok = 5;           // residual tokens per residual item
 constexpr int kStages = 3;           // per-warp pipeline depth
 constexpr int kStageBytes = 2688;    // one packed item (a residual item takes 2560)
 constexpr int kWP = 8, kWR = 7;      // partition weights of a packed / residual item (measured cost ratio)
-constexpr int kMinShare = 8 * kWP;   // least weight per CTA
+constexpr int kWU = 256;             // partition weight of a unit boundary: the extra segment end and merge
+                                     // that a CTA whose range crosses into a new unit pays
+constexpr int kMinShare = kWU + 8 * kWP;   // least weight per CTA (a range always holds an item start)
 constexpr int kPartStride = 132;     // floats per (unit, slot, head): y[128], m, l
 constexpr int kMaxCtas = 512;
 constexpr float kLazy = 8.f;         // log2 headroom before a head's reference max moves
@@ -107,6 +113,7 @@ struct Args {
     int xs_stride;
     int Hkv, g, G, cap, ring;
     int n_q, r, res_start;    // uniform batch: every sequence's lengths (r counts the new token)
+    int det;                  // 1: items go to warps round robin (no claiming): a fixed schedule
     int units, P, S_max;      // CTAs that take a share, partial slots per unit
     int groups_cap, lg2G;     // cap / G and log2(G)
     float scale_log2;
@@ -120,8 +127,16 @@ struct CtaTab {
 // ---- per-unit item counts
 __host__ __device__ __forceinline__ int unit_nri(int r) { return (r + kResTok - 1) / kResTok; }
 __host__ __device__ __forceinline__ int unit_items(int nq, int r) { return unit_nri(r) + nq / kSlice; }
+// a unit's weight: its boundary, then its items
 __host__ __device__ __forceinline__ long long unit_w(int nq, int r) {
-    return (long long)unit_nri(r) * kWR + (long long)(nq / kSlice) * kWP;
+    return kWU + (long long)unit_nri(r) * kWR + (long long)(nq / kSlice) * kWP;
+}
+// the item of a unit (nri residual items) whose start weight is the first one
+// at or after `rem` (0 <= rem < the unit's weight)
+__host__ __device__ __forceinline__ int item_at(long long rem, int nri) {
+    rem = rem > kWU ? rem - kWU : 0;
+    if (rem <= (long long)(nri - 1) * kWR) return (int)((rem + kWR - 1) / kWR);
+    return nri + (int)((rem - (long long)nri * kWR + kWP - 1) / kWP);
 }
 
 // ---- sequence lengths and item prefix sums, by mode.  Uniform batches read the
@@ -200,24 +215,12 @@ __device__ __forceinline__ int part_P(const ArgsDev &) { return dev_tab().P; }
 
 // ---- positions in the work list
 
-// The CTA whose item range holds flat item x: largest c with cta_lo(c) <= x.
-// The ranges have equal weight and an item's weight is 7/8 .. 1 of the mean,
-// so x P / items lands within a step or two of c; the walk from there reads
-// one table entry at a time (the same for the whole warp: kernel-parameter
-// reads with a per-thread index would be serialized).
+// Segment info for the unit holding flat item x, in CTA c's range (one
+// thread).  The CTAs that hold items of the unit are c's neighbours: walks
+// from c over the range table find the first and the last (entries next to
+// c's, mostly in the same constant-cache line; every range is non-empty).
 template <class A>
-__device__ __forceinline__ int cta_of_item(const A &a, int x) {
-    const int P = part_P(a), n = cta_lo(a, P);
-    int c = (int)floor((double)x * (double)P / (double)n);
-    c = c < 0 ? 0 : (c >= P ? P - 1 : c);
-    while (c > 0 && cta_lo(a, c) > x) --c;
-    while (c < P - 1 && cta_lo(a, c + 1) <= x) ++c;
-    return c;
-}
-
-// Segment info for the unit holding flat item x (one thread).
-template <class A>
-__device__ void seg_info(const A &a, int x, int xhi, Seg &s) {
+__device__ void seg_info(const A &a, int c, int x, int xhi, Seg &s) {
     const int b = seq_of_x(a, x);
     const int nq = s_nq(a, b), r = s_r(a, b);
     const int items = unit_items(nq, r);
@@ -232,8 +235,12 @@ __device__ void seg_info(const A &a, int x, int xhi, Seg &s) {
     s.rs = s_rs(a, b);
     s.hi = min(xhi, s.ub + items);
     // CTAs that write a partial for the unit: those whose ranges hold its items
-    s.first = cta_of_item(a, s.ub);
-    s.S_u = cta_of_item(a, s.ub + items - 1) - s.first + 1;
+    const int P = part_P(a), last = s.ub + items - 1;
+    int c0 = c, c1 = c;
+    while (c0 > 0 && cta_lo(a, c0) > s.ub) --c0;
+    while (c1 < P - 1 && cta_lo(a, c1 + 1) <= last) ++c1;
+    s.first = c0;
+    s.S_u = c1 - c0 + 1;
 }
 
 // A warp's place in the work list: unit u (= b Hkv + kh), item k of the unit,
@@ -537,16 +544,17 @@ __device__ void run_cta(const A &a, Smem &sm, int c) {
     pl.v_src = 16 * (lane & 3);
     Cursor pc;
     pc.set(a, min(xlo + warp, xhi - 1));
-    int pq_unit = -1, pq_slot = -1, pstage = 0, nclaim = 0;
+    int pq_unit = -1, pq_slot = -1, pstage = 0, nclaim = 0, nis = 0;
     int xq0 = xhi, xq1 = xhi, xq2 = xhi;   // claimed items in flight, oldest first (xhi = none)
     auto issue_next = [&]() {
-        int x;
-        if (nclaim < kStages - 1) {
-            x = xlo + warp + kWarps * nclaim;
+        int x = 0;
+        if (nis < kStages - 1 || a.det) {   // the first items of each warp are fixed; all of them in det mode
+            x = xlo + warp + kWarps * nis;
         } else {
             if (lane == 0) x = atomicAdd(&sm.next, 1);
             x = __shfl_sync(0xffffffffu, x, 0);
         }
+        ++nis;
         if (x < xhi) {
             pc.advance_to(a, x);
             const uint32_t st = st0 + pstage * kStageBytes;
@@ -576,7 +584,7 @@ __device__ void run_cta(const A &a, Smem &sm, int c) {
     if (tid == 0) {
         sm.zero = make_uint4(0, 0, 0, 0);
         sm.next = xlo + kWarps * (kStages - 1);   // the first kStages-1 items of each warp are fixed
-        seg_info(a, xlo, xhi, sm.seg);
+        seg_info(a, c, xlo, xhi, sm.seg);
     }
     __syncthreads();
 
@@ -595,8 +603,21 @@ __device__ void run_cta(const A &a, Smem &sm, int c) {
     const int qn = lane & 7;
     const bool q_zero = qn & 1;
     const uint32_t q_row_off = ((qn >> 1) * 16 + ((lane >> 3) ^ (qn >> 1))) * 16;
-    // ldmatrix of the key-zero quads: matrices (chunk 2j, chunk 2j, chunk 2j+1, chunk 2j+1)
-    const uint32_t z_lane_off = 16 * (lane >> 4);
+    // key zero-point term: two mma whose A rows are (head, 16-channel chunk) of q and whose
+    // B columns are chunks of the zero row; the term of head h is the sum of the four
+    // diagonal entries D[4h' + j][j] (h' = h mod 2; heads 2, 3 in rows 8-15).  Matrix
+    // m = lane >> 3 of an A load: rows 8 (m & 1) .. +7, channels 8 (m >> 1) .. +7 of each
+    // chunk; the B load: chunks (row & 3) + 4 (m >> 1), channel half m & 1.
+    uint32_t zq_off, zz_off;
+    {
+        const int m = lane >> 3, rr = lane & 7;
+        const int row = ((m & 1) << 3) + rr, h = row >> 2, c8 = 2 * (row & 3) + (m >> 1);
+        zq_off = h * 256 + ((c8 ^ h) << 4);
+        const int cz = 2 * ((rr & 3) + 4 * (m >> 1)) + (m & 1);
+        zz_off = kOffKz + 16 * schunk(cz);
+    }
+    const bool z_diag = t_ == ((g_ & 3) >> 1), z_odd = g_ & 1;
+    const int z_src = 16 * (t_ & 1);
     // residual K rows: matrices (chunk 2kk rows, zero, chunk 2kk+1 rows, zero)
     const int rk_row = lane & 7, rk_m = lane >> 3;
     const bool rk_live = !(rk_m & 1) && rk_row < kResTok;
@@ -726,21 +747,24 @@ __device__ void run_cta(const A &a, Smem &sm, int c) {
                         acc[i][3] *= f;
                     }
                 }
-                // ---- zero-point term sum_c q_c z_c (A = the key-zero chunk in every row)
-                float zc4[4] = {0.f, 0.f, 0.f, 0.f};
-                const uint32_t zb = S + kOffKz + z_lane_off;
-#pragma unroll
-                for (int jj = 0; jj < 4; ++jj) {
-                    uint32_t qf[4];
-                    ldmatrix_x4(qf, q_addr + jj * q_step);
-#pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        const int jc = 2 * jj + e;                     // k-chunk: chunks 2jc, 2jc+1
-                        const int jp = jc < 4 ? jc : (jc ^ 1);         // their position pair under schunk
-                        uint32_t za[4];
-                        ldmatrix_x4(za, zb + 32 * jp);
-                        mma16816(zc4, za, qf[2 * e], qf[2 * e + 1]);
-                    }
+                // ---- zero-point term sum_c q_c z_c of head t_ (two mma, then the diagonal sum)
+                float zc;
+                {
+                    float zd[4] = {0.f, 0.f, 0.f, 0.f};
+                    uint32_t zf[4], qa0[4], qa1[4];
+                    ldmatrix_x4(zf, S + zz_off);
+                    ldmatrix_x4(qa0, qb + zq_off);
+                    ldmatrix_x4(qa1, qb + zq_off + 128);   // chunks 4..7: c8 + 8, and (c8 + 8) ^ h = (c8 ^ h) + 8
+                    mma16816(zd, qa0, zf[0], zf[1]);
+                    mma16816(zd, qa1, zf[2], zf[3]);
+                    float vlo = z_diag ? (z_odd ? zd[1] : zd[0]) : 0.f;   // heads 0, 1
+                    float vhi = z_diag ? (z_odd ? zd[3] : zd[2]) : 0.f;   // heads 2, 3
+                    vlo += __shfl_xor_sync(0xffffffffu, vlo, 4);
+                    vhi += __shfl_xor_sync(0xffffffffu, vhi, 4);
+                    vlo += __shfl_xor_sync(0xffffffffu, vlo, 9);
+                    vhi += __shfl_xor_sync(0xffffffffu, vhi, 9);
+                    const float zl = __shfl_sync(0xffffffffu, vlo, z_src), zh = __shfl_sync(0xffffffffu, vhi, z_src);
+                    zc = t_ < 2 ? zl : zh;
                 }
                 // ---- scores: both m-tiles, one k-chunk at a time; B operand made just in time
                 float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
@@ -774,7 +798,7 @@ __device__ void run_cta(const A &a, Smem &sm, int c) {
                     }
                 }
                 // ---- x = log2 score relative to the reference max m_ref (tokens 2g_, 2g_+1, 16+2g_, 17+2g_)
-                const float zcs = zc4[0] * sl2;
+                const float zcs = zc * sl2;
                 const float sc[4] = {s0[0] + s0[1], s0[2] + s0[3], s1[0] + s1[1], s1[2] + s1[3]};
                 float xv[4];
                 {
@@ -871,7 +895,7 @@ __device__ void run_cta(const A &a, Smem &sm, int c) {
         finish_unit<kMass>(a, sm, sg, c - sg.first);
         if (sg.hi >= xhi) break;
         __syncthreads();   // every thread has read sm.seg and the warp states
-        if (tid == 0) seg_info(a, sg.hi, xhi, sm.seg);
+        if (tid == 0) seg_info(a, c, sg.hi, xhi, sm.seg);
         __syncthreads();
     }
     cp_async_wait<0>();
@@ -912,11 +936,7 @@ __device__ int dev_first_item(const ArgsDev &a, const long long *wbeg, long long
     const long long off = w - wbeg[b];
     const int kh = (int)floor((double)off / (double)W);
     const long long rem = off - kh * W;
-    const int nri = unit_nri(r);
-    int k;
-    if (rem <= (long long)(nri - 1) * kWR) k = (int)((rem + kWR - 1) / kWR);
-    else k = nri + (int)((rem - (long long)nri * kWR + kWP - 1) / kWP);
-    return ib[b] + kh * unit_items(nq, r) + k;
+    return ib[b] + kh * unit_items(nq, r) + item_at(rem, unit_nri(r));
 }
 
 // Device-state mode: build the table, run the CTA's work, and let the last CTA
@@ -1051,6 +1071,8 @@ __global__ void __launch_bounds__(256) mass_kernel(const float4 *__restrict__ xs
 
 // ------------------------------------------------------------ host planning
 
+std::atomic<int> g_deterministic{0};   // minikv_set_deterministic
+
 // Per-device set-up (a function attribute applies to the device current when
 // it is set; the SM count is looked up per device), guarded for calls from
 // several host threads.
@@ -1171,11 +1193,7 @@ Plan plan(const minikv_cache *c, int dev) {
         const long long off = w - wbeg[b];
         const int kh = (int)(off / W);
         const long long rem = off - kh * W;
-        const int nri = unit_nri(r);
-        int k;
-        if (rem <= (long long)(nri - 1) * kWR) k = (int)((rem + kWR - 1) / kWR);
-        else k = nri + (int)((rem - (long long)nri * kWR + kWP - 1) / kWP);
-        p.lo[i] = ibeg[b] + kh * unit_items(nq, r) + k;
+        p.lo[i] = ibeg[b] + kh * unit_items(nq, r) + item_at(rem, unit_nri(r));
     }
     return p;
 }
@@ -1212,6 +1230,8 @@ size_t decode_mass_workspace_bytes(int B, int Hq, int Hkv, int max_tokens) {
     return decode_workspace_bytes(B, Hkv, max_tokens) + mass_stats_bytes(B, Hkv) +
            mass_scores_bytes(B, Hkv, Hq / Hkv, max_tokens);
 }
+
+void decode_set_deterministic(int on) { g_deterministic.store(on ? 1 : 0, std::memory_order_relaxed); }
 
 // Workspace bytes the next decode call on this cache state will use.
 size_t decode_call_workspace_bytes(const minikv_cache *c) {
@@ -1310,6 +1330,7 @@ int decode_launch(minikv_cache *c, const uint16_t *q, const uint16_t *k_new, con
     a.lg2G = 31 - __builtin_clz((unsigned)c->G);
     a.units = p.units; a.P = p.P; a.S_max = p.S_max;
     a.scale_log2 = sm_scale * kLog2e;
+    a.det = g_deterministic.load(std::memory_order_relaxed);
 
     int rc;
     if (c->dseq) {

@@ -37,6 +37,7 @@ int decode_launch(minikv_cache *c, const uint16_t *q, const uint16_t *k_new, con
                   float *mass = nullptr);
 size_t decode_workspace_bytes(int B, int Hkv, int max_tokens);
 size_t decode_mass_workspace_bytes(int B, int Hq, int Hkv, int max_tokens);
+void decode_set_deterministic(int on);
 
 static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -334,6 +335,11 @@ int minikv_decode_attn_mass(minikv_cache *c, const uint16_t *q, const uint16_t *
         return fail(MINIKV_ERR_INVALID_ARG, "decode_attn_mass: mass must be 4-byte aligned");
     return decode_launch(c, q, k_new, v_new, Hq, sm_scale, out, ws, ws_bytes, static_cast<cudaStream_t>(stream),
                          mass);
+}
+
+int minikv_set_deterministic(int on) {
+    decode_set_deterministic(on);
+    return MINIKV_OK;
 }
 
 size_t minikv_workspace_size(int op, int B, int Hq, int Hkv, int T, int D, int W) {

@@ -53,6 +53,7 @@ _SIGS = {
     "minikv_decode_attn": (_I, [ctypes.POINTER(CacheStruct), _P, _P, _P, _I, _F, _P, _P, _Z, _P]),
     "minikv_decode_attn_mass": (_I, [ctypes.POINTER(CacheStruct), _P, _P, _P, _I, _F, _P, _P, _P, _Z, _P]),
     "minikv_decode_attn_static": (_I, [ctypes.POINTER(CacheStruct), _P, _P, _P, _I, _F, _P, _P]),
+    "minikv_set_deterministic": (_I, [_I]),
     "minikv_workspace_size": (_Z, [_I, _I, _I, _I, _I, _I, _I]),
     "minikv_last_error_string": (ctypes.c_char_p, []),
 }
@@ -362,6 +363,12 @@ def decode_attn_mass(cache: MiniKVCache, q: torch.Tensor, k_new: torch.Tensor, v
         _dev(v_new, torch.float16, "v_new"), Hq, float(sm_scale), _dev(out, torch.float16, "out"),
         _dev(mass, torch.float32, "mass"), _dev(ws, torch.uint8, "ws"), ws.numel(), _stream(stream, q.device)))
     return out
+
+
+def set_deterministic(on: bool) -> None:
+    """Fixed assignment of decode items to warps (bit-identical repeat calls)
+    instead of dynamic claiming (the default); process-wide."""
+    _check(lib().minikv_set_deterministic(1 if on else 0))
 
 
 def decode_attn_static(cache: MiniKVCache, q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor,

@@ -362,6 +362,22 @@ MINIKV_API int minikv_decode_attn_static(minikv_cache *c, const uint16_t *q, con
  * tokens a step can attend to). */
 MINIKV_API size_t minikv_workspace_size(int op, int B, int Hq, int Hkv, int T, int D, int W);
 
+/*
+ * minikv_set_deterministic -- choose how the decode calls spread their work
+ * inside a CTA (process-wide; takes effect at the next decode call).
+ *   on = 0 (default): the 16 warps of a CTA claim 32-token items from a
+ *     shared counter, so a warp that the scheduler favours takes more.  Which
+ *     warp sums which items then varies from run to run, and so does the fp32
+ *     rounding of the result: outputs may differ between identical calls in
+ *     the last bits (about 1e-4 relative, far inside the 2e-3 tolerance).
+ *   on = 1: warp w of a CTA takes items w, w + 16, w + 32, .. of its range.
+ *     Identical calls give bit-identical outputs; the step can be slower when
+ *     warps progress unevenly.
+ * The cache contents (packed codes, scales, residual rows) are bit-identical
+ * in both modes.  Returns MINIKV_OK.
+ */
+MINIKV_API int minikv_set_deterministic(int on);
+
 /* Why the last failing call on this host thread failed ("" if none). */
 MINIKV_API const char *minikv_last_error_string(void);
 

@@ -196,3 +196,11 @@ def test_ragged_batch_limit():
     seq = (ctypes.c_int * (3 * (mk.MAX_RAGGED_SEQS + 1)))()
     assert L.minikv_cache_set_ragged(ctypes.byref(c), ctypes.cast(seq, ctypes.c_void_p)) == mk.ERR_UNSUPPORTED
     assert c.seq is None
+
+
+def test_set_deterministic_is_a_host_switch():
+    """The schedule switch needs no device: it only sets what the next decode
+    call passes to its kernel."""
+    L = mk.lib()
+    assert L.minikv_set_deterministic(1) == 0
+    assert L.minikv_set_deterministic(0) == 0

@@ -110,9 +110,19 @@ def test_ragged_decode_vs_oracle(lengths, Hq, Hkv, G, R, steps, device_state):
     print(f"ragged decode max-abs error {worst:.2e}")
 
 
-def test_ragged_equal_lengths_match_uniform_bit_for_bit():
+@pytest.fixture
+def deterministic():
+    mk.set_deterministic(True)
+    try:
+        yield
+    finally:
+        mk.set_deterministic(False)
+
+
+def test_ragged_equal_lengths_match_uniform_bit_for_bit(deterministic):
     """A ragged batch whose sequences all have the same length runs the same
-    schedule as the uniform batch: identical outputs and cache bytes."""
+    schedule as the uniform batch: identical outputs and cache bytes (with the
+    fixed item-to-warp assignment; dynamic claiming may round differently)."""
     B, Hq, Hkv, N, steps = 4, 8, 2, 1000, 3
     k = synth.keys_fp16((B, Hkv, N, 128), synth.seed_of(77, 0, synth.T_K), DEV)
     v = synth.normal_fp16((B, Hkv, N, 128), synth.seed_of(77, 0, synth.T_V), DEV)
@@ -271,3 +281,26 @@ def test_device_state_refuses_a_flush_past_capacity():
     a = cache.arrays()
     for h in range(Hkv):                                                    # the full sequence's packed part intact
         np.testing.assert_array_equal(a["k_codes"][0, h, :64].cpu().numpy().view(np.uint32), ref[0][h].k_codes[:64])
+
+
+def test_deterministic_mode_repeats_bit_for_bit(deterministic):
+    """Fixed item-to-warp assignment: two identical calls (fresh caches, same
+    inputs) give bit-identical outputs, on a shape whose CTAs hold more items
+    than their warps' first two each (where the default mode claims items
+    dynamically).  The default mode agrees with it to well inside the output
+    tolerance."""
+    B, Hq, Hkv, N = 4, 8, 2, 4000
+    k = synth.keys_fp16((B, Hkv, N, 128), synth.seed_of(79, 0, synth.T_K), DEV)
+    v = synth.normal_fp16((B, Hkv, N, 128), synth.seed_of(79, 0, synth.T_V), DEV)
+    q, kn, vn = _step_inputs(B, Hq, Hkv, 80, 0)
+
+    def run():
+        c = mk.MiniKVCache(B, Hkv, 4096 + 64, R=32, Hq=Hq)
+        mk.quant_pack(c, k, v)
+        return mk.decode_attn(c, q, kn, vn)
+
+    a, b = run(), run()
+    assert torch.equal(a, b)
+    mk.set_deterministic(False)
+    d = run()
+    assert float((d.float() - a.float()).abs().max()) <= 2e-4
