@@ -526,7 +526,13 @@ __device__ __forceinline__ void issue_q(const A &a, uint32_t qb, int u, int lane
 
 // ------------------------------------------------------------------ the CTA
 
-template <bool kMass, class A>
+__device__ __forceinline__ void wait_prior_grid() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+__device__ __forceinline__ void launch_dependents() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
+
+// kWait: the CTA does its parameter-only set-up, then waits for the previous
+// kernel on the stream (programmatic dependent launch) before its first global
+// read; otherwise the caller has waited already.
+template <bool kMass, bool kWait, class A>
 __device__ void run_cta(const A &a, Smem &sm, int c) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g_ = lane >> 2, t_ = lane & 3;
@@ -576,16 +582,17 @@ __device__ void run_cta(const A &a, Smem &sm, int c) {
         else xq2 = x;
         ++nclaim;
     };
-#pragma unroll
-    for (int s = 0; s < kStages - 1; ++s) issue_next();   // the first copies go out before any set-up
-
-    // set-up of the first segment while they are in flight (the dynamic claims
-    // start after the barrier below)
+    // set-up of the first segment (kernel parameters and shared memory only: it
+    // may overlap the previous kernel's tail; the dynamic claims start after the
+    // barrier below)
     if (tid == 0) {
         sm.zero = make_uint4(0, 0, 0, 0);
         sm.next = xlo + kWarps * (kStages - 1);   // the first kStages-1 items of each warp are fixed
         seg_info(a, c, xlo, xhi, sm.seg);
     }
+    if (kWait) wait_prior_grid();
+#pragma unroll
+    for (int s = 0; s < kStages - 1; ++s) issue_next();
     __syncthreads();
 
     // ---- consumer constants of this lane
@@ -901,21 +908,23 @@ __device__ void run_cta(const A &a, Smem &sm, int c) {
     cp_async_wait<0>();
 }
 
-__device__ __forceinline__ void wait_prior_grid() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
-
+// Every decode kernel lets the next kernel on the stream be placed at once:
+// its CTAs take SMs as this grid's CTAs leave them and do their parameter-only
+// set-up there; griddepcontrol.wait holds their first global read until this
+// grid has finished and its writes are visible.
 template <bool kMass>
 __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_constant__ ArgsUni a) {
     extern __shared__ __align__(128) unsigned char smem_raw[];
-    wait_prior_grid();
-    run_cta<kMass>(a, *reinterpret_cast<Smem *>(smem_raw), blockIdx.x);
+    launch_dependents();
+    run_cta<kMass, true>(a, *reinterpret_cast<Smem *>(smem_raw), blockIdx.x);
 }
 
 // ragged batch: per-sequence lengths in the parameter table
 template <bool kMass>
 __global__ void __launch_bounds__(kThreads, 1) decode_ragged_kernel(const __grid_constant__ ArgsVar a) {
     extern __shared__ __align__(128) unsigned char smem_raw[];
-    wait_prior_grid();
-    run_cta<kMass>(a, *reinterpret_cast<Smem *>(smem_raw), blockIdx.x);
+    launch_dependents();
+    run_cta<kMass, true>(a, *reinterpret_cast<Smem *>(smem_raw), blockIdx.x);
 }
 
 // First flat item whose start weight is >= w, from the device-state table.
@@ -946,7 +955,8 @@ __device__ int dev_first_item(const ArgsDev &a, const long long *wbeg, long long
 template <bool kMass>
 __global__ void __launch_bounds__(kThreads, 1) decode_dev_kernel(const ArgsDev a) {
     extern __shared__ __align__(128) unsigned char smem_raw[];
-    wait_prior_grid();
+    launch_dependents();
+    wait_prior_grid();   // the state table is written by the previous step
     const int tid = threadIdx.x;
     const int B = nseq(a);
     int *nq = dev_arr(a, 0), *rr = dev_arr(a, 1), *rs = dev_arr(a, 2), *ib = dev_arr(a, 3), *clo = dev_arr(a, 4);
@@ -1001,7 +1011,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_dev_kernel(const ArgsDev a
             clo[cc] = dev_first_item(a, wbeg, (long long)floor((double)cc * (double)Wt / (double)P));
     }
     __syncthreads();
-    if ((int)blockIdx.x < dev_tab().P) run_cta<kMass>(a, *reinterpret_cast<Smem *>(smem_raw), blockIdx.x);
+    if ((int)blockIdx.x < dev_tab().P) run_cta<kMass, false>(a, *reinterpret_cast<Smem *>(smem_raw), blockIdx.x);
     __syncthreads();
     if (tid == 0) {
         const unsigned n = gridDim.x;

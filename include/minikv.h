@@ -368,8 +368,9 @@ MINIKV_API size_t minikv_workspace_size(int op, int B, int Hq, int Hkv, int T, i
  *   on = 0 (default): the 16 warps of a CTA claim 32-token items from a
  *     shared counter, so a warp that the scheduler favours takes more.  Which
  *     warp sums which items then varies from run to run, and so does the fp32
- *     rounding of the result: outputs may differ between identical calls in
- *     the last bits (about 1e-4 relative, far inside the 2e-3 tolerance).
+ *     rounding of the sums: two identical calls may give fp16 outputs that
+ *     differ by about one unit in the last place of the largest outputs
+ *     (5e-4 for outputs below 1), a quarter of the 2e-3 tolerance.
  *   on = 1: warp w of a CTA takes items w, w + 16, w + 32, .. of its range.
  *     Identical calls give bit-identical outputs; the step can be slower when
  *     warps progress unevenly.

@@ -287,7 +287,7 @@ def test_deterministic_mode_repeats_bit_for_bit(deterministic):
     """Fixed item-to-warp assignment: two identical calls (fresh caches, same
     inputs) give bit-identical outputs, on a shape whose CTAs hold more items
     than their warps' first two each (where the default mode claims items
-    dynamically).  The default mode agrees with it to well inside the output
+    dynamically).  The default mode agrees with it to half the output
     tolerance."""
     B, Hq, Hkv, N = 4, 8, 2, 4000
     k = synth.keys_fp16((B, Hkv, N, 128), synth.seed_of(79, 0, synth.T_K), DEV)
@@ -303,4 +303,6 @@ def test_deterministic_mode_repeats_bit_for_bit(deterministic):
     assert torch.equal(a, b)
     mk.set_deterministic(False)
     d = run()
-    assert float((d.float() - a.float()).abs().max()) <= 2e-4
+    # the fp32 sums differ in their last bits; after fp16 rounding that is at most
+    # about one unit in the last place of the largest outputs (here |out| < 1)
+    assert float((d.float() - a.float()).abs().max()) <= 1e-3
