@@ -86,6 +86,7 @@ struct FaArgs {
     float *lse2;        // [B, Hq, W] window rows, log2 domain
     unsigned *status;   // bit 0: a bounded wait expired in some CTA (its outputs are not valid)
     int Hq, Hkv, T, W, nqt;
+    int hg;             // (sequence, head) pairs per scheduling group
     float scale_log2;
 };
 
@@ -124,10 +125,14 @@ __global__ void __launch_bounds__(kFaThreads, 1)
     FaSmem &s = *reinterpret_cast<FaSmem *>(smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u));
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
-    // heads outer, query tiles (heaviest first) inner: the CTAs resident at
-    // one time share one head's K / V in L2
-    const int bh = blockIdx.x / a.nqt;
-    const int qt = a.nqt - 1 - (int)(blockIdx.x % a.nqt);
+    // Groups of hg (sequence, head) pairs whose K / V fit in L2 together; inside
+    // a group, query tiles heaviest first across all its heads, so the longest
+    // CTAs start early and the last wave holds only short ones.
+    const int BH = gridDim.x / a.nqt;
+    const int grp = (int)blockIdx.x / (a.hg * a.nqt), rr = (int)blockIdx.x - grp * a.hg * a.nqt;
+    const int ng = min(a.hg, BH - grp * a.hg);
+    const int bh = grp * a.hg + rr % ng;
+    const int qt = a.nqt - 1 - rr / ng;
     const int b = bh / a.Hq, h = bh % a.Hq;
     const int kvh = b * a.Hkv + h / (a.Hq / a.Hkv);
     const int nkb = qt + 1;   // causal: key blocks 0..qt
@@ -541,6 +546,13 @@ int prefill_launch(const uint16_t *q, const uint16_t *k, const uint16_t *v, int 
         return check_launch("select_prefill: clearing the status word");
     fa.Hq = Hq; fa.Hkv = Hkv; fa.T = T; fa.W = W;
     fa.nqt = (T + kTileM - 1) / kTileM;
+    {   // K and V of one (sequence, head): 2 x T x 128 fp16; about 64 MB of them per group
+        const long long per = 512ll * T;
+        long long hg = (64ll << 20) / per;
+        if (hg < 1) hg = 1;
+        if (hg > (long long)B * Hq) hg = (long long)B * Hq;
+        fa.hg = (int)hg;
+    }
     fa.scale_log2 = sm_scale * kLog2e;
     const size_t fa_smem = sizeof(FaSmem) + 1024;
     const int dev = current_device();
