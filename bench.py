@@ -335,12 +335,12 @@ def make_decode_state(torch, mk, synth, device, warmup, steps):
     G, Gv, R = DECODE["G"], DECODE["Gv"], DECODE["R"]
     if DECODE["batch"] == "max":
         free, _ = torch.cuda.mem_get_info(device)
-        DECODE["batch"], per_seq = max_batch(mk, free, steps=max(512, warmup + 2 * steps + 2))
+        DECODE["batch"], per_seq = max_batch(mk, free, steps=max(512, warmup + 3 * steps + 2))
         DECODE["max_batch_rule"] = (f"largest batch that fits {free / 1e9:.1f} GB of free HBM at "
                                     f"{per_seq / 1e9:.3f} GB per sequence (caches sized for 512 steps)")
     B = DECODE["batch"]
     keeps = decode_keeps()
-    total_steps = max(warmup + 2 * steps + 2, 512 if "max_batch_rule" in DECODE else 0)
+    total_steps = max(warmup + 3 * steps + 2, 512 if "max_batch_rule" in DECODE else 0)
     cap_max = ((max(keeps) + total_steps + 8) // G + 2) * G
     op = mk.OP_DECODE_ATTN_MASS if DECODE.get("mass") else mk.OP_DECODE_ATTN
     ws = torch.zeros(mk.workspace_size(op, B, Hq, Hkv, cap_max + R + G), dtype=torch.uint8, device=device)
@@ -602,7 +602,8 @@ def measure_decode(ctx, args, steps, warmup, with_e2e=True):
     stream = torch.cuda.current_stream(device)
     evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(L)] for _ in range(steps)]
     sev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
-    nbytes = []
+    nbytes = []     # per step and layer: algorithmic bytes of the timed steps
+    nbytes_k = []   # the same for the steps whose launches are timed one by one (eager)
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ctx.barrier()
     torch.cuda.synchronize()
@@ -611,8 +612,8 @@ def measure_decode(ctx, args, steps, warmup, with_e2e=True):
         for s in range(steps):
             p = (warmup + s) % P
             nbytes.append(step_bytes())
-            if eager:
-                layer_calls(qin, knin, vnin, p, evs[s])
+            if eager:   # the step as a caller runs it: nothing between the layer calls
+                layer_calls(qin, knin, vnin, p)
             else:
                 sev[s][0].record(stream)
                 graphs[p].replay()
@@ -620,9 +621,20 @@ def measure_decode(ctx, args, steps, warmup, with_e2e=True):
             mirror.advance()
         t1.record(stream)
         torch.cuda.synchronize()
-    ctx.barrier()
+        ctx.barrier()
+        if eager:
+            # the kernel durations: the same steps again with an event pair around
+            # every launch (the events sit between the kernels, so this pass is not
+            # the one the step time comes from)
+            for s in range(steps):
+                p = (warmup + steps + s) % P
+                nbytes_k.append(step_bytes())
+                layer_calls(qin, knin, vnin, p, evs[s])
+                mirror.advance()
+            torch.cuda.synchronize()
+            ctx.barrier()
     ms = t0.elapsed_time(t1)
-    launch_bytes = [b for sb in nbytes for b in sb]
+    launch_bytes = [b for sb in (nbytes_k if eager else nbytes) for b in sb]
     if eager:
         kern_ms = [evs[s][l][0].elapsed_time(evs[s][l][1]) for s in range(steps) for l in range(L)]
     else:   # a replay runs the L layer launches back to back: its time / L per launch (gaps included)
@@ -640,9 +652,9 @@ def measure_decode(ctx, args, steps, warmup, with_e2e=True):
 
     if with_e2e:
         # ---- end to end: inputs from pinned host memory, outputs back, each step.
-        # Two buffer sets: while step s computes, a copy stream brings step s+1's
-        # inputs in and takes step s-1's outputs out (stream order and events keep
-        # each buffer's copies and its compute apart).
+        # Two buffer sets and two copy streams: while step s computes, one brings
+        # step s+1's inputs in and the other takes step s-1's outputs out; events
+        # keep each buffer's copies and its compute apart.
         hq = qin.cpu().pin_memory()
         hk = knin.cpu().pin_memory()
         hv = vnin.cpu().pin_memory()
@@ -660,31 +672,39 @@ def measure_decode(ctx, args, steps, warmup, with_e2e=True):
                 with torch.cuda.graph(g):
                     layer_calls(dq[i], dk[i], dv[i], 0, o=dout[i])
                 g_e2e.append(g)
-        copy = torch.cuda.Stream(device)
-        in_ready = [torch.cuda.Event() for _ in range(2)]
-        done = [torch.cuda.Event() for _ in range(2)]
+        cin, cout = torch.cuda.Stream(device), torch.cuda.Stream(device)
+        in_ready = [torch.cuda.Event() for _ in range(2)]   # buffer i's inputs have landed
+        done = [torch.cuda.Event() for _ in range(2)]       # step on buffer i computed
+        out_free = [torch.cuda.Event() for _ in range(2)]   # buffer i's outputs copied out
         torch.cuda.synchronize()
         ctx.barrier()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        copy.wait_stream(stream)
+        cin.wait_stream(stream)
+        cout.wait_stream(stream)
         for s in range(steps):
             i, p = s % 2, s % P
-            with torch.cuda.stream(copy):
+            with torch.cuda.stream(cin):
+                if s >= 2:
+                    cin.wait_event(done[i])      # step s-2 has read this buffer's inputs
                 dq[i].copy_(hq[p:p + 1], non_blocking=True)
                 dk[i].copy_(hk[p:p + 1], non_blocking=True)
                 dv[i].copy_(hv[p:p + 1], non_blocking=True)
-                in_ready[i].record(copy)
+                in_ready[i].record(cin)
             stream.wait_event(in_ready[i])
+            if s >= 2:
+                stream.wait_event(out_free[i])   # step s-2's outputs have left this buffer
             if eager:
                 layer_calls(dq[i], dk[i], dv[i], 0, o=dout[i])
             else:
                 g_e2e[i].replay()
             done[i].record(stream)
-            with torch.cuda.stream(copy):
-                copy.wait_event(done[i])
+            with torch.cuda.stream(cout):
+                cout.wait_event(done[i])
                 hout[i].copy_(dout[i], non_blocking=True)
-        stream.wait_stream(copy)
+                out_free[i].record(cout)
+        stream.wait_stream(cin)
+        stream.wait_stream(cout)
         e1.record(stream)
         torch.cuda.synchronize()
         ctx.barrier()
@@ -701,7 +721,8 @@ def measure_decode(ctx, args, steps, warmup, with_e2e=True):
 
 
 def launch_name(eager):
-    return ("eager: one Python call per layer" if eager else
+    return ("eager: one Python call per layer (step time from calls with nothing between them; kernel "
+            "durations from a second pass with an event pair around each launch)" if eager else
             "one CUDA graph replay per step (all layer calls captured, state on the GPU)")
 
 
@@ -712,8 +733,7 @@ def select_preset(name, args):
         DECODE["layers"] = args.layers
     if args.mass and name == args.workload:
         DECODE["mass"] = True
-    if args.launch == "eager" or (args.launch == "auto" and AUTO_EAGER and "contexts" not in DECODE
-                                  and DECODE["batch"] != "max"):
+    if args.launch == "eager" or (args.launch == "auto" and AUTO_EAGER):
         DECODE["eager"] = True
 
 
@@ -721,9 +741,10 @@ def select_preset(name, args):
 # numbers are driver-observed): LLaMA2-13B MHA decode and the pyramid (B = 4).
 SUBLINE_WORKLOADS = ("llama2_13b_decode", "pyramid_44k_decode")
 SUBLINE_STEPS = 16
-# --launch auto: one Python call per layer for uniform batches (its kernel is
-# faster than the device-state kernel a graph replays, and the host keeps up),
-# graph replay for ragged batches (the per-call host cost is higher there)
+# --launch auto: one Python call per layer, for uniform and ragged batches
+# alike.  The host-planned kernel is faster than the device-state kernel a graph
+# replays, the host stays ahead of the GPU, and back-to-back calls let each
+# layer's launch overlap the previous one's drain (programmatic dependent launch).
 AUTO_EAGER = True
 
 
@@ -786,7 +807,10 @@ def run_gpu(args):
                          "peak": pk["hbm"], "unit": "GB/s", "frac": main["achieved_gbs"] / pk["hbm"],
                          "traffic": traffic, "algorithmic_bytes_per_launch": main["mean_launch_bytes"],
                          "mean_launch_us": main["mean_launch_us"], "peak_source": pk["src"],
-                         "traffic_source": traffic_note},
+                         "traffic_source": traffic_note,
+                         # back to back (no events between the launches) consecutive layer
+                         # launches overlap their set-up and drain: the step's time per layer
+                         "back_to_back_us_per_layer": main["ms_per_step"] * 1e3 / DECODE["layers"]},
             "cpu_baseline": cpu,
             "e2e": main["e2e"],
             "gpu_launches": main["launches"],
@@ -812,8 +836,7 @@ def main():
                     help="decode workload (the default one carries the bench line's target)")
     ap.add_argument("--launch", default="auto", choices=["auto", "graph", "eager"],
                     help="graph: state on the GPU, one captured CUDA graph replayed per step; eager: one Python "
-                         "call per layer, host-side state; auto: eager for uniform batches, graph for ragged and "
-                         "max-batch ones")
+                         "call per layer, host-side state; auto: eager")
     ap.add_argument("--mass", action="store_true",
                     help="decode with minikv_decode_attn_mass (H2O-style running attention mass per token)")
     ap.add_argument("--prefill-workload", default="llama2_7b_prefill_select", choices=list(PREFILL_PRESETS))
