@@ -234,6 +234,26 @@ def oracle_decode_rate(budget_s: float, threads: int):
     return sum(counts) / dt, sum(counts), dt
 
 
+def compression(step_bytes):
+    L, B, Hkv = DECODE["layers"], DECODE["batch"], DECODE["kv_heads"]
+    per_layer = step_bytes / L
+    ctx_tokens = sum(DECODE["contexts"]) if "contexts" in DECODE else B * DECODE["context"]
+    kept = sum(seq_keeps()) if "contexts" in DECODE else B * sum(decode_keeps()) / L
+    fp16 = Hkv * 128 * 2 * 2   # K and V bytes per token
+    return {"of_full_context_fp16": per_layer / (ctx_tokens * fp16), "of_kept_fp16": per_layer / (kept * fp16)}
+
+
+def cpu_model():
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
 def cpu_tokens_per_s(rate):
     units_per_step = DECODE["layers"] * DECODE["batch"] * DECODE["kv_heads"]
     return rate * DECODE["batch"] / units_per_step
@@ -785,10 +805,12 @@ def run_gpu(args):
             and not args.mass):
         threads = os.cpu_count() or 1
         rate, n, dt = oracle_decode_rate(args.cpu_seconds, threads)
+        rate1, n1, dt1 = oracle_decode_rate(max(1.0, args.cpu_seconds / 4), 1)
         cpu = {"value": cpu_tokens_per_s(rate), "unit": "tokens/s", "cores": threads, "kind": "oracle",
+               "cpu_model": cpu_model(), "single_thread_value": cpu_tokens_per_s(rate1),
                "sample": f"{n} decode unit-steps (one sequence x KV head of one layer: 6553 kept tokens, 4 query "
                          f"heads, fp64) in {dt:.1f} s on {threads} threads, scaled to 32 layers x 16 x 8 units "
-                         f"per step"}
+                         f"per step; single-thread value from {n1} unit-steps in {dt1:.1f} s on one thread"}
 
     csrc = os.path.join(ROOT, "bit_quantized_evicted_b200", "csrc")
     traffic, traffic_note = recorded_traffic(
@@ -803,6 +825,9 @@ def run_gpu(args):
             "dtype": "u2+f16 (2-bit codes, fp16 scales/residual, fp32 accumulate)", "data": "synthetic",
             "config": main_cfg, "launch": launch_name(eager),
             "hbm_gbs": main["hbm_gbs"], "hbm_frac_of_peak": main["hbm_gbs"] / pk["hbm"],
+            # cache bytes a layer-step reads (packed codes, scales, zeros, fp16 residual) against the
+            # same batch's K and V in fp16: the full context, and the kept tokens only
+            "compression": compression(main["step_bytes"]),
             "roofline": {"bound": "hbm", "kernel": "decode_kernel", "achieved": main["achieved_gbs"],
                          "peak": pk["hbm"], "unit": "GB/s", "frac": main["achieved_gbs"] / pk["hbm"],
                          "traffic": traffic, "algorithmic_bytes_per_launch": main["mean_launch_bytes"],
