@@ -105,7 +105,7 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N)); }
 
-// ---- mbarrier + bulk (TMA, non-tensor) copies -------------------------------
+// ---- mbarriers ----------------------------------------------------------------
 
 __device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(smem_addr(bar)), "r"(count));
@@ -130,15 +130,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint32
     }
     return false;
 }
-// Bulk copy of `bytes` (multiple of 16, both addresses 16-byte aligned) from
-// global to this CTA's shared memory, completing on `bar`.
-__device__ __forceinline__ void bulk_g2s(void *sdst, const void *gsrc, uint32_t bytes, uint64_t *bar) {
-    asm volatile(
-        "cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(smem_addr(sdst)),
-        "l"(gsrc), "r"(bytes), "r"(smem_addr(bar))
-        : "memory");
-}
-
 // ---- the 2-bit quantizer (bit-exact: one IEEE fp32 op per step) -------------
 
 // scale = fp16_rn(fp32(mx - mn) / 3); mn/mx already canonical (+0 for zero).

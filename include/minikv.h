@@ -284,7 +284,7 @@ MINIKV_API int minikv_evict_pack_seq(const float *scores, const uint16_t *k, con
  * On a ragged cache every step runs per sequence, from and into its own state
  * (one launch for the whole batch; the split of packed tokens over CTAs
  * follows the actual per-sequence lengths).
- *   ws: minikv_workspace_size(MINIKV_OP_DECODE_ATTN, B, Hq, Hkv, cap, D, 0)
+ *   ws: minikv_workspace_size(MINIKV_OP_DECODE_ATTN, B, Hq, Hkv, cap + R + G, D, 0)
  *       bytes, ZERO-FILLED before its first use; every call leaves it ready for
  *       the next (its arrival counters return to zero).  Calls that share one
  *       ws must not overlap on the GPU.
