@@ -8,7 +8,7 @@
 //   * residual items: 5 fp16 residual tokens each (the new token included), and
 //   * packed items:   32 packed tokens each (one slice of one key group).
 // The items of all units are laid end to end and cut, by weight (packed 8,
-// residual 7: their measured costs; 256 more at each unit boundary, for the
+// residual 7: their measured costs; 640 more at each unit boundary, for the
 // extra segment end and merge it costs the CTA whose range crosses it), into
 // one contiguous range per SM.  One
 // CTA of 16 warps runs on each SM.  Its warps claim the items of its range one
@@ -65,7 +65,7 @@ constexpr int kResTok = 5;           // residual tokens per residual item
 constexpr int kStages = 3;           // per-warp pipeline depth
 constexpr int kStageBytes = 2688;    // one packed item (a residual item takes 2560)
 constexpr int kWP = 8, kWR = 7;      // partition weights of a packed / residual item (measured cost ratio)
-constexpr int kWU = 256;             // partition weight of a unit boundary: the extra segment end and merge
+constexpr int kWU = 640;             // partition weight of a unit boundary: the extra segment end and merge
                                      // that a CTA whose range crosses into a new unit pays
 constexpr int kMinShare = kWU + 8 * kWP;   // least weight per CTA (a range always holds an item start)
 constexpr int kPartStride = 132;     // floats per (unit, slot, head): y[128], m, l
