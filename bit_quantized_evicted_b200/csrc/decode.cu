@@ -115,6 +115,7 @@ struct Args {
     int n_q, r, res_start;    // uniform batch: every sequence's lengths (r counts the new token)
     int det;                  // 1: items go to warps round robin (no claiming): a fixed schedule
     int units, P, S_max;      // CTAs that take a share, partial slots per unit
+    int nb;                   // sequences (units / Hkv)
     int groups_cap, lg2G;     // cap / G and log2(G)
     float scale_log2;
 };
@@ -145,7 +146,7 @@ __host__ __device__ __forceinline__ int item_at(long long rem, int nri) {
 struct ArgsUni : Args {
     CtaTab cta;
 };
-__host__ __device__ __forceinline__ int nseq(const Args &a) { return a.units / a.Hkv; }
+__host__ __device__ __forceinline__ int nseq(const Args &a) { return a.nb; }
 __device__ __forceinline__ int s_nq(const ArgsUni &a, int) { return a.n_q; }
 __device__ __forceinline__ int s_r(const ArgsUni &a, int) { return a.r; }
 __device__ __forceinline__ int s_rs(const ArgsUni &a, int) { return a.res_start; }
@@ -187,7 +188,8 @@ __device__ __forceinline__ int cta_lo(const ArgsVar &a, int c) { return a.cta.lo
 __device__ __forceinline__ int part_P(const ArgsVar &a) { return a.P; }
 
 // Device-state mode: the table sits behind Smem in dynamic shared memory:
-// DevTab, then n_q[B], r[B], res_start[B], ibeg[B + 1], cta_lo[P + 1] (int).
+// DevTab, then n_q[B], r[B], res_start[B], ibeg[B + 1], cta_lo[P + 1],
+// status[B] (int; P = the launch's partition bound a.P).
 struct ArgsDev : Args {};
 struct DevTab {
     long long Wt;
@@ -961,11 +963,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_dev_kernel(const ArgsDev a
     const int B = nseq(a);
     int *nq = dev_arr(a, 0), *rr = dev_arr(a, 1), *rs = dev_arr(a, 2), *ib = dev_arr(a, 3), *clo = dev_arr(a, 4);
     __shared__ long long wbeg[kMaxRaggedSeqs + 1];
+    int *stw = clo + a.P + 1;   // status words as read
     for (int b = tid; b < B; b += kThreads) {
         const int4 st = __ldcg(reinterpret_cast<const int4 *>(a.dseq) + b);
         nq[b] = st.x;
         rr[b] = st.y + 1;
         rs[b] = st.z;
+        stw[b] = st.w;
     }
     __syncthreads();
     if (tid < 32) {   // exclusive prefix sums of items and weights, 32 sequences per pass
@@ -1012,26 +1016,28 @@ __global__ void __launch_bounds__(kThreads, 1) decode_dev_kernel(const ArgsDev a
     }
     __syncthreads();
     if ((int)blockIdx.x < dev_tab().P) run_cta<kMass, false>(a, *reinterpret_cast<Smem *>(smem_raw), blockIdx.x);
+    Smem &sm = *reinterpret_cast<Smem *>(smem_raw);
     __syncthreads();
     if (tid == 0) {
         const unsigned n = gridDim.x;
-        if (atom_inc_acq_rel(a.grid_counter, n - 1) == n - 1) {
-            for (int b = 0; b < B; ++b) {
-                int4 st = make_int4(nq[b], rr[b], rs[b], __ldcg(a.dseq + 4 * b + 3));   // status stays set
-                if (rr[b] == a.ring) {
-                    if (nq[b] + a.G <= a.cap) {
-                        st.x += a.G;
-                        st.y -= a.G;
-                        st.z = (st.z + a.G) % a.ring;
-                    } else {
-                        st.y -= 1;   // state unchanged
-                        st.w = 1;
-                    }
-                }
-                reinterpret_cast<int4 *>(a.dseq)[b] = st;
-            }
-        }
+        sm.flag = atom_inc_acq_rel(a.grid_counter, n - 1) == n - 1;
     }
+    __syncthreads();
+    if (sm.flag)   // the last CTA: every sequence's new state, one thread per sequence
+        for (int b = tid; b < B; b += kThreads) {
+            int4 st = make_int4(nq[b], rr[b], rs[b], stw[b]);   // a set status stays set
+            if (rr[b] == a.ring) {
+                if (nq[b] + a.G <= a.cap) {
+                    st.x += a.G;
+                    st.y -= a.G;
+                    st.z = (st.z + a.G) % a.ring;
+                } else {
+                    st.y -= 1;   // state unchanged
+                    st.w = 1;
+                }
+            }
+            reinterpret_cast<int4 *>(a.dseq)[b] = st;
+        }
 }
 
 // mass[unit][t] += sum_h 2^(xs[unit][h][t] - M_h) / L_h for the n_u tokens
@@ -1091,7 +1097,7 @@ bool g_attr_done[kMaxDevices] = {};
 int g_sms[kMaxDevices] = {};
 
 size_t dev_smem_bytes(int B, int P) {
-    return sizeof(Smem) + sizeof(DevTab) + (4 * (size_t)B + 1 + (size_t)P + 1) * sizeof(int);
+    return sizeof(Smem) + sizeof(DevTab) + (5 * (size_t)B + 1 + (size_t)P + 1) * sizeof(int);
 }
 
 // the kernels' shared memory is above the 48 KB default: opt in once per device
@@ -1339,6 +1345,7 @@ int decode_launch(minikv_cache *c, const uint16_t *q, const uint16_t *k_new, con
     a.groups_cap = c->cap / c->G;
     a.lg2G = 31 - __builtin_clz((unsigned)c->G);
     a.units = p.units; a.P = p.P; a.S_max = p.S_max;
+    a.nb = c->B;
     a.scale_log2 = sm_scale * kLog2e;
     a.det = g_deterministic.load(std::memory_order_relaxed);
 
