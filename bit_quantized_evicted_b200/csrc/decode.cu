@@ -972,6 +972,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_dev_kernel(const ArgsDev a
         stw[b] = st.w;
     }
     __syncthreads();
+    // The launch-wide ticket, taken as soon as the state is read (release: this
+    // CTA's reads come before it), by the last warp: the CTA whose ticket is
+    // the last one writes the next state while the table is built.
+    unsigned ticket = 0;
+    if (tid == kThreads - 1) ticket = atom_inc_acq_rel(a.grid_counter, gridDim.x - 1);
     if (tid < 32) {   // exclusive prefix sums of items and weights, 32 sequences per pass
         int ci = 0;
         long long cw = 0;
@@ -1014,17 +1019,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_dev_kernel(const ArgsDev a
         for (int cc = tid; cc <= P; cc += kThreads)
             clo[cc] = dev_first_item(a, wbeg, (long long)floor((double)cc * (double)Wt / (double)P));
     }
-    __syncthreads();
-    if ((int)blockIdx.x < dev_tab().P) run_cta<kMass, false>(a, *reinterpret_cast<Smem *>(smem_raw), blockIdx.x);
-    Smem &sm = *reinterpret_cast<Smem *>(smem_raw);
-    __syncthreads();
-    if (tid == 0) {
-        const unsigned n = gridDim.x;
-        sm.flag = atom_inc_acq_rel(a.grid_counter, n - 1) == n - 1;
-    }
-    __syncthreads();
-    if (sm.flag)   // the last CTA: every sequence's new state, one thread per sequence
-        for (int b = tid; b < B; b += kThreads) {
+    // the last ticket's CTA: every sequence's new state, by its last warp
+    if (tid >= kThreads - 32 && __shfl_sync(0xffffffffu, ticket, 31) == gridDim.x - 1)
+        for (int b = tid - (kThreads - 32); b < B; b += 32) {
             int4 st = make_int4(nq[b], rr[b], rs[b], stw[b]);   // a set status stays set
             if (rr[b] == a.ring) {
                 if (nq[b] + a.G <= a.cap) {
@@ -1038,6 +1035,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_dev_kernel(const ArgsDev a
             }
             reinterpret_cast<int4 *>(a.dseq)[b] = st;
         }
+    __syncthreads();
+    if ((int)blockIdx.x < dev_tab().P) run_cta<kMass, false>(a, *reinterpret_cast<Smem *>(smem_raw), blockIdx.x);
 }
 
 // mass[unit][t] += sum_h 2^(xs[unit][h][t] - M_h) / L_h for the n_u tokens
