@@ -950,9 +950,9 @@ __device__ int dev_first_item(const ArgsDev &a, const long long *wbeg, long long
     return ib[b] + kh * unit_items(nq, r) + item_at(rem, unit_nri(r));
 }
 
-// Device-state mode: build the table, run the CTA's work, and let the last CTA
-// of the launch advance the state of every sequence (append; flush G tokens
-// where the ring is full).  A flush that would pass `cap` is not done: the
+// Device-state mode: read the state, build the table, run the CTA's work.  The
+// CTA that takes the last launch-wide ticket after reading the state writes the
+// next state of every sequence (append; flush G tokens where the ring is full).  A flush that would pass `cap` is not done: the
 // sequence keeps its state and its status word is set to 1.
 template <bool kMass>
 __global__ void __launch_bounds__(kThreads, 1) decode_dev_kernel(const ArgsDev a) {

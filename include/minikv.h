@@ -133,8 +133,8 @@ MINIKV_API int minikv_cache_set_ragged(minikv_cache *c, int *seq);
  * _seq forms) write the loaded rows' state into dseq from their kernel, and
  * each decode call runs one launch configuration fixed by the cache's shape:
  * the kernel reads the state, splits this step's packed tokens over its CTAs,
- * and its last CTA advances every sequence's state (minikv_decode_attn_static
- * reads and advances the same state).  A step whose flush would pass `cap` leaves that
+ * and writes every sequence's next state once all its CTAs have read the
+ * current one (minikv_decode_attn_static reads and advances the same state).  A step whose flush would pass `cap` leaves that
  * sequence's state unchanged (its new token is not kept) and sets its status
  * word to 1; the host learns it by reading dseq.  Capacity is therefore not
  * checked on the host in this mode.
