@@ -321,7 +321,8 @@ def run_reference(args):
             "extrapolated": {"value": True, "ms_per_step": True, "timed_seconds": timed, "unit_steps_timed": units,
                              "unit_steps_per_full_step": per_full_step,
                              "unit_steps_per_s": rate},
-            "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": sample},
+            "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle", "cpu_model": cpu_model(),
+                             "sample": sample},
             "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
