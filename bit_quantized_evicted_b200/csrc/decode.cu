@@ -49,6 +49,7 @@
 #include <math.h>
 
 #include <atomic>
+#include <map>
 #include <mutex>
 #include <vector>
 
@@ -65,9 +66,13 @@ constexpr int kResTok = 5;           // residual tokens per residual item
 constexpr int kStages = 3;           // per-warp pipeline depth
 constexpr int kStageBytes = 2688;    // one packed item (a residual item takes 2560)
 constexpr int kWP = 8, kWR = 7;      // partition weights of a packed / residual item (measured cost ratio)
-constexpr int kWU = 640;             // partition weight of a unit boundary: the extra segment end and merge
-                                     // that a CTA whose range crosses into a new unit pays
-constexpr int kMinShare = kWU + 8 * kWP;   // least weight per CTA (a range always holds an item start)
+constexpr int kWU = 640;             // partition weight of a unit boundary in the device-state mode (the
+                                     // host-planned modes pick one per call); also the floor of min_share
+constexpr int kMinShare = kWU + 8 * kWP;   // least weight per CTA at the default boundary weight
+// least weight per CTA for boundary weight wu: a range always holds an item
+// start, and never less than at the default weight (the partial slots of the
+// workspace are sized for that share)
+constexpr long long min_share(int wu) { return (long long)(wu > kWU ? wu : kWU) + 8 * kWP; }
 constexpr int kPartStride = 132;     // floats per (unit, slot, head): y[128], m, l
 constexpr int kMaxCtas = 512;
 constexpr float kLazy = 8.f;         // log2 headroom before a head's reference max moves
@@ -128,14 +133,14 @@ struct CtaTab {
 // ---- per-unit item counts
 __host__ __device__ __forceinline__ int unit_nri(int r) { return (r + kResTok - 1) / kResTok; }
 __host__ __device__ __forceinline__ int unit_items(int nq, int r) { return unit_nri(r) + nq / kSlice; }
-// a unit's weight: its boundary, then its items
-__host__ __device__ __forceinline__ long long unit_w(int nq, int r) {
-    return kWU + (long long)unit_nri(r) * kWR + (long long)(nq / kSlice) * kWP;
+// a unit's weight: its boundary (weight wu), then its items
+__host__ __device__ __forceinline__ long long unit_w(int nq, int r, int wu = kWU) {
+    return wu + (long long)unit_nri(r) * kWR + (long long)(nq / kSlice) * kWP;
 }
 // the item of a unit (nri residual items) whose start weight is the first one
 // at or after `rem` (0 <= rem < the unit's weight)
-__host__ __device__ __forceinline__ int item_at(long long rem, int nri) {
-    rem = rem > kWU ? rem - kWU : 0;
+__host__ __device__ __forceinline__ int item_at(long long rem, int nri, int wu = kWU) {
+    rem = rem > wu ? rem - wu : 0;
     if (rem <= (long long)(nri - 1) * kWR) return (int)((rem + kWR - 1) / kWR);
     return nri + (int)((rem - (long long)nri * kWR + kWP - 1) / kWP);
 }
@@ -554,13 +559,14 @@ __device__ void run_cta(const A &a, Smem &sm, int c) {
     pc.set(a, min(xlo + warp, xhi - 1));
     int pq_unit = -1, pq_slot = -1, pstage = 0, nclaim = 0, nis = 0;
     int xq0 = xhi, xq1 = xhi, xq2 = xhi;   // claimed items in flight, oldest first (xhi = none)
+    int pre = 0;   // lane 0: the next dynamic claim, taken one issue ahead so its latency is hidden
     auto issue_next = [&]() {
         int x = 0;
         if (nis < kStages - 1 || a.det) {   // the first items of each warp are fixed; all of them in det mode
             x = xlo + warp + kWarps * nis;
         } else {
-            if (lane == 0) x = atomicAdd(&sm.next, 1);
-            x = __shfl_sync(0xffffffffu, x, 0);
+            x = __shfl_sync(0xffffffffu, pre, 0);
+            if (lane == 0) pre = atomicAdd(&sm.next, 1);
         }
         ++nis;
         if (x < xhi) {
@@ -596,6 +602,7 @@ __device__ void run_cta(const A &a, Smem &sm, int c) {
 #pragma unroll
     for (int s = 0; s < kStages - 1; ++s) issue_next();
     __syncthreads();
+    if (!a.det && lane == 0) pre = atomicAdd(&sm.next, 1);   // the first dynamic claim
 
     // ---- consumer constants of this lane
     const float sl2 = a.scale_log2, sl2w = a.scale_log2 * kScoreUnit;
@@ -1147,10 +1154,10 @@ struct Plan {
     std::vector<int> lo;     // host-planned modes: first item of each CTA (P + 1 entries)
 };
 
-// CTAs that take a share: one per SM, at least kMinShare weight each
-long long cta_count(long long Wt, int slots) {
+// CTAs that take a share: one per SM, at least min_share(wu) weight each
+long long cta_count(long long Wt, int slots, int wu = kWU) {
     long long P = slots;
-    if (P > Wt / kMinShare) P = Wt / kMinShare;
+    if (P > Wt / min_share(wu)) P = Wt / min_share(wu);
     if (P > kMaxCtas) P = kMaxCtas;
     return P < 1 ? 1 : P;
 }
@@ -1159,37 +1166,42 @@ long long cta_count(long long Wt, int slots) {
 // least `share` wide: the CTA ranges its items can fall into.
 int slots_bound(long long W, long long share) { return (int)(W / share + 2); }
 
-Plan plan(const minikv_cache *c, int dev) {
-    Plan p;
-    p.units = c->B * c->Hkv;
-    const int ring = c->R + c->G;
-    if (c->dseq) {
-        // device-state mode: one configuration for every state the cache can hold;
-        // the kernel partitions this step's items itself
-        const long long Wmax = unit_w(c->cap, ring);
-        p.P = (int)cta_count((long long)p.units * Wmax, sm_count(dev));
-        p.S_max = slots_bound(Wmax, kMinShare);
-        if (p.S_max > p.P) p.S_max = p.P;
-        p.max_n = c->cap + ring;
-        return p;
-    }
-    const bool ragged = c->seq != nullptr;
-    // per-sequence item and weight prefix sums (uniform: one state for every sequence)
-    std::vector<long long> wbeg(c->B + 1, 0);
-    std::vector<int> ibeg(c->B + 1, 0);
+// ---- host partition of the work list (uniform and ragged batches)
+//
+// The items of all units are cut into one contiguous range per CTA at equal
+// steps of weight.  A unit weighs its items (kWP per packed item, kWR per
+// residual item) plus a boundary weight wu placed before its first item, so a
+// cut that lands in that region moves to the unit's first item and a range
+// that crosses into a unit carries wu less item weight.  Which wu balances the
+// CTAs best depends on the batch: with units a little larger than a share
+// (Mistral-7B GQA, B=16, 6553 kept tokens; 128 units on 148 SMs) one CTA per
+// unit and no split is fastest, with many small units or a ragged batch a
+// small wu is.  So each call takes, from a few candidates, the wu whose cuts
+// minimise a cost model of the slowest CTA: the weight of its items, plus
+// kSegCost for every unit it works on (the end of a segment), plus kSplitCost
+// for every unit it shares with another CTA (partial write, arrival, merge).
+// The two costs were fitted to measured launch times of five batch shapes at
+// boundary weights from 0 to 2^20; with them the model ranks each shape's
+// fastest measured weight first.
+constexpr int kWuCand[] = {128, 256, 512, 896, 1280, 1 << 20};
+constexpr long long kSegCost = 120, kSplitCost = 200;
+
+struct Shape {              // per-sequence state of this call (n_q, r = residual tokens + the new one)
+    int B, Hkv;
+    std::vector<int> nq, r, ibeg;
+};
+
+// Cuts of the work list for boundary weight wu: P, S_max and lo of p.
+void cut(const Shape &s, int wu, int sms, Plan &p) {
+    std::vector<long long> wbeg(s.B + 1, 0);
     long long Wmax = 0;
-    p.max_n = 0;
-    for (int b = 0; b < c->B; ++b) {
-        const int s = ragged ? b : 0;
-        const int r = seq_nres(c, s) + 1, nq = seq_nq(c, s);
-        if (nq + r > p.max_n) p.max_n = nq + r;
-        const long long W = unit_w(nq, r);
+    for (int b = 0; b < s.B; ++b) {
+        const long long W = unit_w(s.nq[b], s.r[b], wu);
         if (W > Wmax) Wmax = W;
-        wbeg[b + 1] = wbeg[b] + (long long)c->Hkv * W;
-        ibeg[b + 1] = ibeg[b] + c->Hkv * unit_items(nq, r);
+        wbeg[b + 1] = wbeg[b] + (long long)s.Hkv * W;
     }
-    const long long Wt = wbeg[c->B];
-    p.P = (int)cta_count(Wt, sm_count(dev));
+    const long long Wt = wbeg[s.B];
+    p.P = (int)cta_count(Wt, sms, wu);
     p.S_max = slots_bound(Wmax, Wt / p.P);
     if (p.S_max > p.P) p.S_max = p.P;
     // first item whose start weight is >= floor(i Wt / P), for each CTA boundary i
@@ -1198,18 +1210,117 @@ Plan plan(const minikv_cache *c, int dev) {
     for (int i = 0; i <= p.P; ++i) {
         const long long w = (long long)((__int128)i * Wt / p.P);
         if (w >= Wt) {
-            p.lo[i] = ibeg[c->B];
+            p.lo[i] = s.ibeg[s.B];
             continue;
         }
         while (wbeg[b + 1] <= w) ++b;
-        const int s = ragged ? b : 0;
-        const int r = seq_nres(c, s) + 1, nq = seq_nq(c, s);
-        const long long W = unit_w(nq, r);
+        const long long W = unit_w(s.nq[b], s.r[b], wu);
         const long long off = w - wbeg[b];
         const int kh = (int)(off / W);
         const long long rem = off - kh * W;
-        p.lo[i] = ibeg[b] + kh * unit_items(nq, r) + item_at(rem, unit_nri(r));
+        p.lo[i] = s.ibeg[b] + kh * unit_items(s.nq[b], s.r[b]) + item_at(rem, unit_nri(s.r[b]), wu);
     }
+}
+
+// Modelled cost of the slowest CTA of a cut (see above).
+long long slowest_cta(const Shape &s, const Plan &p) {
+    long long worst = 0;
+    int b = 0, kh = 0;   // the unit that holds lo[c]
+    for (int c = 0; c < p.P; ++c) {
+        const int x0 = p.lo[c], x1 = p.lo[c + 1];
+        if (x0 >= x1) continue;
+        for (;;) {
+            const int n = unit_items(s.nq[b], s.r[b]);
+            if (x0 < s.ibeg[b] + (kh + 1) * n) break;
+            if (++kh == s.Hkv) {
+                kh = 0;
+                ++b;
+            }
+        }
+        long long cost = 0;
+        for (int bb = b, kk = kh; bb < s.B;) {
+            const int n = unit_items(s.nq[bb], s.r[bb]), nri = unit_nri(s.r[bb]);
+            const int us = s.ibeg[bb] + kk * n, ue = us + n;
+            if (us >= x1) break;
+            const int lo = x0 > us ? x0 : us, hi = x1 < ue ? x1 : ue;
+            int res = (hi < us + nri ? hi : us + nri) - lo;
+            if (res < 0) res = 0;
+            cost += (long long)res * kWR + (long long)(hi - lo - res) * kWP + kSegCost;
+            if (lo > us || hi < ue) cost += kSplitCost;
+            if (++kk == s.Hkv) {
+                kk = 0;
+                ++bb;
+            }
+        }
+        if (cost > worst) worst = cost;
+    }
+    return worst;
+}
+
+// The boundary weight of the cheapest modelled cut; ties go to the smaller
+// weight.  A pure function of the call's state, so the same state always gets
+// the same cuts (a small exact-key cache per host thread saves the search).
+int choose_wu(const Shape &s, int sms, bool uniform) {
+    std::vector<int> key;
+    key.reserve(5 + 2 * s.B);
+    key.push_back(sms);
+    key.push_back(s.Hkv);
+    key.push_back(s.B);
+    key.push_back(uniform ? 1 : 0);
+    for (int b = 0; b < (uniform ? 1 : s.B); ++b) {
+        key.push_back(s.nq[b]);
+        key.push_back(s.r[b]);
+    }
+    thread_local std::map<std::vector<int>, int> memo;
+    const auto it = memo.find(key);
+    if (it != memo.end()) return it->second;
+    int best_wu = kWU;
+    long long best = -1;
+    Plan p;
+    for (const int wu : kWuCand) {
+        cut(s, wu, sms, p);
+        const long long v = slowest_cta(s, p);
+        if (best < 0 || v < best) {
+            best = v;
+            best_wu = wu;
+        }
+    }
+    if (memo.size() >= 256) memo.clear();
+    memo.emplace(std::move(key), best_wu);
+    return best_wu;
+}
+
+Plan plan(const minikv_cache *c, int dev) {
+    Plan p;
+    p.units = c->B * c->Hkv;
+    const int ring = c->R + c->G;
+    if (c->dseq) {
+        // device-state mode: one configuration for every state the cache can hold;
+        // the kernel partitions this step's items itself, at boundary weight kWU
+        const long long Wmax = unit_w(c->cap, ring);
+        p.P = (int)cta_count((long long)p.units * Wmax, sm_count(dev));
+        p.S_max = slots_bound(Wmax, kMinShare);
+        if (p.S_max > p.P) p.S_max = p.P;
+        p.max_n = c->cap + ring;
+        return p;
+    }
+    const bool ragged = c->seq != nullptr;
+    Shape s;
+    s.B = c->B;
+    s.Hkv = c->Hkv;
+    s.nq.resize(c->B);
+    s.r.resize(c->B);
+    s.ibeg.assign(c->B + 1, 0);
+    p.max_n = 0;
+    for (int b = 0; b < c->B; ++b) {
+        const int q = ragged ? b : 0;
+        s.nq[b] = seq_nq(c, q);
+        s.r[b] = seq_nres(c, q) + 1;
+        if (s.nq[b] + s.r[b] > p.max_n) p.max_n = s.nq[b] + s.r[b];
+        s.ibeg[b + 1] = s.ibeg[b] + c->Hkv * unit_items(s.nq[b], s.r[b]);
+    }
+    const int sms = sm_count(dev);
+    cut(s, choose_wu(s, sms, !ragged), sms, p);
     return p;
 }
 
