@@ -959,7 +959,8 @@ __device__ int dev_first_item(const ArgsDev &a, const long long *wbeg, long long
 
 // Device-state mode: read the state, build the table, run the CTA's work.  The
 // CTA that takes the last launch-wide ticket after reading the state writes the
-// next state of every sequence (append; flush G tokens where the ring is full).  A flush that would pass `cap` is not done: the
+// next state of every sequence (append; flush G tokens where the ring is full)
+// once its items are done.  A flush that would pass `cap` is not done: the
 // sequence keeps its state and its status word is set to 1.
 template <bool kMass>
 __global__ void __launch_bounds__(kThreads, 1) decode_dev_kernel(const ArgsDev a) {
@@ -980,8 +981,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_dev_kernel(const ArgsDev a
     }
     __syncthreads();
     // The launch-wide ticket, taken as soon as the state is read (release: this
-    // CTA's reads come before it), by the last warp: the CTA whose ticket is
-    // the last one writes the next state while the table is built.
+    // CTA's reads come before it) by the last thread.  Its value is first looked
+    // at after the CTA's items, so the round trip is off the path to them: the
+    // CTA whose ticket is the last one then writes the next state.
     unsigned ticket = 0;
     if (tid == kThreads - 1) ticket = atom_inc_acq_rel(a.grid_counter, gridDim.x - 1);
     if (tid < 32) {   // exclusive prefix sums of items and weights, 32 sequences per pass
@@ -1026,7 +1028,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_dev_kernel(const ArgsDev a
         for (int cc = tid; cc <= P; cc += kThreads)
             clo[cc] = dev_first_item(a, wbeg, (long long)floor((double)cc * (double)Wt / (double)P));
     }
-    // the last ticket's CTA: every sequence's new state, by its last warp
+    __syncthreads();
+    if ((int)blockIdx.x < dev_tab().P) run_cta<kMass, false>(a, *reinterpret_cast<Smem *>(smem_raw), blockIdx.x);
+    // the last ticket's CTA: every sequence's new state, by its last warp (the
+    // state words kept in shared memory past the CTA's own Smem)
     if (tid >= kThreads - 32 && __shfl_sync(0xffffffffu, ticket, 31) == gridDim.x - 1)
         for (int b = tid - (kThreads - 32); b < B; b += 32) {
             int4 st = make_int4(nq[b], rr[b], rs[b], stw[b]);   // a set status stays set
@@ -1042,8 +1047,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_dev_kernel(const ArgsDev a
             }
             reinterpret_cast<int4 *>(a.dseq)[b] = st;
         }
-    __syncthreads();
-    if ((int)blockIdx.x < dev_tab().P) run_cta<kMass, false>(a, *reinterpret_cast<Smem *>(smem_raw), blockIdx.x);
 }
 
 // mass[unit][t] += sum_h 2^(xs[unit][h][t] - M_h) / L_h for the n_u tokens

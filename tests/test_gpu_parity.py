@@ -47,6 +47,10 @@ def _kv(B, H, N, seed, device=DEV):
     (1, 1, 160 + 128 + 50, 64, 16, 128, 256),
     (1, 2, 0, 32, 128, 32, 64),        # empty
     (3, 2, 32 * 40 + 31, 32, 128, 0, 32 * 40 + 32),   # R = 0
+    (1, 2, 32 * 8 + 40, 32, 32, 32, 320),             # Gv = 32
+    (1, 1, 128 * 3 + 100, 128, 128, 64, 512),         # G = 128: one block per group
+    (4, 8, 32 * 40 + 40, 32, 128, 32, 32 * 41),       # 1280 groups: blocks pack several, double-buffered
+    (2, 8, 64 * 60 + 100, 64, 64, 64, 64 * 61),       # the same at G = 64
 ])
 def test_quant_pack_bitexact(B, H, N, G, Gv, R, cap):
     k, v = _kv(B, H, N, 101 + N)
