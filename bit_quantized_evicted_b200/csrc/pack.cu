@@ -119,11 +119,18 @@ __device__ __forceinline__ float fma_sat(float a, float b, float c) {
     asm("fma.rn.sat.f32 %0, %1, %2, %3;\n" : "=f"(d) : "f"(a), "f"(b), "f"(c));
     return d;
 }
-// w + code(x) * wgt, with code(x) that of quant_code_thr (zero and thresholds
-// of x's channel or block).  w and wgt are small integers (wgt a power of 4,
-// at most 8 codes per sum: below 2^16), so every step is exact.
-__device__ __forceinline__ float add_code(float w, float x, float zero, float c1, float c2, float c3, float wgt) {
-    const float d = __fsub_rn(x, zero);
+// d = fp32(x - zero) for the two fp16 halves of w (low half first): the
+// mixed-precision subtraction widens x exactly and rounds once, as
+// __fsub_rn(fp32(x), zero) does
+__device__ __forceinline__ void sub_h2(uint32_t w, float z0, float z1, float &d0, float &d1) {
+    asm("{\n .reg .f16 l, h;\n mov.b32 {l, h}, %2;\n sub.rn.f32.f16 %0, l, %3;\n sub.rn.f32.f16 %1, h, %4;\n}\n"
+        : "=f"(d0), "=f"(d1) : "r"(w), "f"(z0), "f"(z1));
+}
+// w + code(d) * wgt, with code(d) that of quant_code_thr for d = fp32(x - zero)
+// and the scaled thresholds of x's channel or block.  w and wgt are small
+// integers (wgt a power of 4, at most 8 codes per sum: below 2^16), so every
+// step is exact.
+__device__ __forceinline__ float add_code_d(float w, float d, float c1, float c2, float c3, float wgt) {
     w = fmaf(fma_sat(d, kCmpScale, c1), wgt, w);
     w = fmaf(fma_sat(d, kCmpScale, c2), wgt, w);
     return fmaf(fma_sat(d, kCmpScale, c3), wgt, w);
@@ -204,10 +211,10 @@ __device__ __forceinline__ void pack_keys_tile(const uint16_t *kt, uint32_t *cod
         float hw = kCodeBase;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            float x0, x1;
-            split_h2(w4(v, i), x0, x1);
-            hw = add_code(hw, x0, z[2 * i], t1[2 * i], t2[2 * i], t3[2 * i], (float)(1 << (4 * i)));
-            hw = add_code(hw, x1, z[2 * i + 1], t1[2 * i + 1], t2[2 * i + 1], t3[2 * i + 1], (float)(1 << (4 * i + 2)));
+            float d0, d1;
+            sub_h2(w4(v, i), z[2 * i], z[2 * i + 1], d0, d1);
+            hw = add_code_d(hw, d0, t1[2 * i], t2[2 * i], t3[2 * i], (float)(1 << (4 * i)));
+            hw = add_code_d(hw, d1, t1[2 * i + 1], t2[2 * i + 1], t3[2 * i + 1], (float)(1 << (4 * i + 2)));
         }
         const uint32_t h = code_bits(hw);
         const uint32_t other = __shfl_xor_sync(0xffffffffu, h, 8);
@@ -287,11 +294,11 @@ __device__ __forceinline__ void pack_values_tile(const uint16_t *vt, int Gv, uin
             float c[2] = {kCodeBase, kCodeBase};   // the word's low and high 16 bits (8 channels each)
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-                float x0, x1;
-                split_h2(w[8 * h + i], x0, x1);
+                float d0, d1;
+                sub_h2(w[8 * h + i], zh[h], zh[h], d0, d1);
                 const int j = i & 3;
-                c[i >> 2] = add_code(c[i >> 2], x0, zh[h], t1[h], t2[h], t3[h], (float)(1 << (4 * j)));
-                c[i >> 2] = add_code(c[i >> 2], x1, zh[h], t1[h], t2[h], t3[h], (float)(1 << (4 * j + 2)));
+                c[i >> 2] = add_code_d(c[i >> 2], d0, t1[h], t2[h], t3[h], (float)(1 << (4 * j)));
+                c[i >> 2] = add_code_d(c[i >> 2], d1, t1[h], t2[h], t3[h], (float)(1 << (4 * j + 2)));
             }
             cw[h] = code_bits(c[0]) | (code_bits(c[1]) << 16);
         }
