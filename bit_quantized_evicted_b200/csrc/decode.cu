@@ -1153,6 +1153,7 @@ int seq_rs(const minikv_cache *c, int b) { return c->seq ? c->seq[3 * b + 2] : c
 
 struct Plan {
     int units, P, S_max;
+    int wu;                  // unit-boundary weight of the cut
     int max_n;               // most tokens any unit attends to this step
     std::vector<int> lo;     // host-planned modes: first item of each CTA (P + 1 entries)
 };
@@ -1305,6 +1306,7 @@ Plan plan(const minikv_cache *c, int dev) {
         p.S_max = slots_bound(Wmax, kMinShare);
         if (p.S_max > p.P) p.S_max = p.P;
         p.max_n = c->cap + ring;
+        p.wu = kWU;
         return p;
     }
     const bool ragged = c->seq != nullptr;
@@ -1323,7 +1325,8 @@ Plan plan(const minikv_cache *c, int dev) {
         s.ibeg[b + 1] = s.ibeg[b] + c->Hkv * unit_items(s.nq[b], s.r[b]);
     }
     const int sms = sm_count(dev);
-    cut(s, choose_wu(s, sms, !ragged), sms, p);
+    p.wu = choose_wu(s, sms, !ragged);
+    cut(s, p.wu, sms, p);
     return p;
 }
 
@@ -1361,6 +1364,22 @@ size_t decode_mass_workspace_bytes(int B, int Hq, int Hkv, int max_tokens) {
 }
 
 void decode_set_deterministic(int on) { g_deterministic.store(on ? 1 : 0, std::memory_order_relaxed); }
+
+// The launch the next decode call on this cache state makes: CTAs, boundary
+// weight and (host-planned modes, n_first >= P + 1) each CTA's first item.
+int decode_plan_info(const minikv_cache *c, int *ctas, int *wu, int *first, int n_first) {
+    const int dev = current_device();
+    const Plan p = plan(c, dev < 0 ? 0 : dev);
+    *ctas = p.P;
+    *wu = p.wu;
+    if (first && !c->dseq) {
+        if (n_first < p.P + 1)
+            return fail(MINIKV_ERR_INVALID_ARG, "decode_plan: first_items needs %d entries, %d given", p.P + 1,
+                        n_first);
+        for (int i = 0; i <= p.P; ++i) first[i] = p.lo[i];
+    }
+    return MINIKV_OK;
+}
 
 // Workspace bytes the next decode call on this cache state will use.
 size_t decode_call_workspace_bytes(const minikv_cache *c) {

@@ -38,6 +38,7 @@ int decode_launch(minikv_cache *c, const uint16_t *q, const uint16_t *k_new, con
 size_t decode_workspace_bytes(int B, int Hkv, int max_tokens);
 size_t decode_mass_workspace_bytes(int B, int Hq, int Hkv, int max_tokens);
 void decode_set_deterministic(int on);
+int decode_plan_info(const minikv_cache *c, int *ctas, int *wu, int *first, int n_first);
 
 static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -340,6 +341,17 @@ int minikv_decode_attn_mass(minikv_cache *c, const uint16_t *q, const uint16_t *
 int minikv_set_deterministic(int on) {
     decode_set_deterministic(on);
     return MINIKV_OK;
+}
+
+int minikv_decode_plan(const minikv_cache *c, int *ctas, int *boundary_weight, int *first_items, int n_first) {
+    const int rc = check_cache(c);
+    if (rc) return rc;
+    if (!ctas || !boundary_weight || n_first < 0 || (n_first > 0 && !first_items))
+        return fail(MINIKV_ERR_INVALID_ARG, "decode_plan: null output or negative n_first");
+    if ((size_t)c->B * c->Hkv > 65535) return fail(MINIKV_ERR_UNSUPPORTED, "decode_plan: B*Hkv above 65535");
+    if ((size_t)c->B * c->Hkv * (c->cap / 32 + (c->R + c->G + 4) / 5) >= (1u << 31))
+        return fail(MINIKV_ERR_UNSUPPORTED, "decode_plan: B*Hkv*(cap/32 + (R+G)/5) must stay below 2^31");
+    return decode_plan_info(c, ctas, boundary_weight, n_first > 0 ? first_items : nullptr, n_first);
 }
 
 size_t minikv_workspace_size(int op, int B, int Hq, int Hkv, int T, int D, int W) {

@@ -54,6 +54,7 @@ _SIGS = {
     "minikv_decode_attn_mass": (_I, [ctypes.POINTER(CacheStruct), _P, _P, _P, _I, _F, _P, _P, _P, _Z, _P]),
     "minikv_decode_attn_static": (_I, [ctypes.POINTER(CacheStruct), _P, _P, _P, _I, _F, _P, _P]),
     "minikv_set_deterministic": (_I, [_I]),
+    "minikv_decode_plan": (_I, [ctypes.POINTER(CacheStruct), ctypes.POINTER(_I), ctypes.POINTER(_I), _P, _I]),
     "minikv_workspace_size": (_Z, [_I, _I, _I, _I, _I, _I, _I]),
     "minikv_last_error_string": (ctypes.c_char_p, []),
 }
@@ -363,6 +364,20 @@ def decode_attn_mass(cache: MiniKVCache, q: torch.Tensor, k_new: torch.Tensor, v
         _dev(v_new, torch.float16, "v_new"), Hq, float(sm_scale), _dev(out, torch.float16, "out"),
         _dev(mass, torch.float32, "mass"), _dev(ws, torch.uint8, "ws"), ws.numel(), _stream(stream, q.device)))
     return out
+
+
+def decode_plan(cache) -> tuple:
+    """(CTAs, boundary weight, first item of each CTA's range + the item count)
+    of the next decode call on `cache` (a MiniKVCache or a bound CacheStruct);
+    host logic only.  The list is empty for a device-resident state."""
+    c = cache.c if hasattr(cache, "c") else cache
+    ctas, wu = _I(0), _I(0)
+    _check(lib().minikv_decode_plan(ctypes.byref(c), ctypes.byref(ctas), ctypes.byref(wu), None, 0))
+    if c.dseq:
+        return ctas.value, wu.value, []
+    first = (_I * (ctas.value + 1))()
+    _check(lib().minikv_decode_plan(ctypes.byref(c), ctypes.byref(ctas), ctypes.byref(wu), first, ctas.value + 1))
+    return ctas.value, wu.value, list(first)
 
 
 def set_deterministic(on: bool) -> None:

@@ -357,6 +357,30 @@ MINIKV_API int minikv_decode_attn_static(minikv_cache *c, const uint16_t *q, con
 #define MINIKV_OP_DECODE_ATTN    3
 #define MINIKV_OP_DECODE_ATTN_MASS 4
 
+/*
+ * minikv_decode_plan -- how the next minikv_decode_attn (or _mass, _static)
+ * call on this cache state splits its work.  Host logic only: touches no
+ * device memory and launches nothing; without a GPU it assumes 148 SMs.
+ * The work list: for each (sequence, KV head) unit in order,
+ * ceil((n_res + 1) / 5) residual items of up to 5 fp16 tokens (the new token
+ * included), then n_packed / 32 packed items of 32 tokens.  It is cut into
+ * one contiguous range per CTA at equal steps of a weight: 8 per packed
+ * item, 7 per residual item, plus a boundary weight before each unit's first
+ * item, chosen per call from 128, 256, 512, 896, 1280 and 2^20 by a cost
+ * model of the slowest CTA (2^20 gives one CTA per unit when units are few).
+ *   *ctas: CTAs that take a range (at most one per SM).
+ *   *boundary_weight: the boundary weight of the cut (640 for a cache with
+ *     device-resident state, whose CTAs cut the list themselves on the GPU).
+ *   first_items: if n_first > 0, at least *ctas + 1 entries: the first item of
+ *     each CTA's range, then the number of items.  Not written for a cache
+ *     with device-resident state.
+ * The answer depends only on the cache's shape and state (and the SM count).
+ * Errors: INVALID_ARG (null, bad cache, n_first too small), UNSUPPORTED (as
+ * for minikv_decode_attn: B*Hkv or the item count too large).
+ */
+MINIKV_API int minikv_decode_plan(const minikv_cache *c, int *ctas, int *boundary_weight, int *first_items,
+                                  int n_first);
+
 /* Scratch bytes an op needs.  For MINIKV_OP_DECODE_ATTN and
  * MINIKV_OP_DECODE_ATTN_MASS pass the cache capacity plus R+G as T (the most
  * tokens a step can attend to). */
