@@ -1226,8 +1226,9 @@ void cut(const Shape &s, int wu, int sms, Plan &p) {
     }
 }
 
-// Modelled cost of the slowest CTA of a cut (see above).
-long long slowest_cta(const Shape &s, const Plan &p) {
+// Modelled cost of the slowest CTA of a cut (see above); stops early once it
+// reaches `stop` (a cost that cannot win), if stop >= 0.
+long long slowest_cta(const Shape &s, const Plan &p, long long stop) {
     long long worst = 0;
     int b = 0, kh = 0;   // the unit that holds lo[c]
     for (int c = 0; c < p.P; ++c) {
@@ -1257,14 +1258,18 @@ long long slowest_cta(const Shape &s, const Plan &p) {
             }
         }
         if (cost > worst) worst = cost;
+        if (stop >= 0 && worst >= stop) return worst;
     }
     return worst;
 }
 
 // The boundary weight of the cheapest modelled cut; ties go to the smaller
-// weight.  A pure function of the call's state, so the same state always gets
-// the same cuts (a small exact-key cache per host thread saves the search).
-int choose_wu(const Shape &s, int sms, bool uniform) {
+// weight.  The model is evaluated with each sequence's residual count r moved
+// to the middle of its 32-token bucket (it moves the choice little, and a
+// batch then keeps its weight for up to 32 steps).  A pure function of the
+// call's state, so the same state always gets the same cut; a small cache per
+// host thread, keyed by the bucketed state, saves the search.
+int choose_wu(const Shape &s, int sms, bool uniform, int ring) {
     std::vector<int> key;
     key.reserve(5 + 2 * s.B);
     key.push_back(sms);
@@ -1273,17 +1278,23 @@ int choose_wu(const Shape &s, int sms, bool uniform) {
     key.push_back(uniform ? 1 : 0);
     for (int b = 0; b < (uniform ? 1 : s.B); ++b) {
         key.push_back(s.nq[b]);
-        key.push_back(s.r[b]);
+        key.push_back(s.r[b] >> 5);
     }
     thread_local std::map<std::vector<int>, int> memo;
     const auto it = memo.find(key);
     if (it != memo.end()) return it->second;
+    Shape m = s;   // the bucketed state
+    for (int b = 0; b < s.B; ++b) {
+        const int rc = (s.r[b] >> 5) * 32 + 16;
+        m.r[b] = rc < 1 ? 1 : rc > ring ? ring : rc;
+        m.ibeg[b + 1] = m.ibeg[b] + s.Hkv * unit_items(m.nq[b], m.r[b]);
+    }
     int best_wu = kWU;
     long long best = -1;
     Plan p;
     for (const int wu : kWuCand) {
-        cut(s, wu, sms, p);
-        const long long v = slowest_cta(s, p);
+        cut(m, wu, sms, p);
+        const long long v = slowest_cta(m, p, best);
         if (best < 0 || v < best) {
             best = v;
             best_wu = wu;
@@ -1325,7 +1336,7 @@ Plan plan(const minikv_cache *c, int dev) {
         s.ibeg[b + 1] = s.ibeg[b] + c->Hkv * unit_items(s.nq[b], s.r[b]);
     }
     const int sms = sm_count(dev);
-    p.wu = choose_wu(s, sms, !ragged);
+    p.wu = choose_wu(s, sms, !ragged, ring);
     cut(s, p.wu, sms, p);
     return p;
 }
