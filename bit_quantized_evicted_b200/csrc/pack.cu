@@ -4,7 +4,9 @@
 // sub-channel (per-channel) key quantization and per-token value quantization
 // into a compact layout.  The newest r tokens stay fp16 in the residual ring.
 //
-// Memory-bound: 512 B read and 84 B written per packed token and KV head.
+// Traffic: 512 B read and 84 B written per packed token and KV head.  The
+// group packer streams it at about half the HBM rate; its limit is instruction
+// issue (about 8 instructions per quantized element).
 //
 // G = 32 or 64: pack_groups_kernel.  Each 128-thread block loops over key
 // groups (unit, group) with a stride of the grid, double-buffered: while it
