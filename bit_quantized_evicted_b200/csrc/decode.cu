@@ -8,10 +8,10 @@
 //   * residual items: 5 fp16 residual tokens each (the new token included), and
 //   * packed items:   32 packed tokens each (one slice of one key group).
 // The items of all units are laid end to end and cut, by weight (packed 8,
-// residual 7: their measured costs; 640 more at each unit boundary, for the
-// extra segment end and merge it costs the CTA whose range crosses it), into
-// one contiguous range per SM.  One
-// CTA of 16 warps runs on each SM.  Its warps claim the items of its range one
+// residual 7: their measured costs; plus a boundary weight before each unit,
+// picked per call by a cost model of the slowest CTA, see the host partition
+// below), into one contiguous range per SM.  One CTA of 16 warps runs on each
+// SM that takes a range.  Its warps claim the items of its range one
 // at a time from a shared-memory counter (so warps the scheduler favours simply
 // take more items, and all finish together) and stream them through per-warp
 // 3-stage cp.async pipelines (16 bytes per lane per copy, written to
