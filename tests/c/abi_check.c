@@ -1,7 +1,7 @@
 /*
  * Plain C11 user of libminikv.so: compiles against include/minikv.h alone and
  * exercises the calls that need no GPU (sizes, binding a cache descriptor,
- * ragged state, argument errors).  Exit status 0 = every check held.
+ * ragged state, the decode cut, argument errors).  Exit status 0 = every check held.
  */
 #include <stdint.h>
 #include <stdio.h>
@@ -49,6 +49,17 @@ int main(void)
     CHECK(minikv_decode_attn(&c, p, p, p, 48, 0.1f, o, (void *)p, 1 << 20, NULL) == MINIKV_ERR_UNSUPPORTED);
     CHECK(minikv_decode_attn_mass(&c, p, p, p, 32, 0.1f, o, NULL, (void *)p, 1 << 20, NULL) ==
           MINIKV_ERR_INVALID_ARG);
+
+    /* the decode cut of the Mistral-7B step (6400 packed + 153 residual tokens per unit): one CTA
+     * per unit of 31 residual + 200 packed items, boundary weight 2^20 */
+    c.n_packed = 6400;
+    c.n_res = 153;
+    int ctas = 0, wu = 0, first[160];
+    CHECK(minikv_decode_plan(&c, &ctas, &wu, first, 160) == MINIKV_OK);
+    CHECK(ctas == 128 && wu == (1 << 20) && first[0] == 0 && first[1] == 231 && first[128] == 128 * 231);
+    CHECK(minikv_decode_plan(&c, &ctas, &wu, first, 10) == MINIKV_ERR_INVALID_ARG);
+    c.n_packed = 0;
+    c.n_res = 0;
 
     /* workspace sizes */
     CHECK(minikv_workspace_size(MINIKV_OP_TOPK_EVICT, 1, 32, 32, 4096, 128, 32) == 0);
